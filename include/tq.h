@@ -1,0 +1,182 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) TurboQuant library, libtq.so.
+ *
+ * TurboQuant inner-product quantizer, as summarised on the reference pages
+ * (page titles):
+ *   quant_prune_distill #674 "TurboQuant": the two problem statements
+ *     (MSE-optimal; inner-product-optimal and unbiased); the MSE quantizer
+ *     rotates by a random orthogonal matrix (not Hadamard) and rounds on a
+ *     Lloyd-Max grid; the inner-product quantizer spends b-1 bits on the MSE
+ *     quantizer and 1 bit on a QJL sketch of the residual (random matrix,
+ *     then the sign).
+ *   RecSysChannel #256 "TurboQuant: Redefining AI efficiency with extreme
+ *     compression": normalised vectors times a random matrix have nearly
+ *     N(0, 1/d) coordinates; thresholds are precomputed; a 1-bit
+ *     per-coordinate correction makes the inner-product estimate unbiased.
+ *   seeallochnaya #3476: rotation spreads outliers; 1-D k-means boundaries,
+ *     denser in the centre; residual -> random matrix -> sign; "parallelises
+ *     well on a GPU".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All pointers named d_* are DEVICE pointers of the current CUDA device;
+ *    the caller allocates and owns them.  The library allocates no memory
+ *    and keeps no global state.  `stream` is a cudaStream_t (NULL = the
+ *    legacy default stream); every call is asynchronous on it.
+ *  - Return value: TQ_OK (0) or a negative TQ_ERR_* code; a call that
+ *    returns an error has launched nothing that writes an output, except
+ *    TQ_ERR_CUDA (a launch failed; the outputs are undefined).  Calls never
+ *    abort the process.
+ *  - Supported shapes: d a multiple of 128, 128 <= d <= 4096; b (total bits
+ *    per coordinate) in 1..4; G (groups) >= 1; n, nq >= 0 (0 is a no-op).
+ *  - Groups: group g has its own Pi_g and S_g, drawn from seed + g; arrays
+ *    are group-major: x [G][n][d], codes [G][n][W], norms [G][n],
+ *    queries [G][nq][d], scores [G][nq][n], top-k [G][nq][k].  For KV-cache
+ *    keys a group is a KV head and its nq query heads share it (GQA).
+ *  - W = b * d / 32 uint32 words per code record.  Layout (ours; the pages
+ *    give none): d/32 blocks of b words, block w holding coordinates
+ *    32w..32w+31 (j = coordinate - 32w):
+ *      b = 1: word 0 bit j = z_j
+ *      b = 2: word j/16, bits 2(j%16)+{0,1} = idx_j, z_j
+ *      b = 3: word j/16, bits 2(j%16)+{0,1} = idx_j (2 bits); word 2 bit j = z_j
+ *      b = 4: word j/8,  bits 4(j%8)+{0,1,2,3} = idx_j (3 bits), z_j
+ *    idx_j = Lloyd-Max cell of the rotated coordinate, z_j = [(S r)_j >= 0].
+ *    The two fp32 norms |x| and |r| are stored in separate arrays.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define TQ_OK                  0
+#define TQ_ERR_ARG            -1  /* null pointer, negative size, bad enum   */
+#define TQ_ERR_UNSUPPORTED    -2  /* d not a multiple of 128, b outside 1..4 */
+#define TQ_ERR_WORKSPACE      -3  /* ws_bytes below tq_workspace_bytes()     */
+#define TQ_ERR_CUDA           -4  /* a CUDA launch or API call failed        */
+#define TQ_ERR_DEVICE_TIMEOUT -5  /* a bounded device-side wait gave up      */
+#define TQ_ERR_MISMATCH       -6  /* codebook does not match the call's d/b  */
+
+/* element types of caller inputs */
+#define TQ_F32  0
+#define TQ_BF16 1
+
+/* operation ids for tq_workspace_bytes */
+#define TQ_OP_BUILD   0
+#define TQ_OP_ENCODE  1
+#define TQ_OP_SCORE   2
+#define TQ_OP_TOPK    3
+#define TQ_OP_DECODE  4
+#define TQ_OP_EXACT   5
+
+/* Host-side codebook (quant_prune_distill #674: Lloyd-Max grid for the
+ * target bit width; RecSysChannel #256 item 1: thresholds computed in
+ * advance).  Filled by tq_build_codebook; plain data, caller-owned, may be
+ * copied.  centroids[j] / boundaries[j] are the Lloyd-Max centroids and cell
+ * boundaries of N(0,1) for 2^(b-1) levels, multiplied by 1/sqrt(d) and
+ * rounded to fp32; unused entries are 0.  For b = 1 there are no levels. */
+typedef struct tq_codebook {
+    int32_t  d;            /* vector dimension                              */
+    int32_t  b;            /* total bits per coordinate (index bits b-1 + 1) */
+    int32_t  levels;       /* 2^(b-1), or 0 for b = 1                        */
+    int32_t  groups;       /* G: number of (Pi, S) pairs built               */
+    uint64_t seed;         /* group g uses seed + g                          */
+    float    centroids[8];
+    float    boundaries[8];
+    double   distortion;   /* Lloyd-Max mean squared error for N(0,1)        */
+} tq_codebook_t;
+
+/* Bytes of device workspace an operation needs for the given sizes (0 when
+ * it needs none).  op is a TQ_OP_*; arguments that do not apply are
+ * ignored.  Never fails: returns (size_t)-1 for unsupported shapes. */
+TQ_API size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int nq, int k);
+
+/* Human-readable name of a status code (static string). */
+TQ_API const char *tq_status_str(int status);
+
+/* E0, parameters (once per (d, b, seed, G); not on the timed path).
+ * quant_prune_distill #674: "random orthogonal matrix (not Hadamard)" and
+ * the Lloyd-Max grid; seeallochnaya #3476 step 2 "a random matrix".
+ *  - Pi_g = Q diag(sign R_jj) from the Householder QR (fp64, on the device)
+ *    of the d x d Gaussian matrix G_g[i][j] = N_(seed+g, stream 0)[i*d+j];
+ *    written row-major fp32 to d_Pi[g] so that y = Pi_g x.
+ *  - S_g[i][j] = N_(seed+g, stream 1)[i*d+j] rounded to fp32 -> d_S[g].
+ *  - N_(s, t)[m]: Box-Muller pairs over SplitMix64 stream t of seed s
+ *    (counter form, state mix64(s XOR t*0x9E3779B97F4A7C15)).
+ *  - cb (host) receives the fp32 codebook, computed on the host in fp64.
+ * d_Pi, d_S: [G][d][d] fp32.  d_ws: >= tq_workspace_bytes(TQ_OP_BUILD,...).
+ * Synchronous with respect to the host only in that it returns after
+ * enqueueing; the matrices are ready once `stream` reaches this point. */
+TQ_API int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook_t *cb,
+                      float *d_Pi, float *d_S, void *d_ws, size_t ws_bytes,
+                      void *stream);
+
+/* E1-E6, encode (quant_prune_distill #674 inner-product quantizer;
+ * RecSysChannel #256 caveat 1: normalise, multiply by a random matrix):
+ *   |x|, y = Pi_g x / |x| (y = 0 for x = 0), idx_i = #{j : beta_j <= y_i},
+ *   r = y - c[idx], |r|, z_i = [(S_g r)_i >= 0], packed as above.
+ * d_x: [G][n][d], element type x_dtype (TQ_F32 or TQ_BF16).
+ * d_codes: [G][n][W] uint32; d_xnorm, d_rnorm: [G][n] fp32. */
+TQ_API int tq_encode(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
+              int G, int64_t n, const void *d_x, int x_dtype,
+              uint32_t *d_codes, float *d_xnorm, float *d_rnorm,
+              void *d_ws, size_t ws_bytes, void *stream);
+
+/* S0 + S1, scores (quant_prune_distill #674: inner-product quantization with
+ * an unbiased estimate; comuna.ru "8x faster attention logits"):
+ *   qr = Pi_g q, u = S_g qr,
+ *   s = |x| ( <qr, c[idx]> + |r| sqrt(pi/2)/d <u, 2z - 1> ).
+ * d_q: [G][nq][d] (q_dtype); d_scores: [G][nq][n] fp32 (raw inner-product
+ * estimates, no softmax scaling). */
+TQ_API int tq_score(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
+             int G, int64_t n, const uint32_t *d_codes, const float *d_xnorm,
+             const float *d_rnorm, int nq, const void *d_q, int q_dtype,
+             float *d_scores, void *d_ws, size_t ws_bytes, void *stream);
+
+/* S2, top-k search over the codes (comuna.ru: vector search recall): the k
+ * largest estimated scores per query, ordered by score descending then id
+ * ascending.  1 <= k <= 32 and k <= n.  d_vals: [G][nq][k] fp32;
+ * d_ids: [G][nq][k] int64 (index within the group). */
+TQ_API int tq_topk(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
+            int G, int64_t n, const uint32_t *d_codes, const float *d_xnorm,
+            const float *d_rnorm, int nq, const void *d_q, int q_dtype, int k,
+            float *d_vals, int64_t *d_ids, void *d_ws, size_t ws_bytes,
+            void *stream);
+
+/* Dequantization (quant_prune_distill #674: "inverse rotation and
+ * renormalisation"):  xhat = |x| Pi_g^T (c[idx] + |r| sqrt(pi/2)/d S_g^T (2z-1)).
+ * d_xhat: [G][n][d] fp32.  Support path, not part of the timed step. */
+TQ_API int tq_decode(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
+              int G, int64_t n, const uint32_t *d_codes, const float *d_xnorm,
+              const float *d_rnorm, float *d_xhat, void *d_ws, size_t ws_bytes,
+              void *stream);
+
+/* Unquantized baseline of the attention-logit comparison (comuna.ru:
+ * "4-bit TurboQuant ... vs 32-bit unquantized keys"): exact fp32 logits
+ *   out[g][t][v] = <q[g][t], keys[g][v]>  for fp32 keys [G][n][d] and
+ * queries [G][nq][d] (q_dtype).  No workspace. */
+TQ_API int tq_logits_fp32(int d, int G, int64_t n, const float *d_keys, int nq,
+                   const void *d_q, int q_dtype, float *d_out, void *stream);
+
+/* Exact fp32 inner-product top-k (ground truth for recall@k of the vector
+ * search comparison on the pages), same ordering and shapes as tq_topk;
+ * d_x: [G][n][d] fp32. */
+TQ_API int tq_exact_topk(int d, int G, int64_t n, const float *d_x, int nq,
+                  const void *d_q, int q_dtype, int k, float *d_vals,
+                  int64_t *d_ids, void *d_ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H */

@@ -1,0 +1,45 @@
+// Status strings and workspace sizing of the C ABI.
+#include "tq_internal.cuh"
+
+using namespace tq;
+
+extern "C" const char* tq_status_str(int status) {
+    switch (status) {
+        case TQ_OK: return "ok";
+        case TQ_ERR_ARG: return "invalid argument";
+        case TQ_ERR_UNSUPPORTED: return "unsupported shape (d must be a multiple of 128 in [128, 4096], b in 1..4)";
+        case TQ_ERR_WORKSPACE: return "workspace missing or smaller than tq_workspace_bytes()";
+        case TQ_ERR_CUDA: return "CUDA error";
+        case TQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case TQ_ERR_MISMATCH: return "codebook does not match the call";
+        default: return "unknown status";
+    }
+}
+
+extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int nq, int k) {
+    if (d < kMinD || d > kMaxD || d % 128) return (size_t)-1;
+    if (G < 1 || n < 0 || nq < 0 || k < 0) return (size_t)-1;
+    const size_t dd = (size_t)d * d;
+    const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;
+    const int64_t ntiles = (n + kTopkTile - 1) / kTopkTile;
+    const size_t qbuf = align256((size_t)G * nq * d * 4);
+    const size_t parts = align256((size_t)G * nq * ntiles * k * 4) +
+                         align256((size_t)G * nq * ntiles * k * 8);
+    switch (op) {
+        case TQ_OP_BUILD:
+            return 2 * align256(dd * 8) + 2 * align256((size_t)d * 8);
+        case TQ_OP_ENCODE:
+            if (b < 1 || b > 4) return (size_t)-1;
+            return 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
+        case TQ_OP_SCORE:
+            return 2 * qbuf;
+        case TQ_OP_TOPK:
+            return 2 * qbuf + parts;
+        case TQ_OP_DECODE:
+            return 2 * align256((size_t)chunk * d * 4);
+        case TQ_OP_EXACT:
+            return align256((size_t)nq * ((chunk + 3) & ~int64_t(3)) * 4) + parts;
+        default:
+            return (size_t)-1;
+    }
+}

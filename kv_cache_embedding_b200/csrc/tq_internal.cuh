@@ -1,0 +1,69 @@
+// Internal helpers of libtq (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tq.h"
+
+namespace tq {
+
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ULL;
+constexpr int kMinD = 128;
+constexpr int kMaxD = 4096;
+constexpr int kMaxK = 32;           // largest top-k
+constexpr int kTopkTile = 1024;     // keys per top-k tile (one partial list each)
+constexpr int64_t kEncodeChunk = 65536;  // rows per encode/decode chunk
+
+// Codebook passed to kernels by value (kernel parameter space).
+struct KCodebook {
+    float c[8];
+    float beta[8];
+    int levels;   // 2^(b-1), 0 for b = 1
+};
+
+inline KCodebook make_kcodebook(const tq_codebook_t* cb) {
+    KCodebook k;
+    for (int i = 0; i < 8; ++i) {
+        k.c[i] = cb->centroids[i];
+        k.beta[i] = cb->boundaries[i];
+    }
+    k.levels = cb->levels;
+    return k;
+}
+
+__host__ __device__ inline int words_per_vector(int d, int b) { return d / 32 * b; }
+
+__device__ __forceinline__ float load_f32(const float* p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_f32(const __nv_bfloat16* p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+
+// Strictly better in top-k order: larger value, then smaller id.
+__device__ __forceinline__ bool better(float va, int64_t ia, float vb, int64_t ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline bool valid_db(int d, int b) {
+    return d >= kMinD && d <= kMaxD && d % 128 == 0 && b >= 1 && b <= 4;
+}
+
+}  // namespace tq
+
+#define TQ_TRY_CUDA(expr)                               \
+    do {                                                \
+        cudaError_t tq_e_ = (expr);                     \
+        if (tq_e_ != cudaSuccess) return TQ_ERR_CUDA;   \
+    } while (0)
+
+#define TQ_CHECK_LAUNCH() TQ_TRY_CUDA(cudaPeekAtLastError())
+
+// Entry points of the individual translation units (C++ linkage, internal).
+namespace tq {
+int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const float* B,
+                 bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
+                 cudaStream_t s);
+}

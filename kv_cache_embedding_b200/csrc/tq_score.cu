@@ -1,0 +1,658 @@
+// S0-S2: query transform, scoring over packed codes, top-k; dequantization;
+// the unquantized fp32 logit baseline and the exact fp32 top-k.
+//
+// Pages: quant_prune_distill #674 (inner-product quantization, unbiased
+// estimate; dequantization = inverse rotation and renormalisation);
+// RecSysChannel #256 item 2 (1-bit per-coordinate correction -> unbiased
+// inner products); comuna.ru "Google speeds up LLMs 8x" (attention logits
+// from 4-bit keys vs 32-bit keys; vector-search recall).
+//
+// Estimator (for a record with norms |x|, |r|, cells idx, signs z):
+//   s = |x| ( <qr, c[idx]> + |r| sqrt(pi/2)/d <u, 2z - 1> ),  qr = Pi q, u = S qr.
+#include <algorithm>
+#include <cmath>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+namespace {
+
+constexpr float kSqrtHalfPi = 1.2533141373155002512f;  // sqrt(pi/2)
+
+// Decode coordinate j (0..31) of a block: cell index and sign bit.
+template <int B>
+__device__ __forceinline__ void field(const uint32_t* w, int j, int& cell, uint32_t& z) {
+    if (B == 1) {
+        cell = 0;
+        z = (w[0] >> j) & 1u;
+    } else if (B == 2) {
+        const uint32_t f = (w[j >> 4] >> (2 * (j & 15))) & 3u;
+        cell = (int)(f & 1u);
+        z = f >> 1;
+    } else if (B == 3) {
+        cell = (int)((w[j >> 4] >> (2 * (j & 15))) & 3u);
+        z = (w[2] >> j) & 1u;
+    } else {
+        const uint32_t f = (w[j >> 3] >> (4 * (j & 7))) & 15u;
+        cell = (int)(f & 7u);
+        z = f >> 3;
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void load_block(const uint32_t* __restrict__ rec, int blk,
+                                           uint32_t w[4]) {
+    const uint32_t* p = rec + blk * B;
+    if (B == 4) {
+        const uint4 t = __ldg(reinterpret_cast<const uint4*>(p));
+        w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    } else if (B == 2) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2*>(p));
+        w[0] = t.x; w[1] = t.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < B; ++i) w[i] = __ldg(p + i);
+    }
+}
+
+// Score QC queries (rows of s_qr / s_u in shared memory) against one record.
+template <int B, int QC>
+__device__ __forceinline__ void score_record(const uint32_t* __restrict__ rec, int d,
+                                             const float* s_qr, const float* s_u,
+                                             const float* s_c, float am[QC], float aq[QC]) {
+#pragma unroll
+    for (int q = 0; q < QC; ++q) am[q] = aq[q] = 0.f;
+    for (int blk = 0; blk < d / 32; ++blk) {
+        uint32_t w[4];
+        load_block<B>(rec, blk, w);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            int cell;
+            uint32_t z;
+            field<B>(w, j, cell, z);
+            const float yh = (B == 1) ? 0.f : s_c[cell];
+            const float t = z ? 1.f : -1.f;
+            const int i = blk * 32 + j;
+#pragma unroll
+            for (int q = 0; q < QC; ++q) {
+                if (B != 1) am[q] = fmaf(s_qr[q * d + i], yh, am[q]);
+                aq[q] = fmaf(s_u[q * d + i], t, aq[q]);
+            }
+        }
+    }
+}
+
+__device__ void load_queries(const float* __restrict__ qr, const float* __restrict__ u,
+                             int64_t q0, int qn, int QC, int d, float* s_qr, float* s_u) {
+    for (int e = threadIdx.x; e < QC * d; e += blockDim.x) {
+        const int q = e / d;
+        const float a = (q < qn) ? qr[(q0 + q) * d + (e % d)] : 0.f;
+        const float b = (q < qn) ? u[(q0 + q) * d + (e % d)] : 0.f;
+        s_qr[e] = a;
+        s_u[e] = b;
+    }
+}
+
+// grid: (key blocks of 128, G, query chunks); scores [G][nq][n]
+template <int B, int QC>
+__global__ __launch_bounds__(128) void k_score(const uint32_t* __restrict__ codes,
+                                               const float* __restrict__ xnorm,
+                                               const float* __restrict__ rnorm, int64_t n, int d,
+                                               int nq, const float* __restrict__ qr,
+                                               const float* __restrict__ u, KCodebook cb,
+                                               float* __restrict__ scores) {
+    extern __shared__ __align__(16) float smem[];
+    float* s_qr = smem;
+    float* s_u = smem + QC * d;
+    __shared__ float s_c[8];
+    const int g = blockIdx.y;
+    const int q0 = blockIdx.z * QC;
+    const int qn = min(QC, nq - q0);
+    if (threadIdx.x < 8) s_c[threadIdx.x] = cb.c[threadIdx.x];
+    load_queries(qr, u, (int64_t)g * nq + q0, qn, QC, d, s_qr, s_u);
+    __syncthreads();
+    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= n) return;
+    const int W = words_per_vector(d, B);
+    const int64_t gv = (int64_t)g * n + v;
+    float am[QC], aq[QC];
+    score_record<B, QC>(codes + gv * W, d, s_qr, s_u, s_c, am, aq);
+    const float xn = xnorm[gv];
+    const float kap = kSqrtHalfPi / (float)d * rnorm[gv];
+#pragma unroll
+    for (int q = 0; q < QC; ++q)
+        if (q < qn) scores[((int64_t)g * nq + q0 + q) * n + v] = xn * (am[q] + kap * aq[q]);
+}
+
+// ---- top-k -------------------------------------------------------------
+// Warp-wide selection of the best K of `count` scores in shared memory
+// (element e has id id0 + e); removed/invalid entries hold -inf.
+// Results go to vals/ids[0..K).  Lane 0 writes.
+__device__ void warp_select(float* s, int count, int64_t id0, int K, float* vals, int64_t* ids) {
+    const int lane = threadIdx.x % 32;
+    for (int r = 0; r < K; ++r) {
+        float bv = -INFINITY;
+        int be = -1;
+        for (int e = lane; e < count; e += 32) {
+            const float v = s[e];
+            if (v != -INFINITY && (be < 0 || v > bv)) {  // ascending e: first max wins ties
+                bv = v;
+                be = e;
+            }
+        }
+        int64_t bid = (be < 0) ? INT64_MAX : id0 + be;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int64_t oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+            }
+        }
+        if (lane == 0) {
+            vals[r] = bv;
+            ids[r] = bid;
+        }
+        if (bid != INT64_MAX && (bid - id0) % 32 == lane) s[bid - id0] = -INFINITY;
+        __syncwarp();
+    }
+}
+
+// grid: (tiles of kTopkTile keys, G, query chunks of QC <= 8); 256 threads.
+// Writes the tile's best K per query to part_vals/part_ids
+// [G][nq][ntiles][K].
+template <int B, int QC>
+__global__ __launch_bounds__(256) void k_score_topk_tile(
+    const uint32_t* __restrict__ codes, const float* __restrict__ xnorm,
+    const float* __restrict__ rnorm, int64_t n, int d, int nq, const float* __restrict__ qr,
+    const float* __restrict__ u, KCodebook cb, int K, int ntiles, float* __restrict__ part_vals,
+    int64_t* __restrict__ part_ids) {
+    extern __shared__ __align__(16) float smem[];
+    float* s_qr = smem;
+    float* s_u = smem + QC * d;
+    float* s_sc = smem + 2 * QC * d;  // [QC][kTopkTile]
+    __shared__ float s_c[8];
+    const int g = blockIdx.y;
+    const int q0 = blockIdx.z * QC;
+    const int qn = min(QC, nq - q0);
+    const int64_t t0 = (int64_t)blockIdx.x * kTopkTile;
+    if (threadIdx.x < 8) s_c[threadIdx.x] = cb.c[threadIdx.x];
+    load_queries(qr, u, (int64_t)g * nq + q0, qn, QC, d, s_qr, s_u);
+    __syncthreads();
+    const int W = words_per_vector(d, B);
+    const float k0 = kSqrtHalfPi / (float)d;
+    for (int e = threadIdx.x; e < kTopkTile; e += blockDim.x) {
+        const int64_t v = t0 + e;
+        if (v < n) {
+            const int64_t gv = (int64_t)g * n + v;
+            float am[QC], aq[QC];
+            score_record<B, QC>(codes + gv * W, d, s_qr, s_u, s_c, am, aq);
+            const float xn = xnorm[gv];
+            const float kap = k0 * rnorm[gv];
+#pragma unroll
+            for (int q = 0; q < QC; ++q) s_sc[q * kTopkTile + e] = xn * (am[q] + kap * aq[q]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < QC; ++q) s_sc[q * kTopkTile + e] = -INFINITY;
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x / 32;
+    if (warp < qn) {
+        const int64_t o = (((int64_t)g * nq + q0 + warp) * ntiles + blockIdx.x) * K;
+        warp_select(s_sc + warp * kTopkTile, kTopkTile, t0, K, part_vals + o, part_ids + o);
+    }
+}
+
+// Plain score rows -> per-tile partial top-K (exact search path).
+// grid: (tiles, rows); scores [rows][ncols] with column c having id col0 + c.
+__global__ __launch_bounds__(256) void k_rows_topk_tile(const float* __restrict__ sc, int64_t ld,
+                                                        int64_t ncols, int64_t col0, int K,
+                                                        int ntiles_total, int tile0,
+                                                        float* __restrict__ part_vals,
+                                                        int64_t* __restrict__ part_ids) {
+    __shared__ float s[kTopkTile];
+    const int64_t row = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * kTopkTile;
+    for (int e = threadIdx.x; e < kTopkTile; e += blockDim.x)
+        s[e] = (c0 + e < ncols) ? sc[row * ld + c0 + e] : -INFINITY;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int64_t o = (row * ntiles_total + tile0 + blockIdx.x) * K;
+        warp_select(s, kTopkTile, col0 + c0, K, part_vals + o, part_ids + o);
+    }
+}
+
+// Merge [rows][ntiles][K] partial lists into the final K per row.
+// One block (256 threads) per row; K rounds of block-wide arg-max.
+__global__ __launch_bounds__(256) void k_topk_merge(float* __restrict__ part_vals,
+                                                    int64_t* __restrict__ part_ids, int ntiles,
+                                                    int K, float* __restrict__ vals,
+                                                    int64_t* __restrict__ ids) {
+    __shared__ float s_v[8];
+    __shared__ int64_t s_i[8];
+    __shared__ int64_t s_pos[8];
+    const int64_t row = blockIdx.x;
+    float* pv = part_vals + row * ntiles * K;
+    int64_t* pi = part_ids + row * ntiles * K;
+    const int count = ntiles * K;
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    for (int r = 0; r < K; ++r) {
+        float bv = -INFINITY;
+        int64_t bid = INT64_MAX, bpos = -1;
+        for (int e = threadIdx.x; e < count; e += blockDim.x) {
+            const int64_t id = pi[e];
+            if (id == INT64_MAX) continue;
+            const float v = pv[e];
+            if (better(v, id, bv, bid)) {
+                bv = v;
+                bid = id;
+                bpos = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int64_t oid = __shfl_xor_sync(0xffffffffu, bid, o);
+            const int64_t op = __shfl_xor_sync(0xffffffffu, bpos, o);
+            if (better(ov, oid, bv, bid)) {
+                bv = ov;
+                bid = oid;
+                bpos = op;
+            }
+        }
+        if (lane == 0) {
+            s_v[warp] = bv;
+            s_i[warp] = bid;
+            s_pos[warp] = bpos;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float v = s_v[0];
+            int64_t id = s_i[0], pos = s_pos[0];
+            for (int w = 1; w < 8; ++w)
+                if (better(s_v[w], s_i[w], v, id)) {
+                    v = s_v[w];
+                    id = s_i[w];
+                    pos = s_pos[w];
+                }
+            vals[row * K + r] = v;
+            ids[row * K + r] = id;
+            if (pos >= 0) pi[pos] = INT64_MAX;
+        }
+        __syncthreads();
+    }
+}
+
+// ---- dequantization -------------------------------------------------------
+// T = 2z - 1 (fp32 rows) for the rows of a chunk.
+template <int B>
+__global__ void k_signs(const uint32_t* __restrict__ codes, int64_t rows, int d,
+                        float* __restrict__ T) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= rows * (d / 32)) return;
+    const int64_t row = e / (d / 32);
+    const int blk = (int)(e % (d / 32));
+    uint32_t w[4];
+    load_block<B>(codes + row * words_per_vector(d, B), blk, w);
+    for (int j = 0; j < 32; ++j) {
+        int cell;
+        uint32_t z;
+        field<B>(w, j, cell, z);
+        T[row * d + blk * 32 + j] = z ? 1.f : -1.f;
+    }
+}
+
+// E = c[idx] + |r| sqrt(pi/2)/d * E  (E holds S^T (2z - 1) on entry).
+template <int B>
+__global__ void k_combine(const uint32_t* __restrict__ codes, const float* __restrict__ rnorm,
+                          int64_t rows, int d, KCodebook cb, float* __restrict__ E) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= rows * (d / 32)) return;
+    const int64_t row = e / (d / 32);
+    const int blk = (int)(e % (d / 32));
+    uint32_t w[4];
+    load_block<B>(codes + row * words_per_vector(d, B), blk, w);
+    const float kap = kSqrtHalfPi / (float)d * rnorm[row];
+    for (int j = 0; j < 32; ++j) {
+        int cell;
+        uint32_t z;
+        field<B>(w, j, cell, z);
+        const float yh = (B == 1) ? 0.f : cb.c[cell];
+        float* p = E + row * d + blk * 32 + j;
+        *p = yh + kap * (*p);
+    }
+}
+
+// ---- unquantized fp32 logits ---------------------------------------------
+// 8 lanes per key (4 keys per warp); each lane takes every 8th float4 of the
+// key, fp32 products for QC queries held in shared memory, 3-step reduction.
+template <int QC, typename TQ>
+__global__ __launch_bounds__(256) void k_logits_fp32(const float* __restrict__ keys, int64_t n,
+                                                     int d, int nq, const TQ* __restrict__ q,
+                                                     float* __restrict__ out) {
+    extern __shared__ __align__(16) float s_q[];  // [QC][d]
+    const int g = blockIdx.y;
+    const int q0 = blockIdx.z * QC;
+    const int qn = min(QC, nq - q0);
+    for (int e = threadIdx.x; e < QC * d; e += blockDim.x) {
+        const int qq = e / d;
+        s_q[e] = (qq < qn) ? load_f32(q, ((int64_t)g * nq + q0 + qq) * d + e % d) : 0.f;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x % 32;
+    const int sub = lane % 8;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    for (int64_t base = wid * 4; base < n; base += warps * 4) {
+        const int64_t v = base + lane / 8;
+        float acc[QC];
+#pragma unroll
+        for (int qq = 0; qq < QC; ++qq) acc[qq] = 0.f;
+        if (v < n) {
+            const float4* kr = reinterpret_cast<const float4*>(keys + ((int64_t)g * n + v) * d);
+            for (int f = sub; f < d / 4; f += 8) {
+                const float4 kv = __ldg(kr + f);
+#pragma unroll
+                for (int qq = 0; qq < QC; ++qq) {
+                    const float4 qv = *reinterpret_cast<const float4*>(s_q + qq * d + 4 * f);
+                    acc[qq] = fmaf(kv.x, qv.x, acc[qq]);
+                    acc[qq] = fmaf(kv.y, qv.y, acc[qq]);
+                    acc[qq] = fmaf(kv.z, qv.z, acc[qq]);
+                    acc[qq] = fmaf(kv.w, qv.w, acc[qq]);
+                }
+            }
+        }
+#pragma unroll
+        for (int qq = 0; qq < QC; ++qq) {
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) acc[qq] += __shfl_xor_sync(0xffffffffu, acc[qq], o);
+        }
+        if (v < n && sub < QC) {
+#pragma unroll
+            for (int qq = 0; qq < QC; ++qq)
+                if (qq == sub && qq < qn) out[((int64_t)g * nq + q0 + qq) * n + v] = acc[qq];
+        }
+    }
+}
+
+// ---- helpers ----------------------------------------------------------------
+int score_qc(int d) { return d <= 1536 ? 8 : (d <= 3072 ? 4 : 2); }
+
+template <int B, int QC>
+int launch_score_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
+                   int G, int nq, const float* qr, const float* u, const KCodebook& kc,
+                   float* scores, cudaStream_t s) {
+    const size_t smem = (size_t)2 * QC * d * sizeof(float);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score<B, QC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem));
+    dim3 grid((unsigned)((n + 127) / 128), (unsigned)G, (unsigned)((nq + QC - 1) / QC));
+    k_score<B, QC><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+template <int B>
+int launch_score_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
+                   int G, int nq, const float* qr, const float* u, const KCodebook& kc,
+                   float* scores, cudaStream_t s) {
+    switch (score_qc(d)) {
+        case 8: return launch_score_t<B, 8>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
+        case 4: return launch_score_t<B, 4>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
+        default: return launch_score_t<B, 2>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
+    }
+}
+
+template <int B, int QC>
+int launch_topk_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
+                  int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
+                  int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
+    const size_t smem = ((size_t)2 * QC * d + (size_t)QC * kTopkTile) * sizeof(float);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score_topk_tile<B, QC>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid((unsigned)ntiles, (unsigned)G, (unsigned)((nq + QC - 1) / QC));
+    k_score_topk_tile<B, QC><<<grid, 256, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, K,
+                                                     ntiles, pv, pi);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+template <int B>
+int launch_topk_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
+                  int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
+                  int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
+    switch (score_qc(d)) {
+        case 8:
+            return launch_topk_t<B, 8>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
+        case 4:
+            return launch_topk_t<B, 4>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
+        default:
+            return launch_topk_t<B, 2>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
+    }
+}
+
+// qr = Q Pi^T, u = qr S^T for every group (fp32 SIMT GEMM).
+int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const void* d_q,
+               int q_dtype, float* qr, float* u, cudaStream_t s) {
+    const size_t dd = (size_t)d * d;
+    const size_t esz = (q_dtype == TQ_F32) ? 4 : 2;
+    for (int g = 0; g < G; ++g) {
+        const void* qg = (const char*)d_q + (size_t)g * nq * d * esz;
+        int rc = launch_sgemm(nq, d, d, qg, q_dtype, d, d_Pi + g * dd, true, d,
+                              qr + (size_t)g * nq * d, d, nullptr, 0, s);
+        if (rc) return rc;
+        rc = launch_sgemm(nq, d, d, qr + (size_t)g * nq * d, TQ_F32, d, d_S + g * dd, true, d,
+                          u + (size_t)g * nq * d, d, nullptr, 0, s);
+        if (rc) return rc;
+    }
+    return TQ_OK;
+}
+
+int check_common(const tq_codebook_t* cb, int G, int64_t n, int nq, int q_dtype) {
+    if (!cb || G < 1 || n < 0 || nq < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (!valid_db(cb->d, cb->b)) return TQ_ERR_UNSUPPORTED;
+    if (cb->groups < G) return TQ_ERR_MISMATCH;
+    return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                        int64_t n, const uint32_t* d_codes, const float* d_xnorm,
+                        const float* d_rnorm, int nq, const void* d_q, int q_dtype,
+                        float* d_scores, void* d_ws, size_t ws_bytes, void* stream) {
+    int rc = check_common(cb, G, n, nq, q_dtype);
+    if (rc) return rc;
+    if (n == 0 || nq == 0) return TQ_OK;
+    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_scores) return TQ_ERR_ARG;
+    const int d = cb->d, b = cb->b;
+    if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_SCORE, d, b, G, n, nq, 0))
+        return TQ_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    float* qr = (float*)d_ws;
+    float* u = (float*)((char*)d_ws + align256((size_t)G * nq * d * 4));
+    rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
+    if (rc) return rc;
+    const KCodebook kc = make_kcodebook(cb);
+    switch (b) {
+        case 1: return launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
+        case 2: return launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
+        case 3: return launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
+        default: return launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
+    }
+}
+
+extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                       int64_t n, const uint32_t* d_codes, const float* d_xnorm,
+                       const float* d_rnorm, int nq, const void* d_q, int q_dtype, int k,
+                       float* d_vals, int64_t* d_ids, void* d_ws, size_t ws_bytes,
+                       void* stream) {
+    int rc = check_common(cb, G, n, nq, q_dtype);
+    if (rc) return rc;
+    if (k < 1 || k > kMaxK || (int64_t)k > n) return (n == 0 && nq == 0) ? TQ_OK : TQ_ERR_ARG;
+    if (nq == 0) return TQ_OK;
+    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_vals || !d_ids)
+        return TQ_ERR_ARG;
+    const int d = cb->d, b = cb->b;
+    if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_TOPK, d, b, G, n, nq, k))
+        return TQ_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int ntiles = (int)((n + kTopkTile - 1) / kTopkTile);
+    char* p = (char*)d_ws;
+    float* qr = (float*)p;
+    p += align256((size_t)G * nq * d * 4);
+    float* u = (float*)p;
+    p += align256((size_t)G * nq * d * 4);
+    float* pv = (float*)p;
+    p += align256((size_t)G * nq * ntiles * k * 4);
+    int64_t* pi = (int64_t*)p;
+    rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
+    if (rc) return rc;
+    const KCodebook kc = make_kcodebook(cb);
+    switch (b) {
+        case 1: rc = launch_topk_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
+        case 2: rc = launch_topk_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
+        case 3: rc = launch_topk_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
+        default: rc = launch_topk_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
+    }
+    if (rc) return rc;
+    k_topk_merge<<<(unsigned)(G * nq), 256, 0, s>>>(pv, pi, ntiles, k, d_vals, d_ids);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                         int64_t n, const uint32_t* d_codes, const float* d_xnorm,
+                         const float* d_rnorm, float* d_xhat, void* d_ws, size_t ws_bytes,
+                         void* stream) {
+    int rc = check_common(cb, G, n, 0, TQ_F32);
+    if (rc) return rc;
+    if (n == 0) return TQ_OK;
+    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_xhat) return TQ_ERR_ARG;
+    const int d = cb->d, b = cb->b;
+    if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_DECODE, d, b, G, n, 0, 0))
+        return TQ_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const KCodebook kc = make_kcodebook(cb);
+    const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;
+    float* T = (float*)d_ws;
+    float* E = (float*)((char*)d_ws + align256((size_t)chunk * d * 4));
+    const int W = words_per_vector(d, b);
+    const size_t dd = (size_t)d * d;
+    for (int g = 0; g < G; ++g) {
+        for (int64_t r0 = 0; r0 < n; r0 += chunk) {
+            const int64_t rows = (n - r0) < chunk ? (n - r0) : chunk;
+            const int64_t off = (int64_t)g * n + r0;
+            const uint32_t* cg = d_codes + off * W;
+            const unsigned blocks = (unsigned)((rows * (d / 32) + 255) / 256);
+            switch (b) {
+                case 1: k_signs<1><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                case 2: k_signs<2><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                case 3: k_signs<3><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                default: k_signs<4><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+            }
+            TQ_CHECK_LAUNCH();
+            // E = T S   (E[v][j] = sum_i T[v][i] S[i][j])
+            rc = launch_sgemm((int)rows, d, d, T, TQ_F32, d, d_S + g * dd, false, d, E, d, nullptr,
+                              0, s);
+            if (rc) return rc;
+            switch (b) {
+                case 1: k_combine<1><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                case 2: k_combine<2><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                case 3: k_combine<3><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                default: k_combine<4><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+            }
+            TQ_CHECK_LAUNCH();
+            // xhat = |x| E Pi   (xhat[v][j] = |x_v| sum_i E[v][i] Pi[i][j])
+            rc = launch_sgemm((int)rows, d, d, E, TQ_F32, d, d_Pi + g * dd, false, d,
+                              d_xhat + (size_t)off * d, d, d_xnorm + off, 2, s);
+            if (rc) return rc;
+        }
+    }
+    return TQ_OK;
+}
+
+template <typename TQ>
+static int launch_logits(const float* keys, int64_t n, int d, int G, int nq, const TQ* q,
+                         float* out, cudaStream_t s) {
+    const int QC = nq >= 8 ? 8 : (nq >= 4 ? 4 : (nq >= 2 ? 2 : 1));
+    const size_t smem = (size_t)QC * d * 4;
+    const unsigned bx = (unsigned)std::min<int64_t>((n + 31) / 32, 148 * 16);
+    dim3 grid(bx, (unsigned)G, (unsigned)((nq + QC - 1) / QC));
+#define TQ_LG(QCV)                                                                           \
+    do {                                                                                     \
+        TQ_TRY_CUDA(cudaFuncSetAttribute(k_logits_fp32<QCV, TQ>,                             \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,        \
+                                         (int)smem));                                        \
+        k_logits_fp32<QCV, TQ><<<grid, 256, smem, s>>>(keys, n, d, nq, q, out);              \
+    } while (0)
+    switch (QC) {
+        case 8: TQ_LG(8); break;
+        case 4: TQ_LG(4); break;
+        case 2: TQ_LG(2); break;
+        default: TQ_LG(1); break;
+    }
+#undef TQ_LG
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+extern "C" int tq_logits_fp32(int d, int G, int64_t n, const float* d_keys, int nq,
+                              const void* d_q, int q_dtype, float* d_out, void* stream) {
+    if (G < 1 || n < 0 || nq < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (d < kMinD || d > kMaxD || d % 128) return TQ_ERR_UNSUPPORTED;
+    if (n == 0 || nq == 0) return TQ_OK;
+    if (!d_keys || !d_q || !d_out) return TQ_ERR_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (q_dtype == TQ_F32) return launch_logits<float>(d_keys, n, d, G, nq, (const float*)d_q, d_out, s);
+    return launch_logits<__nv_bfloat16>(d_keys, n, d, G, nq, (const __nv_bfloat16*)d_q, d_out, s);
+}
+
+extern "C" int tq_exact_topk(int d, int G, int64_t n, const float* d_x, int nq, const void* d_q,
+                             int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
+                             size_t ws_bytes, void* stream) {
+    if (G < 1 || n < 0 || nq < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (d < kMinD || d > kMaxD || d % 128) return TQ_ERR_UNSUPPORTED;
+    if (nq == 0) return TQ_OK;
+    if (k < 1 || k > kMaxK || (int64_t)k > n) return TQ_ERR_ARG;
+    if (!d_x || !d_q || !d_vals || !d_ids) return TQ_ERR_ARG;
+    if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_EXACT, d, 1, G, n, nq, k))
+        return TQ_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int ntiles = (int)((n + kTopkTile - 1) / kTopkTile);
+    const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;  // multiple of kTopkTile
+    char* p = (char*)d_ws;
+    float* sc = (float*)p;
+    p += align256((size_t)nq * ((chunk + 3) & ~int64_t(3)) * 4);
+    float* pv = (float*)p;
+    p += align256((size_t)G * nq * ntiles * k * 4);
+    int64_t* pi = (int64_t*)p;
+    const size_t esz = (q_dtype == TQ_F32) ? 4 : 2;
+    for (int g = 0; g < G; ++g) {
+        const void* qg = (const char*)d_q + (size_t)g * nq * d * esz;
+        for (int64_t c0 = 0; c0 < n; c0 += chunk) {
+            const int64_t cols = (n - c0) < chunk ? (n - c0) : chunk;
+            const int64_t ld = (cols + 3) & ~int64_t(3);
+            int rc = launch_sgemm(nq, (int)cols, d, qg, q_dtype, d, d_x + ((size_t)g * n + c0) * d,
+                                  true, d, sc, (int)ld, nullptr, 0, s);
+            if (rc) return rc;
+            const int tiles = (int)((cols + kTopkTile - 1) / kTopkTile);
+            dim3 grid((unsigned)tiles, (unsigned)nq);
+            k_rows_topk_tile<<<grid, 256, 0, s>>>(sc, ld, cols, c0, k, ntiles,
+                                                  (int)(c0 / kTopkTile),
+                                                  pv + (size_t)g * nq * ntiles * k,
+                                                  pi + (size_t)g * nq * ntiles * k);
+            TQ_CHECK_LAUNCH();
+        }
+    }
+    k_topk_merge<<<(unsigned)(G * nq), 256, 0, s>>>(pv, pi, ntiles, k, d_vals, d_ids);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}

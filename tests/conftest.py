@@ -9,3 +9,28 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(scope="session")
+def oracle_lib():
+    from oracle import build as ob
+    return ob.build()
+
+
+@pytest.fixture(scope="session")
+def tq_lib():
+    """Build libtq.so in-tree (no-op when up to date) and return the binding."""
+    from kv_cache_embedding_b200 import build as kb
+    kb.build()
+    import kv_cache_embedding_b200 as tq
+    return tq
+
+
+@pytest.fixture(scope="session")
+def cuda(tq_lib):
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("test marked gpu but no CUDA device is visible")
+    return torch.device("cuda:0")

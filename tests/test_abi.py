@@ -1,0 +1,97 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+include/tq.h declares, sizes workspaces and rejects bad arguments before any
+device work (no GPU needed for these paths)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    return re.findall(r"^TQ_API\s+[\w\s\*]+?\b(tq_\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for must in ("tq_build_codebook", "tq_encode", "tq_score", "tq_topk", "tq_decode",
+                 "tq_workspace_bytes", "tq_status_str"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(tq_lib):
+    lib = C.CDLL(tq_lib.binding.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) == set(tq_lib.binding.EXPORTS)
+
+
+def test_status_strings(tq_lib):
+    B = tq_lib.binding
+    for s in (B.TQ_OK, B.TQ_ERR_ARG, B.TQ_ERR_UNSUPPORTED, B.TQ_ERR_WORKSPACE, B.TQ_ERR_CUDA,
+              B.TQ_ERR_DEVICE_TIMEOUT, B.TQ_ERR_MISMATCH):
+        assert B.tq_status_str(s) and B.tq_status_str(s) != "unknown status"
+    assert B.tq_status_str(12345) == "unknown status"
+
+
+def test_codebook_struct_layout(tq_lib):
+    B = tq_lib.binding
+    assert C.sizeof(B.tq_codebook_t) == 96
+    assert B.tq_codebook_t.seed.offset == 16
+    assert B.tq_codebook_t.distortion.offset == 88
+
+
+def test_workspace_sizes(tq_lib):
+    B = tq_lib.binding
+    big = (1 << 64) - 1
+    assert B.tq_workspace_bytes(B.TQ_OP_BUILD, 128, 4, 1, 0, 0, 0) >= 2 * 128 * 128 * 8
+    assert B.tq_workspace_bytes(B.TQ_OP_ENCODE, 100, 4, 1, 10, 0, 0) == big
+    assert B.tq_workspace_bytes(B.TQ_OP_ENCODE, 128, 5, 1, 10, 0, 0) == big
+    e1 = B.tq_workspace_bytes(B.TQ_OP_ENCODE, 128, 4, 1, 1000, 0, 0)
+    e2 = B.tq_workspace_bytes(B.TQ_OP_ENCODE, 128, 4, 1, 10 ** 7, 0, 0)
+    assert 0 < e1 < e2 and e2 == B.tq_workspace_bytes(B.TQ_OP_ENCODE, 128, 4, 1, 10 ** 8, 0, 0)
+    s = B.tq_workspace_bytes(B.TQ_OP_SCORE, 128, 4, 8, 32768, 4, 0)
+    assert s >= 2 * 8 * 4 * 128 * 4
+    t = B.tq_workspace_bytes(B.TQ_OP_TOPK, 128, 4, 1, 10 ** 6, 1024, 10)
+    assert t >= 1024 * ((10 ** 6 + 1023) // 1024) * 10 * 12
+    assert B.tq_workspace_bytes(99, 128, 4, 1, 1, 1, 1) == big
+
+
+def test_bad_arguments_rejected_without_device_work(tq_lib):
+    B = tq_lib.binding
+    cb = B.tq_codebook_t()
+    lib = B.lib
+    # unsupported shapes: rejected before any CUDA call
+    assert lib.tq_build_codebook(100, 4, 0, 1, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    assert lib.tq_build_codebook(128, 5, 0, 1, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    assert lib.tq_build_codebook(128, 4, 0, 0, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_build_codebook(128, 4, 0, 1, None, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_build_codebook(128, 4, 0, 1, C.byref(cb), 1, 1, 1, 16, None) == B.TQ_ERR_WORKSPACE
+    # a codebook that was never built: d = 0
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    cb.d, cb.b, cb.groups, cb.levels = 128, 4, 1, 8
+    assert lib.tq_encode(C.byref(cb), 1, 1, 2, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_MISMATCH
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, 10, 1, 7, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, -1, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, 10, None, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 8, None) == B.TQ_ERR_WORKSPACE
+    assert lib.tq_encode(C.byref(cb), 1, 1, 1, 0, None, 0, None, None, None, None, 0, None) == B.TQ_OK
+    assert lib.tq_score(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 4, 1, 0, 1, 1, 8, None) == B.TQ_ERR_WORKSPACE
+    assert lib.tq_score(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 0, 1, 0, 1, 1, 8, None) == B.TQ_OK
+    assert lib.tq_topk(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 4, 1, 0, 0, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 4, 1, 0, 11, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk(C.byref(cb), 1, 1, 1, 100, 1, 1, 1, 4, 1, 0, 33, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_decode(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 1, 1, 8, None) == B.TQ_ERR_WORKSPACE
+    assert lib.tq_logits_fp32(96, 1, 10, 1, 1, 1, 0, 1, None) == B.TQ_ERR_UNSUPPORTED
+    assert lib.tq_exact_topk(128, 1, 10, 1, 1, 1, 0, 20, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+
+
+def test_binding_raises_on_error(tq_lib):
+    B = tq_lib.binding
+    cb = B.tq_codebook_t()
+    with pytest.raises(B.TQError) as e:
+        B.tq_encode(cb, 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None)
+    assert e.value.status == B.TQ_ERR_UNSUPPORTED

@@ -1,0 +1,222 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, at sizes the
+oracle finishes in seconds: several tiles and ragged tails, every bit width,
+fp32 and bf16 inputs, GQA groups, edge cases."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import oracle as O
+from tests import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _f64(t):
+    return t.detach().cpu().to(torch.float64).numpy()
+
+
+@pytest.fixture(scope="module")
+def quant(cuda, tq_lib):
+    cache = {}
+
+    def get(d, b, seed=0, groups=1):
+        key = (d, b, seed, groups)
+        if key not in cache:
+            cache[key] = tq_lib.TurboQuant(d, b, seed=seed, groups=groups, device=cuda)
+            torch.cuda.synchronize()
+        return cache[key]
+    return get
+
+
+@pytest.fixture(scope="module")
+def oparams():
+    cache = {}
+
+    def get(d, b, seed):
+        key = (d, b, seed)
+        if key not in cache:
+            cache[key] = O.Params(d, b, seed)
+        return cache[key]
+    return get
+
+
+# ---------------------------------------------------------------- parameters
+@pytest.mark.parametrize("d,b,G", [(128, 4, 2), (128, 2, 1), (1536, 3, 1)])
+def test_parameters_match_oracle(quant, oparams, d, b, G):
+    tq = quant(d, b, 0, G)
+    for g in range(G):
+        P = oparams(d, b, g)
+        pi = _np(tq.Pi[g])
+        diff = pi.view(np.int32).astype(np.int64) - P.Pi.view(np.int32).astype(np.int64)
+        assert np.abs(diff).max() <= 1, "Pi differs by more than one fp32 ulp"
+        assert (diff != 0).mean() < 1e-3
+        S = _np(tq.S[g])
+        sd = S.view(np.int32).astype(np.int64) - P.S.view(np.int32).astype(np.int64)
+        assert np.abs(sd).max() <= 1 and (sd != 0).sum() <= 2
+    c, beta = O.codebook(d, b)
+    np.testing.assert_array_equal(tq.centroids().numpy(), c)
+    np.testing.assert_array_equal(tq.boundaries().numpy(), beta)
+    pi64 = tq.Pi[0].double()
+    assert (pi64.T @ pi64 - torch.eye(d, dtype=torch.float64, device=pi64.device)).abs().max() < 1e-5
+
+
+# ---------------------------------------------------------------- encode
+def _encode_both(quant, oparams, x, d, b, groups=1):
+    """x: CPU tensor [G, n, d]; returns list of (gpu, oracle) per group."""
+    tq = quant(d, b, 0, groups)
+    codes = tq.encode(x.cuda())
+    torch.cuda.synchronize()
+    out = []
+    for g in range(groups):
+        P = oparams(d, b, g)
+        ora = O.encode(P, x[g].to(torch.float64).numpy(), diagnostics=True)
+        gpu = (_np(codes.codes[g]).view(np.uint32), _np(codes.xnorm[g]), _np(codes.rnorm[g]))
+        out.append((gpu, ora, P))
+    return out
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_encode_tiny_config(quant, oparams, b):
+    """4096 x 128 fp32 rows, norms U[0.5, 2] (the small workload)."""
+    x = synth.gaussian_rows(4096, 128, seed=1)[None]
+    for gpu, ora, P in _encode_both(quant, oparams, x, 128, b):
+        rep = PT.compare_encode(128, b, P.beta, gpu, ora)
+        assert rep["codes_identical_fraction"] > 0.98, rep
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_encode_kv_bf16_ragged_groups(quant, oparams, b):
+    """bf16 keys with x20 outlier channels, 2 KV heads, a ragged row count."""
+    x = synth.kv_keys(2, 3001, 128, seed=1)
+    for gpu, ora, P in _encode_both(quant, oparams, x, 128, b, groups=2):
+        PT.compare_encode(128, b, P.beta, gpu, ora)
+
+
+@pytest.mark.parametrize("d,b", [(1536, 2), (1536, 4), (3072, 3)])
+def test_encode_large_dims(quant, oparams, d, b):
+    x = synth.gaussian_rows(257, d, seed=2, unit=True)[None]
+    for gpu, ora, P in _encode_both(quant, oparams, x, d, b):
+        PT.compare_encode(d, b, P.beta, gpu, ora)
+
+
+def test_encode_edge_rows(quant, oparams):
+    d, b = 128, 4
+    x = synth.gaussian_rows(40, d, seed=3)
+    x[5] = 0.0                 # zero vector
+    x[6] = 1e-30               # denormal-scale row
+    x[7] = 1e30 / math.sqrt(d)  # very large row
+    x[8, :] = 0.0
+    x[8, 17] = 2.0              # axis-aligned row
+    for gpu, ora, P in _encode_both(quant, oparams, x[None], d, b):
+        PT.compare_encode(d, b, P.beta, gpu, ora, bound_flags=False)
+    tq = quant(d, b)
+    one = tq.encode(x[:1].cuda()[None])
+    empty = tq.encode(x[:0].cuda()[None])
+    torch.cuda.synchronize()
+    assert one.codes.shape == (1, 1, 16) and empty.codes.shape == (1, 0, 16)
+
+
+# ---------------------------------------------------------------- score / top-k / decode
+def _oracle_records(oparams, x, d, b, seed=0):
+    P = oparams(d, b, seed)
+    codes, xn, rn = O.encode(P, x.to(torch.float64).numpy())
+    return P, codes, xn, rn
+
+
+def _to_codes(tq_lib, codes, xn, rn, device):
+    return tq_lib.Codes(torch.from_numpy(codes.view(np.int32)).to(device)[None],
+                        torch.from_numpy(xn).to(device)[None],
+                        torch.from_numpy(rn).to(device)[None])
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_score_tiny_config(quant, oparams, tq_lib, cuda, b):
+    d = 128
+    x = synth.gaussian_rows(4096, d, seed=1)
+    q = synth.gaussian_rows(64, d, seed=2, norm_range=None)
+    P, codes, xn, rn = _oracle_records(oparams, x, d, b)
+    s_ora = O.score(P, codes, xn, rn, q.numpy())
+    tq = quant(d, b)
+    s_gpu = _np(tq.score(_to_codes(tq_lib, codes, xn, rn, cuda), q.cuda()[None])[0])
+    PT.compare_scores(s_gpu, s_ora, np.linalg.norm(_f64(q), axis=1), xn.astype(np.float64))
+
+
+def test_score_gqa_bf16_groups(quant, oparams, tq_lib, cuda):
+    d, b, G = 128, 4, 2
+    keys = synth.kv_keys(G, 1500, d, seed=1)
+    qs = synth.kv_queries(2 * G, G, d, seed=2)  # [G, 2, d]
+    tq = quant(d, b, 0, G)
+    recs = [_oracle_records(oparams, keys[g], d, b, seed=g) for g in range(G)]
+    codes = tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[1].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[3]) for r in recs]).to(cuda))
+    s_gpu = _np(tq.score(codes, qs.cuda()))
+    for g in range(G):
+        P, c, xn, rn = recs[g]
+        s_ora = O.score(P, c, xn, rn, _f64(qs[g]))
+        PT.compare_scores(s_gpu[g], s_ora, np.linalg.norm(_f64(qs[g]), axis=1), xn.astype(np.float64))
+
+
+@pytest.mark.parametrize("n,k,nq", [(4096, 10, 17), (2500, 1, 3), (2500, 32, 3), (33, 32, 2)])
+def test_topk(quant, oparams, tq_lib, cuda, n, k, nq):
+    d, b = 128, 4
+    x = synth.gaussian_rows(n, d, seed=4)
+    q = synth.gaussian_rows(nq, d, seed=5, norm_range=None)
+    P, codes, xn, rn = _oracle_records(oparams, x, d, b)
+    s_ora = O.score(P, codes, xn, rn, q.numpy())
+    tq = quant(d, b)
+    vals, ids = tq.topk(_to_codes(tq_lib, codes, xn, rn, cuda), q.cuda()[None], k)
+    PT.compare_topk(_np(vals[0]), _np(ids[0]), s_ora, k, np.linalg.norm(_f64(q), axis=1),
+                    float(xn.max()))
+
+
+@pytest.mark.parametrize("b", [1, 3, 4])
+def test_decode(quant, oparams, tq_lib, cuda, b):
+    d = 128
+    x = synth.gaussian_rows(700, d, seed=6)
+    P, codes, xn, rn = _oracle_records(oparams, x, d, b)
+    ref = O.decode(P, codes, xn, rn)
+    got = _np(quant(d, b).decode(_to_codes(tq_lib, codes, xn, rn, cuda))[0]).astype(np.float64)
+    err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() <= 1e-4, err.max()
+
+
+def test_logits_fp32(tq_lib, cuda):
+    G, n, d = 2, 3000, 128
+    keys = synth.gaussian_rows(G * n, d, seed=7, norm_range=None).reshape(G, n, d)
+    q = synth.kv_queries(8, G, d, seed=8).float()
+    out = _np(tq_lib.logits_fp32(keys.cuda(), q.cuda()))
+    ref = np.einsum("gqd,gnd->gqn", _f64(q), _f64(keys))
+    tol = 1e-5 * np.linalg.norm(_f64(q), axis=2)[:, :, None] * np.linalg.norm(_f64(keys), axis=2)[:, None, :]
+    assert np.all(np.abs(out - ref) <= tol)
+
+
+def test_exact_topk(tq_lib, cuda):
+    n, d, nq, k = 5000, 256, 7, 10
+    x = synth.gaussian_rows(n, d, seed=9, unit=True)
+    q = synth.gaussian_rows(nq, d, seed=10, unit=True)
+    vals, ids = tq_lib.exact_topk(x.cuda()[None], q.cuda()[None], k)
+    ex = O.exact_scores(_f64(x), _f64(q))
+    PT.compare_topk(_np(vals[0]), _np(ids[0]), ex, k, np.ones(nq), 1.0)
+
+
+def test_errors_on_device(quant, tq_lib, cuda):
+    tq = quant(128, 4)
+    B = tq_lib.binding
+    x = torch.zeros(1, 10, 128, device=cuda)
+    with pytest.raises(B.TQError) as e:
+        B.tq_encode(tq.cb, tq.Pi.data_ptr(), tq.S.data_ptr(), 1, 10, x.data_ptr(), B.TQ_F32,
+                    x.data_ptr(), x.data_ptr(), x.data_ptr(), x.data_ptr(), 16,
+                    torch.cuda.current_stream().cuda_stream)
+    assert e.value.status == B.TQ_ERR_WORKSPACE
+    with pytest.raises(ValueError):
+        tq.encode(torch.zeros(10, 64, device=cuda))
+    torch.cuda.synchronize()
