@@ -1,0 +1,484 @@
+"""Benchmark of the TurboQuant hot path on B200: encode -> score -> top-k.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config kv|decode|tiny|search|larged]
+                    [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of synthetic input:
+tq_encode of every vector, tq_score of the queries against all codes and
+tq_topk (top-10) for the same queries.  Default workload ("kv"): KV-cache keys
+bf16 [8 KV heads, 32768 tokens, 128], b = 4, with 4 decode query heads per KV
+head (GQA 4:1, 32 query heads).  Inputs sit in HBM before the timed region;
+L2 (126 MB) is flushed by writing a 256 MB buffer between timed steps.
+
+Multi-GPU (torchrun, one rank per GPU): weak scaling -- every rank encodes and
+scores its own independent batch (the vectors are independent problems, so
+there is no data-path collective); the time is the max over ranks.
+
+--impl reference times the plain CPU oracle on the host cores on a bounded
+sample of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "tq_encode Mvec/s and tq_score scores/s over packed codes; HBM GB/s vs B200 peak"
+
+CONFIGS = {
+    # name: G groups, n vectors/group, d, b, input kind, queries per group, k
+    "kv": dict(G=8, n=32768, d=128, b=4, x="kv", nq=4, q="kv", k=10, score=True, topk=True,
+               desc="KV keys bf16 [1,8,32768,128] (4 outlier channels x20 per head), b=4; "
+                    "decode queries bf16 32 heads GQA 4:1"),
+    "decode": dict(G=8, n=131072, d=128, b=4, x="kv", nq=4, q="kv", k=10, score=True, topk=True,
+                   desc="decode attention logits, Llama-3.1-8B-shaped: 32 q heads / 8 KV heads, "
+                        "head_dim 128, context 131072, bf16, b=4"),
+    "tiny": dict(G=1, n=4096, d=128, b=4, x="rows", nq=64, q="gauss", k=10, score=True, topk=True,
+                 desc="tiny: 4096 x 128 fp32 rows (norms U[0.5,2]), 64 queries, b=4"),
+    "search": dict(G=1, n=1_000_000, d=1536, b=4, x="unit", nq=1024, q="unit", k=10, score=False,
+                   topk=True, desc="embedding search: 1e6 x 1536 fp32 unit rows, 1024 queries, "
+                                   "b=4, top-10"),
+    "larged": dict(G=1, n=1_000_000, d=3072, b=4, x="rows", nq=256, q="gauss", k=10, score=True,
+                   topk=True, desc="large-d: 1e6 x 3072 fp32 rows (norms U[0.5,2]), 256 queries, "
+                                   "b=4"),
+}
+
+FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 CUDA-core peak at max SM clock
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sus=p.get("bf16_tflops_sustained", p["bf16_tflops"]), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------- inputs
+def make_inputs(cfg, device, seed_offset=0, max_rows=None):
+    import synth
+    G, n, d, nq = cfg["G"], cfg["n"], cfg["d"], cfg["nq"]
+    if max_rows is not None and n > max_rows:
+        G, n = 1, max_rows
+    s = 1 + 100 * seed_offset
+    if cfg["x"] == "kv":
+        x = synth.kv_keys(G, n, d, seed=s, device=device)
+    elif cfg["x"] == "unit":
+        x = synth.gaussian_rows(G * n, d, seed=s, device=device, unit=True).reshape(G, n, d)
+    else:
+        x = synth.gaussian_rows(G * n, d, seed=s, device=device).reshape(G, n, d)
+    if cfg["q"] == "kv":
+        q = synth.kv_queries(G * nq, G, d, seed=s + 1, device=device, key_seed=s)
+    elif cfg["q"] == "unit":
+        q = synth.gaussian_rows(G * nq, d, seed=s + 1, device=device, unit=True).reshape(G, nq, d)
+    else:
+        q = synth.gaussian_rows(G * nq, d, seed=s + 1, device=device,
+                                norm_range=None).reshape(G, nq, d)
+    return x.contiguous(), q.contiguous()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling every 50 ms in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.t:
+                self.t.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [r for (ts, r) in self.rows if t0 <= ts <= t1 and len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- our arm
+class Step:
+    """One pass of the hot path with preallocated outputs and workspaces."""
+
+    def __init__(self, tq, cfg, x, q):
+        import kv_cache_embedding_b200 as K
+        self.K = K
+        self.cfg = cfg
+        self.tq = tq
+        self.x, self.q = x, q
+        G, n, d, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["nq"], cfg["k"]
+        dev = x.device
+        self.codes = K.Codes(torch.empty(G, n, tq.words, dtype=torch.int32, device=dev),
+                             torch.empty(G, n, dtype=torch.float32, device=dev),
+                             torch.empty(G, n, dtype=torch.float32, device=dev))
+        self.scores = torch.empty(G, nq, n, dtype=torch.float32, device=dev) if cfg["score"] else None
+        self.topk = (torch.empty(G, nq, k, dtype=torch.float32, device=dev),
+                     torch.empty(G, nq, k, dtype=torch.int64, device=dev)) if cfg["topk"] else None
+        B = K.binding
+        need = max(B.tq_workspace_bytes(B.TQ_OP_ENCODE, d, cfg["b"], G, n, nq, k),
+                   B.tq_workspace_bytes(B.TQ_OP_SCORE, d, cfg["b"], G, n, nq, k),
+                   B.tq_workspace_bytes(B.TQ_OP_TOPK, d, cfg["b"], G, n, nq, k))
+        tq.ws.get(need)
+        self.ev = None
+
+    def run(self, events=None):
+        """events: optional list of 4 CUDA events recorded between the calls."""
+        tq = self.tq
+        if events:
+            events[0].record()
+        tq.encode(self.x, out=self.codes)
+        if events:
+            events[1].record()
+        if self.scores is not None:
+            tq.score(self.codes, self.q, out=self.scores)
+        if events:
+            events[2].record()
+        if self.topk is not None:
+            tq.topk(self.codes, self.q, self.cfg["k"], out=self.topk)
+        if events:
+            events[3].record()
+
+
+def count_launches(step):
+    """Kernels launched by one step, counted with the CUDA profiler (CUPTI)."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step.run()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type.name == "CUDA"
+                 and not e.name.startswith(("Memcpy", "Memset", "cudaMem"))]
+        ours = [nm.replace("(anonymous namespace)::", "") for nm in names if "tq::" in nm]
+        return len(ours), sorted({nm.split("(")[0] for nm in ours})
+    except Exception as e:  # profiler unavailable
+        return None, [f"profiler unavailable: {e}"]
+
+
+def alg_bytes_flops(cfg):
+    G, n, d, b, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
+    esz = 2 if cfg["x"] == "kv" else 4
+    rec = b * d // 8 + 8
+    enc_bytes = G * n * (d * esz + rec)
+    enc_flops = 4.0 * d * d * G * n
+    score_bytes = G * n * rec + G * nq * n * 4
+    score_flops = 4.0 * d * G * n * nq
+    topk_bytes = G * n * rec + G * nq * k * 12
+    return dict(enc_bytes=enc_bytes, enc_flops=enc_flops, score_bytes=score_bytes,
+                score_flops=score_flops, topk_bytes=topk_bytes, rec=rec)
+
+
+def run_ours(args, cfg, rank, world, dist):
+    import kv_cache_embedding_b200 as K
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    x, q = make_inputs(cfg, dev, seed_offset=rank)
+    tq = K.TurboQuant(cfg["d"], cfg["b"], seed=0, groups=cfg["G"], device=dev)
+    step = Step(tq, cfg, x, q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    nlaunch, kernel_names = count_launches(step) if not args.no_count else (None, [])
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.2)
+    tw = time.time()  # clocks are summarised over warm-up + timed steps (GPU under load)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step.run(evs[i])
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    t1 = time.time()
+    time.sleep(0.3)
+    sampler.stop()
+    enc = [e[0].elapsed_time(e[1]) for e in evs]
+    sco = [e[1].elapsed_time(e[2]) for e in evs]
+    tpk = [e[2].elapsed_time(e[3]) for e in evs]
+    tot_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    if dist:
+        t = torch.tensor([tot_ms, sum(enc), sum(sco), sum(tpk)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        tot_ms, se, ss, st = t.tolist()
+    else:
+        se, ss, st = sum(enc), sum(sco), sum(tpk)
+    K_ = args.steps
+    ms_step = tot_ms / K_
+    units = cfg["G"] * cfg["n"] * world
+    value = units * K_ / (tot_ms / 1e3) / 1e6
+
+    # e2e: host (pinned) inputs -> device, the same path through the public API,
+    # results back to pinned host buffers, every step.
+    xh = x.cpu().pin_memory()
+    qh = q.cpu().pin_memory()
+    xd = torch.empty_like(x)
+    qd = torch.empty_like(q)
+    ch = torch.empty(step.codes.codes.shape, dtype=torch.int32).pin_memory()
+    xnh = torch.empty(step.codes.xnorm.shape).pin_memory()
+    rnh = torch.empty(step.codes.rnorm.shape).pin_memory()
+    sh = torch.empty(step.scores.shape).pin_memory() if step.scores is not None else None
+    tvh = torch.empty(step.topk[0].shape).pin_memory() if step.topk is not None else None
+    tih = torch.empty(step.topk[1].shape, dtype=torch.int64).pin_memory() if step.topk is not None else None
+    e2e_step = Step(tq, cfg, xd, qd)
+    e2e_step.codes, e2e_step.scores, e2e_step.topk = step.codes, step.scores, step.topk
+
+    def e2e_once():
+        xd.copy_(xh, non_blocking=True)
+        qd.copy_(qh, non_blocking=True)
+        e2e_step.run()
+        ch.copy_(step.codes.codes, non_blocking=True)
+        xnh.copy_(step.codes.xnorm, non_blocking=True)
+        rnh.copy_(step.codes.rnorm, non_blocking=True)
+        if sh is not None:
+            sh.copy_(step.scores, non_blocking=True)
+        if tvh is not None:
+            tvh.copy_(step.topk[0], non_blocking=True)
+            tih.copy_(step.topk[1], non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_once()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    if dist:
+        dist.barrier()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_once()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    h2d = xh.numel() * xh.element_size() + qh.numel() * qh.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in (ch, xnh, rnh, sh, tvh, tih) if t is not None)
+
+    ab = alg_bytes_flops(cfg)
+    pk = peaks()
+    enc_ms = se / K_
+    score_ms = ss / K_ if cfg["score"] else None
+    topk_ms = st / K_ if cfg["topk"] else None
+    # dominant kernel: the encode call (rotation + QJL contractions on CUDA cores)
+    ach = ab["enc_flops"] / (enc_ms / 1e3) / 1e12
+    roofline = {"bound": "alu", "achieved": round(ach, 3), "peak": round(FFMA_PEAK_TFLOPS, 1),
+                "unit": "TFLOP/s", "frac": round(ach / FFMA_PEAK_TFLOPS, 4), "traffic": None,
+                "kernel": "tq_encode (sgemm rotation + QJL projection, fp32 FFMA)",
+                "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+    out = {
+        "metric": METRIC, "value": round(value, 4), "unit": "Mvec/s", "n_gpus": world,
+        "steps": K_, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded; shapes of the pages' KV-cache / embedding workloads)",
+        "config": {"workload": f"{args.config}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
+                   "d": cfg["d"], "b": cfg["b"], "queries_per_group": cfg["nq"], "k": cfg["k"],
+                   "l2": "flushed (256 MB write) between timed steps",
+                   "parallelism": f"dp{world} (independent batches per GPU)"},
+        "encode": {"ms": round(enc_ms, 5),
+                   "mvec_s": round(cfg["G"] * cfg["n"] / enc_ms / 1e3, 3),
+                   "gbs": round(ab["enc_bytes"] / enc_ms / 1e6, 2),
+                   "hbm_frac": round(ab["enc_bytes"] / enc_ms / 1e6 / pk["hbm"], 4)},
+        "roofline": roofline,
+        "e2e": {"value": round(units / e2e_ms / 1e3, 4), "unit": "Mvec/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": (nlaunch * K_) if nlaunch is not None else None,
+        "gpu_launches_per_step": nlaunch,
+        "kernels": kernel_names,
+        "clocks": sampler.summary(tw, t1),
+        "peaks": pk,
+    }
+    if score_ms is not None:
+        sg = ab["score_bytes"] / score_ms / 1e6
+        out["score"] = {"ms": round(score_ms, 5),
+                        "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / score_ms * 1e3, 1),
+                        "gbs": round(sg, 2), "hbm_frac": round(sg / pk["hbm"], 4)}
+    if topk_ms is not None:
+        out["topk"] = {"ms": round(topk_ms, 5),
+                       "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / topk_ms * 1e3, 1)}
+    if args.config == "decode" and rank == 0:
+        out["fp32_baseline"] = fp32_baseline(cfg, x, q, flush, args)
+    return out
+
+
+def fp32_baseline(cfg, x, q, flush, args):
+    """Unquantized fp32 keys: logits kernel time vs tq_score on packed codes."""
+    import kv_cache_embedding_b200 as K
+    keys = x.float()
+    out = torch.empty(cfg["G"], cfg["nq"], cfg["n"], dtype=torch.float32, device=x.device)
+    for _ in range(3):
+        K.logits_fp32(keys, q, out)
+    ts = []
+    for _ in range(max(3, min(args.steps, 50))):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        K.logits_fp32(keys, q, out)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = sum(ts) / len(ts)
+    byts = keys.numel() * 4 + out.numel() * 4
+    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1)}
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample(cfg, target_s=10.0, max_units=None):
+    """Run the oracle's encode -> score -> top-k on a bounded sample of the
+    workload; returns (vectors, seconds, description)."""
+    import numpy as np
+    from oracle import oracle as O
+    G, n, d, b, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
+    x, q = make_inputs(cfg, "cpu", max_rows=65536)
+    n = min(n, x.shape[1])
+    params = O.Params(d, b, 0)  # one group's parameters (built outside the timing)
+
+    def run(rows):
+        xs = x[0, :rows].to(torch.float64).numpy()
+        qs = q[0].to(torch.float64).numpy()
+        t = time.perf_counter()
+        codes, xn, rn = O.encode(params, xs)
+        s = O.score(params, codes, xn, rn, qs)
+        O.topk(s, min(k, rows))
+        return time.perf_counter() - t
+
+    rows = min(n, 256)
+    dt = run(rows)
+    cap = max_units or n
+    while dt < target_s / 4 and rows < min(n, cap):
+        rows = min(n, cap, rows * 4)
+        dt = run(rows)
+    return rows, dt, (f"{rows} of the {G * n} vectors (group 0), oracle encode + score of "
+                      f"{nq} queries + top-{k}, extrapolated per vector")
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    steps = []
+    for i in range(args.warmup + args.steps):
+        rows, dt, desc = oracle_sample(cfg, target_s=max(0.5, 8.0 / max(args.steps, 1)))
+        if i >= args.warmup:
+            steps.append((rows, dt))
+    rows = sum(r for r, _ in steps)
+    secs = sum(t for _, t in steps)
+    value = rows / secs / 1e6
+    cores = int(os.environ.get("OMP_NUM_THREADS", cpu_cores()))
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mvec/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / len(steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.config}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
+                   "d": cfg["d"], "b": cfg["b"]},
+        "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "Mvec/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="kv", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-count", action="store_true",
+                    help="skip the profiler-based launch count (for runs under ncu)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)))
+        return 0
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as td
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = td
+    out = run_ours(args, cfg, rank, world, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows, dt, desc = oracle_sample(cfg, target_s=10.0)
+        out["cpu_baseline"] = {"value": rows / dt / 1e6, "unit": "Mvec/s",
+                               "cores": int(os.environ.get("OMP_NUM_THREADS", cpu_cores())),
+                               "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(out))
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
