@@ -67,6 +67,8 @@ extern "C" {
 #define TQ_ERR_CUDA           -4  /* a CUDA launch or API call failed        */
 #define TQ_ERR_DEVICE_TIMEOUT -5  /* a bounded device-side wait gave up      */
 #define TQ_ERR_MISMATCH       -6  /* codebook does not match the call's d/b  */
+#define TQ_ERR_SCRATCH_LIMIT  -7  /* tq_topk_noalloc: sizes need more scratch
+                                     than TQ_NOALLOC_SCRATCH_BYTES            */
 
 /* element types of caller inputs */
 #define TQ_F32  0
@@ -175,6 +177,39 @@ TQ_API int tq_logits_fp32(int d, int G, int64_t n, const float *d_keys, int nq,
 TQ_API int tq_exact_topk(int d, int G, int64_t n, const float *d_x, int nq,
                   const void *d_q, int q_dtype, int k, float *d_vals,
                   int64_t *d_ids, void *d_ws, size_t ws_bytes, void *stream);
+
+/* Top-k without a caller workspace, for callers that cannot allocate device
+ * memory.  The pages have no counterpart of this entry point; it exists for
+ * the deployment, not for the method.
+ *
+ * Some callers of a KV-cache or vector-search library cannot call cudaMalloc
+ * (or any allocator) at the point where they search: serving engines that
+ * hand all device memory to their own pool at start-up and forbid libraries
+ * from taking more, plugins that run inside another runtime's stream without
+ * access to its allocator, and real-time paths where an allocation may block
+ * on device synchronisation.  They still pass inputs and outputs; the scratch
+ * that tq_topk would take from d_ws (transformed queries, per-tile candidate
+ * lists) comes from one static device array of TQ_NOALLOC_SCRATCH_BYTES
+ * (8 MiB) inside libtq, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ * Same arguments, results, ordering and errors as tq_topk, without d_ws and
+ * ws_bytes.  Returns TQ_ERR_SCRATCH_LIMIT, having launched nothing, when
+ * tq_workspace_bytes(TQ_OP_TOPK, d, b, G, n, nq, k) exceeds the array (for
+ * d = 128, b = 4: e.g. 8 KV heads x 4 query heads x 131072 tokens, k = 10 fits).
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  It allocates nothing: no cudaMalloc, cudaFree
+ * or allocating library routine.  Every call on a device shares the one
+ * array, which keeps the last call's contents (each call overwrites all of
+ * the scratch it reads, nothing relies on it starting at zero): calls that
+ * overlap on the GPU (different streams, or host threads) race on it and
+ * must be serialised by the caller. */
+#define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+TQ_API int tq_topk_noalloc(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
+                           int G, int64_t n, const uint32_t *d_codes, const float *d_xnorm,
+                           const float *d_rnorm, int nq, const void *d_q, int q_dtype, int k,
+                           float *d_vals, int64_t *d_ids, void *stream);
 
 #ifdef __cplusplus
 }

@@ -18,6 +18,8 @@ TQ_ERR_WORKSPACE = -3
 TQ_ERR_CUDA = -4
 TQ_ERR_DEVICE_TIMEOUT = -5
 TQ_ERR_MISMATCH = -6
+TQ_ERR_SCRATCH_LIMIT = -7
+TQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 TQ_F32 = 0
 TQ_BF16 = 1
@@ -25,7 +27,7 @@ TQ_BF16 = 1
 TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT = range(6)
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_encode", "tq_score",
-           "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk")
+           "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc")
 
 
 class tq_codebook_t(C.Structure):
@@ -66,6 +68,8 @@ def _load():
     L.tq_score.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, P, P, sz, P]
     L.tq_topk.restype = i32
     L.tq_topk.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P, sz, P]
+    L.tq_topk_noalloc.restype = i32
+    L.tq_topk_noalloc.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P]
     L.tq_decode.restype = i32
     L.tq_decode.argtypes = [cbp, P, P, i32, i64, P, P, P, P, P, sz, P]
     L.tq_logits_fp32.restype = i32
@@ -113,6 +117,15 @@ def tq_topk(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k,
             d_ws, ws_bytes, stream):
     return _ok("tq_topk", lib.tq_topk(C.byref(cb), d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm,
                                       nq, d_q, q_dtype, k, d_vals, d_ids, d_ws, ws_bytes, stream))
+
+
+def tq_topk_noalloc(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
+                    d_ids, stream):
+    """tq_topk with its scratch in the library's fixed device array (no
+    workspace argument, nothing allocated); see include/tq.h."""
+    return _ok("tq_topk_noalloc", lib.tq_topk_noalloc(C.byref(cb), d_Pi, d_S, G, n, d_codes,
+                                                      d_xnorm, d_rnorm, nq, d_q, q_dtype, k,
+                                                      d_vals, d_ids, stream))
 
 
 def tq_decode(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, d_xhat, d_ws, ws_bytes, stream):

@@ -12,6 +12,7 @@ extern "C" const char* tq_status_str(int status) {
         case TQ_ERR_CUDA: return "CUDA error";
         case TQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
         case TQ_ERR_MISMATCH: return "codebook does not match the call";
+        case TQ_ERR_SCRATCH_LIMIT: return "sizes need more scratch than tq_topk_noalloc's fixed 8 MiB array";
         default: return "unknown status";
     }
 }
