@@ -135,6 +135,13 @@ TQ_API int tq_encode(const tq_codebook_t *cb, const float *d_Pi, const float *d_
               uint32_t *d_codes, float *d_xnorm, float *d_rnorm,
               void *d_ws, size_t ws_bytes, void *stream);
 
+/* Device status of the last tq_encode that used d_ws (its first 4 bytes):
+ * TQ_OK, or TQ_ERR_DEVICE_TIMEOUT when a bounded device-side wait of the
+ * tensor-core encode gave up (the kernel then drains its in-flight copies,
+ * releases tensor memory and exits; its outputs are undefined).  Copies the
+ * word to the host and synchronises `stream`. */
+TQ_API int tq_device_status(const void *d_ws, void *stream);
+
 /* S0 + S1, scores (quant_prune_distill #674: inner-product quantization with
  * an unbiased estimate; comuna.ru "8x faster attention logits"):
  *   qr = Pi_g q, u = S_g qr,

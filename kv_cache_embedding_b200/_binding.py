@@ -27,7 +27,8 @@ TQ_BF16 = 1
 TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT = range(6)
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_encode", "tq_score",
-           "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc")
+           "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
+           "tq_device_status")
 
 
 class tq_codebook_t(C.Structure):
@@ -70,6 +71,8 @@ def _load():
     L.tq_topk.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P, sz, P]
     L.tq_topk_noalloc.restype = i32
     L.tq_topk_noalloc.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P]
+    L.tq_device_status.restype = i32
+    L.tq_device_status.argtypes = [P, P]
     L.tq_decode.restype = i32
     L.tq_decode.argtypes = [cbp, P, P, i32, i64, P, P, P, P, P, sz, P]
     L.tq_logits_fp32.restype = i32
@@ -105,6 +108,11 @@ def tq_encode(cb, d_Pi, d_S, G, n, d_x, x_dtype, d_codes, d_xnorm, d_rnorm, d_ws
               stream):
     return _ok("tq_encode", lib.tq_encode(C.byref(cb), d_Pi, d_S, G, n, d_x, x_dtype, d_codes,
                                           d_xnorm, d_rnorm, d_ws, ws_bytes, stream))
+
+
+def tq_device_status(d_ws, stream):
+    """Status word the last tq_encode left in d_ws (synchronises the stream)."""
+    return lib.tq_device_status(d_ws, stream)
 
 
 def tq_score(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, d_scores, d_ws,

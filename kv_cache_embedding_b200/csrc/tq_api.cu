@@ -31,7 +31,7 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
             return 2 * align256(dd * 8) + 2 * align256((size_t)d * 8);
         case TQ_OP_ENCODE:
             if (b < 1 || b > 4) return (size_t)-1;
-            return 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
+            return 256 + 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
         case TQ_OP_SCORE:
             return 2 * qbuf;
         case TQ_OP_TOPK:
@@ -43,4 +43,13 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
         default:
             return (size_t)-1;
     }
+}
+
+extern "C" int tq_device_status(const void* d_ws, void* stream) {
+    if (!d_ws) return TQ_ERR_ARG;
+    int word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    TQ_TRY_CUDA(cudaMemcpyAsync(&word, d_ws, sizeof(int), cudaMemcpyDeviceToHost, s));
+    TQ_TRY_CUDA(cudaStreamSynchronize(s));
+    return word == 0 ? TQ_OK : TQ_ERR_DEVICE_TIMEOUT;
 }

@@ -115,10 +115,15 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     const size_t need = tq_workspace_bytes(TQ_OP_ENCODE, d, b, G, n, 0, 0);
     if (need > 0 && (!d_ws || ws_bytes < need)) return TQ_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
+    // the first 256 bytes of the workspace hold the device status word
+    if (encode_tc_supported(d, x_dtype, G, n))  // d = 128 bf16 keys: fused tensor-core kernel
+        return launch_encode_tc(cb, d_Pi, d_S, G, n, d_x, d_codes, d_xnorm, d_rnorm,
+                                (int*)d_ws, s);
+    TQ_TRY_CUDA(cudaMemsetAsync(d_ws, 0, sizeof(int), s));
     const KCodebook kc = make_kcodebook(cb);
     const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;
-    float* Y = (float*)d_ws;
-    float* P = (float*)((char*)d_ws + align256((size_t)chunk * d * 4));
+    float* Y = (float*)((char*)d_ws + 256);
+    float* P = (float*)((char*)Y + align256((size_t)chunk * d * 4));
     uint8_t* IX = (uint8_t*)((char*)P + align256((size_t)chunk * d * 4));
     const int W = words_per_vector(d, b);
     const size_t esz = (x_dtype == TQ_F32) ? 4 : 2;

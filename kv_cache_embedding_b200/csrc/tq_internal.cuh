@@ -13,7 +13,7 @@ constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ULL;
 constexpr int kMinD = 128;
 constexpr int kMaxD = 4096;
 constexpr int kMaxK = 32;           // largest top-k
-constexpr int kTopkTile = 1024;     // keys per top-k tile (one partial list each)
+constexpr int kTopkTile = 256;      // keys per top-k tile (one partial list each)
 constexpr int64_t kEncodeChunk = 65536;  // rows per encode/decode chunk
 
 // Codebook passed to kernels by value (kernel parameter space).
@@ -66,4 +66,8 @@ namespace tq {
 int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const float* B,
                  bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
                  cudaStream_t s);
+bool encode_tc_supported(int d, int x_dtype, int G, int64_t n);
+int launch_encode_tc(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                     int64_t n, const void* d_x, uint32_t* d_codes, float* d_xnorm,
+                     float* d_rnorm, int* d_err, cudaStream_t s);
 }

@@ -11,6 +11,7 @@
 //   s = |x| ( <qr, c[idx]> + |r| sqrt(pi/2)/d <u, 2z - 1> ),  qr = Pi q, u = S qr.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 
 #include "tq_internal.cuh"
 
@@ -55,73 +56,161 @@ __device__ __forceinline__ void load_block(const uint32_t* __restrict__ rec, int
     }
 }
 
-// Score QC queries (rows of s_qr / s_u in shared memory) against one record.
-template <int B, int QC>
-__device__ __forceinline__ void score_record(const uint32_t* __restrict__ rec, int d,
-                                             const float* s_qr, const float* s_u,
-                                             const float* s_c, float am[QC], float aq[QC]) {
+// ---- scoring, v2 ---------------------------------------------------------
+// Thread = KP keys; block = 128 threads; queries in passes of NQ.  Shared
+// memory holds, per query, the pairs (qr_i, u_i) interleaved, and a 16-entry
+// table mapping a coordinate's field f to (c[idx], 2z - 1), so decoding a
+// coordinate is one bit-field extract and one conflict-free 8-byte load
+// (every entry owns its own bank pair).  Each query pair is loaded once per
+// two coordinates and reused by the thread's KP keys.  Accumulators are
+// (mse, qjl) pairs; with F2 they are updated by the packed fma.rn.f32x2.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+template <bool F2>
+__device__ __forceinline__ float2 pair_fma(float2 a, float2 b, float2 c) {
+    if (F2) return ffma2(a, b, c);
+    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+}
+
+// Field of coordinate j (0..31) of a block as the decode-table index.
+template <int B>
+__device__ __forceinline__ uint32_t field_index(const uint32_t (&w)[4], int j) {
+    if (B == 1) return (w[0] >> j) & 1u;
+    if (B == 2) return (w[j >> 4] >> (2 * (j & 15))) & 3u;
+    if (B == 3) return ((w[j >> 4] >> (2 * (j & 15))) & 3u) | (((w[2] >> j) & 1u) << 2);
+    return (w[j >> 3] >> (4 * (j & 7))) & 15u;
+}
+
+// Decode table entry f -> (c[idx], 2z - 1) for the field layouts above.
+template <int B>
+__device__ __forceinline__ float2 table_entry(const KCodebook& cb, int f) {
+    if (B == 1) return make_float2(0.f, (f & 1) ? 1.f : -1.f);
+    if (B == 2) return make_float2(cb.c[f & 1], (f & 2) ? 1.f : -1.f);
+    if (B == 3) return make_float2(cb.c[f & 3], (f & 4) ? 1.f : -1.f);
+    return make_float2(cb.c[f & 7], (f & 8) ? 1.f : -1.f);
+}
+
+// Shared-memory setup common to the scoring kernels: the 16-entry decode
+// table and the NQ queries' (qr_i, u_i) pairs starting at query q0.
+template <int B, int NQ>
+__device__ __forceinline__ void load_score_smem(const KCodebook& cb, const float* __restrict__ qr,
+                                                const float* __restrict__ u, int64_t row0, int qn,
+                                                int d, float2* s_qu, float2* s_tab) {
+    if (threadIdx.x < 16) {
+        float2 e = make_float2(0.f, 0.f);
+        switch (threadIdx.x) {  // static indices keep the codebook in parameter space
+#define TQ_TAB(F) case F: e = table_entry<B>(cb, F); break;
+            TQ_TAB(0) TQ_TAB(1) TQ_TAB(2) TQ_TAB(3) TQ_TAB(4) TQ_TAB(5) TQ_TAB(6) TQ_TAB(7)
+            TQ_TAB(8) TQ_TAB(9) TQ_TAB(10) TQ_TAB(11) TQ_TAB(12) TQ_TAB(13) TQ_TAB(14) TQ_TAB(15)
+#undef TQ_TAB
+        }
+        s_tab[threadIdx.x] = e;
+    }
+    for (int e = threadIdx.x; e < NQ * d; e += blockDim.x) {
+        const int qq = e / d, i = e % d;
+        const int64_t row = row0 + qq;
+        s_qu[e] = (qq < qn) ? make_float2(qr[row * d + i], u[row * d + i]) : make_float2(0.f, 0.f);
+    }
+}
+
+// Accumulate (mse, qjl) pairs of KP records against NQ queries.
+template <int B, int NQ, int KP, bool F2>
+__device__ __forceinline__ void score_keys(const uint32_t* const (&rec)[KP], int d,
+                                           const float2* s_qu, const float2* s_tab,
+                                           float2 (&acc)[KP][NQ]) {
+    uint32_t wcur[KP][4], wnext[KP][4];
 #pragma unroll
-    for (int q = 0; q < QC; ++q) am[q] = aq[q] = 0.f;
+    for (int k = 0; k < KP; ++k) load_block<B>(rec[k], 0, wcur[k]);
     for (int blk = 0; blk < d / 32; ++blk) {
-        uint32_t w[4];
-        load_block<B>(rec, blk, w);
+        if (blk + 1 < d / 32) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            int cell;
-            uint32_t z;
-            field<B>(w, j, cell, z);
-            const float yh = (B == 1) ? 0.f : s_c[cell];
-            const float t = z ? 1.f : -1.f;
-            const int i = blk * 32 + j;
+            for (int k = 0; k < KP; ++k) load_block<B>(rec[k], blk + 1, wnext[k]);
+        }
+        const float2* qb = s_qu + blk * 32;
 #pragma unroll
-            for (int q = 0; q < QC; ++q) {
-                if (B != 1) am[q] = fmaf(s_qr[q * d + i], yh, am[q]);
-                aq[q] = fmaf(s_u[q * d + i], t, aq[q]);
+        for (int j = 0; j < 32; j += 2) {
+            float2 e0[KP], e1[KP];
+#pragma unroll
+            for (int k = 0; k < KP; ++k) {
+                e0[k] = s_tab[field_index<B>(wcur[k], j)];
+                e1[k] = s_tab[field_index<B>(wcur[k], j + 1)];
             }
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq) {
+                const float4 p = *reinterpret_cast<const float4*>(qb + qq * d + j);
+                const float2 p0 = make_float2(p.x, p.y), p1 = make_float2(p.z, p.w);
+#pragma unroll
+                for (int k = 0; k < KP; ++k) {
+                    acc[k][qq] = pair_fma<F2>(p0, e0[k], acc[k][qq]);
+                    acc[k][qq] = pair_fma<F2>(p1, e1[k], acc[k][qq]);
+                }
+            }
+        }
+        if (blk + 1 < d / 32) {
+#pragma unroll
+            for (int k = 0; k < KP; ++k)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) wcur[k][w] = wnext[k][w];
         }
     }
 }
 
-__device__ void load_queries(const float* __restrict__ qr, const float* __restrict__ u,
-                             int64_t q0, int qn, int QC, int d, float* s_qr, float* s_u) {
-    for (int e = threadIdx.x; e < QC * d; e += blockDim.x) {
-        const int q = e / d;
-        const float a = (q < qn) ? qr[(q0 + q) * d + (e % d)] : 0.f;
-        const float b = (q < qn) ? u[(q0 + q) * d + (e % d)] : 0.f;
-        s_qr[e] = a;
-        s_u[e] = b;
-    }
-}
-
-// grid: (key blocks of 128, G, query chunks); scores [G][nq][n]
-template <int B, int QC>
-__global__ __launch_bounds__(128) void k_score(const uint32_t* __restrict__ codes,
-                                               const float* __restrict__ xnorm,
-                                               const float* __restrict__ rnorm, int64_t n, int d,
-                                               int nq, const float* __restrict__ qr,
-                                               const float* __restrict__ u, KCodebook cb,
-                                               float* __restrict__ scores) {
-    extern __shared__ __align__(16) float smem[];
-    float* s_qr = smem;
-    float* s_u = smem + QC * d;
-    __shared__ float s_c[8];
+template <int B, int NQ, int KP, bool F2>
+__global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ codes,
+                                                const float* __restrict__ xnorm,
+                                                const float* __restrict__ rnorm, int64_t n, int d,
+                                                int nq, const float* __restrict__ qr,
+                                                const float* __restrict__ u, KCodebook cb,
+                                                float* __restrict__ scores) {
+    extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d] pairs (qr_i, u_i)
+    __shared__ float2 s_tab[16];
     const int g = blockIdx.y;
-    const int q0 = blockIdx.z * QC;
-    const int qn = min(QC, nq - q0);
-    if (threadIdx.x < 8) s_c[threadIdx.x] = cb.c[threadIdx.x];
-    load_queries(qr, u, (int64_t)g * nq + q0, qn, QC, d, s_qr, s_u);
+    const int q0 = blockIdx.z * NQ;
+    const int qn = min(NQ, nq - q0);
+    load_score_smem<B, NQ>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
     __syncthreads();
-    const int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= n) return;
     const int W = words_per_vector(d, B);
-    const int64_t gv = (int64_t)g * n + v;
-    float am[QC], aq[QC];
-    score_record<B, QC>(codes + gv * W, d, s_qr, s_u, s_c, am, aq);
-    const float xn = xnorm[gv];
-    const float kap = kSqrtHalfPi / (float)d * rnorm[gv];
+    int64_t v[KP];
+    bool ok[KP];
 #pragma unroll
-    for (int q = 0; q < QC; ++q)
-        if (q < qn) scores[((int64_t)g * nq + q0 + q) * n + v] = xn * (am[q] + kap * aq[q]);
+    for (int k = 0; k < KP; ++k) {
+        v[k] = ((int64_t)blockIdx.x * KP + k) * blockDim.x + threadIdx.x;
+        ok[k] = v[k] < n;
+    }
+    float2 acc[KP][NQ];
+#pragma unroll
+    for (int k = 0; k < KP; ++k)
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) acc[k][qq] = make_float2(0.f, 0.f);
+    const uint32_t* rec[KP];
+#pragma unroll
+    for (int k = 0; k < KP; ++k) rec[k] = codes + ((int64_t)g * n + (ok[k] ? v[k] : 0)) * W;
+
+    score_keys<B, NQ, KP, F2>(rec, d, s_qu, s_tab, acc);
+    const float k0 = kSqrtHalfPi / (float)d;
+#pragma unroll
+    for (int k = 0; k < KP; ++k) {
+        if (!ok[k]) continue;
+        const int64_t gv = (int64_t)g * n + v[k];
+        const float xn = xnorm[gv];
+        const float kap = k0 * rnorm[gv];
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq)
+            if (qq < qn)
+                scores[((int64_t)g * nq + q0 + qq) * n + v[k]] =
+                    xn * (acc[k][qq].x + kap * acc[k][qq].y);
+    }
 }
 
 // ---- top-k -------------------------------------------------------------
@@ -159,42 +248,56 @@ __device__ void warp_select(float* s, int count, int64_t id0, int K, float* vals
     }
 }
 
-// grid: (tiles of kTopkTile keys, G, query chunks of QC <= 8); 256 threads.
-// Writes the tile's best K per query to part_vals/part_ids
+// grid: (tiles of kTopkTile keys, G, query passes of NQ <= 8); 256 threads,
+// KP = 4 keys each.  Scores of the tile go to shared memory, then warp q
+// selects the tile's best K for query q0 + q into part_vals/part_ids
 // [G][nq][ntiles][K].
-template <int B, int QC>
+template <int B, int NQ, bool F2>
 __global__ __launch_bounds__(256) void k_score_topk_tile(
     const uint32_t* __restrict__ codes, const float* __restrict__ xnorm,
     const float* __restrict__ rnorm, int64_t n, int d, int nq, const float* __restrict__ qr,
     const float* __restrict__ u, KCodebook cb, int K, int ntiles, float* __restrict__ part_vals,
     int64_t* __restrict__ part_ids) {
-    extern __shared__ __align__(16) float smem[];
-    float* s_qr = smem;
-    float* s_u = smem + QC * d;
-    float* s_sc = smem + 2 * QC * d;  // [QC][kTopkTile]
-    __shared__ float s_c[8];
+    constexpr int KP = kTopkTile / 256;
+    extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d], then scores [NQ][kTopkTile]
+    float* s_sc = reinterpret_cast<float*>(s_qu + NQ * d);
+    __shared__ float2 s_tab[16];
     const int g = blockIdx.y;
-    const int q0 = blockIdx.z * QC;
-    const int qn = min(QC, nq - q0);
+    const int q0 = blockIdx.z * NQ;
+    const int qn = min(NQ, nq - q0);
     const int64_t t0 = (int64_t)blockIdx.x * kTopkTile;
-    if (threadIdx.x < 8) s_c[threadIdx.x] = cb.c[threadIdx.x];
-    load_queries(qr, u, (int64_t)g * nq + q0, qn, QC, d, s_qr, s_u);
+    load_score_smem<B, NQ>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
     __syncthreads();
     const int W = words_per_vector(d, B);
+    int64_t v[KP];
+    bool ok[KP];
+    const uint32_t* rec[KP];
+#pragma unroll
+    for (int k = 0; k < KP; ++k) {
+        v[k] = t0 + k * 256 + threadIdx.x;
+        ok[k] = v[k] < n;
+        rec[k] = codes + ((int64_t)g * n + (ok[k] ? v[k] : 0)) * W;
+    }
+    float2 acc[KP][NQ];
+#pragma unroll
+    for (int k = 0; k < KP; ++k)
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) acc[k][qq] = make_float2(0.f, 0.f);
+    score_keys<B, NQ, KP, F2>(rec, d, s_qu, s_tab, acc);
     const float k0 = kSqrtHalfPi / (float)d;
-    for (int e = threadIdx.x; e < kTopkTile; e += blockDim.x) {
-        const int64_t v = t0 + e;
-        if (v < n) {
-            const int64_t gv = (int64_t)g * n + v;
-            float am[QC], aq[QC];
-            score_record<B, QC>(codes + gv * W, d, s_qr, s_u, s_c, am, aq);
+#pragma unroll
+    for (int k = 0; k < KP; ++k) {
+        const int e = k * 256 + threadIdx.x;
+        if (ok[k]) {
+            const int64_t gv = (int64_t)g * n + v[k];
             const float xn = xnorm[gv];
             const float kap = k0 * rnorm[gv];
 #pragma unroll
-            for (int q = 0; q < QC; ++q) s_sc[q * kTopkTile + e] = xn * (am[q] + kap * aq[q]);
+            for (int qq = 0; qq < NQ; ++qq)
+                s_sc[qq * kTopkTile + e] = xn * (acc[k][qq].x + kap * acc[k][qq].y);
         } else {
 #pragma unroll
-            for (int q = 0; q < QC; ++q) s_sc[q * kTopkTile + e] = -INFINITY;
+            for (int qq = 0; qq < NQ; ++qq) s_sc[qq * kTopkTile + e] = -INFINITY;
         }
     }
     __syncthreads();
@@ -378,42 +481,64 @@ __global__ __launch_bounds__(256) void k_logits_fp32(const float* __restrict__ k
 }
 
 // ---- helpers ----------------------------------------------------------------
-int score_qc(int d) { return d <= 1536 ? 8 : (d <= 3072 ? 4 : 2); }
 
-template <int B, int QC>
-int launch_score_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
-                   int G, int nq, const float* qr, const float* u, const KCodebook& kc,
-                   float* scores, cudaStream_t s) {
-    const size_t smem = (size_t)2 * QC * d * sizeof(float);
-    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score<B, QC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem));
-    dim3 grid((unsigned)((n + 127) / 128), (unsigned)G, (unsigned)((nq + QC - 1) / QC));
-    k_score<B, QC><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores);
+template <int B, int NQ, bool F2>
+int launch_score2_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
+                    int G, int nq, const float* qr, const float* u, const KCodebook& kc,
+                    float* scores, cudaStream_t s) {
+    constexpr int KP = 2;
+    const size_t smem = (size_t)NQ * d * sizeof(float2);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score2<B, NQ, KP, F2>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    dim3 grid((unsigned)((n + 128 * KP - 1) / (128 * KP)), (unsigned)G,
+              (unsigned)((nq + NQ - 1) / NQ));
+    k_score2<B, NQ, KP, F2><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
+
+// Queries per pass: as many as the group has, up to what shared memory holds.
+int score_nq(int d, int nq) {
+    const int cap = d <= 1536 ? 8 : (d <= 3072 ? 4 : 2);
+    int p = 1;
+    while (p < nq && p < cap) p <<= 1;
+    return p;
+}
+
+// packed f32x2 accumulation (sm_100 fma.rn.f32x2); TQ_SCORE_FFMA2=0 selects plain FFMA
+const bool g_score_f2 = [] {
+    const char* e = getenv("TQ_SCORE_FFMA2");
+    return !(e && e[0] == '0');
+}();
 
 template <int B>
 int launch_score_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                    int G, int nq, const float* qr, const float* u, const KCodebook& kc,
                    float* scores, cudaStream_t s) {
-    switch (score_qc(d)) {
-        case 8: return launch_score_t<B, 8>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
-        case 4: return launch_score_t<B, 4>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
-        default: return launch_score_t<B, 2>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, s);
+#define TQ_SC(NQV)                                                                          \
+    return g_score_f2 ? launch_score2_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
+                                                      scores, s)                            \
+                      : launch_score2_t<B, NQV, false>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
+                                                       scores, s)
+    switch (score_nq(d, nq)) {
+        case 1: TQ_SC(1);
+        case 2: TQ_SC(2);
+        case 4: TQ_SC(4);
+        default: TQ_SC(8);
     }
+#undef TQ_SC
 }
 
-template <int B, int QC>
+template <int B, int NQ, bool F2>
 int launch_topk_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
                   int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
-    const size_t smem = ((size_t)2 * QC * d + (size_t)QC * kTopkTile) * sizeof(float);
-    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score_topk_tile<B, QC>,
+    const size_t smem = (size_t)NQ * d * sizeof(float2) + (size_t)NQ * kTopkTile * sizeof(float);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score_topk_tile<B, NQ, F2>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    dim3 grid((unsigned)ntiles, (unsigned)G, (unsigned)((nq + QC - 1) / QC));
-    k_score_topk_tile<B, QC><<<grid, 256, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, K,
-                                                     ntiles, pv, pi);
+    dim3 grid((unsigned)ntiles, (unsigned)G, (unsigned)((nq + NQ - 1) / NQ));
+    k_score_topk_tile<B, NQ, F2><<<grid, 256, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, K,
+                                                          ntiles, pv, pi);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -422,21 +547,98 @@ template <int B>
 int launch_topk_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
                   int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
-    switch (score_qc(d)) {
-        case 8:
-            return launch_topk_t<B, 8>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
-        case 4:
-            return launch_topk_t<B, 4>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
-        default:
-            return launch_topk_t<B, 2>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, ntiles, pv, pi, s);
+#define TQ_TK(NQV)                                                                              \
+    return g_score_f2 ? launch_topk_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, K,    \
+                                                    ntiles, pv, pi, s)                          \
+                      : launch_topk_t<B, NQV, false>(codes, xn, rn, n, d, G, nq, qr, u, kc, K,   \
+                                                     ntiles, pv, pi, s)
+    switch (score_nq(d, nq)) {
+        case 1: TQ_TK(1);
+        case 2: TQ_TK(2);
+        case 4: TQ_TK(4);
+        default: TQ_TK(8);
+    }
+#undef TQ_TK
+}
+
+// qr = Pi_g q and u = S_g qr for one (query, group) per block: one warp per
+// output row (coalesced row reads, shuffle reduction), qr kept in shared
+// memory for the second product.  Used when there are few queries per group.
+template <typename TQ>
+__global__ __launch_bounds__(512) void k_query_prep(const float* __restrict__ Pi,
+                                                    const float* __restrict__ S, int d, int nq,
+                                                    const TQ* __restrict__ q,
+                                                    float* __restrict__ qr,
+                                                    float* __restrict__ u) {
+    extern __shared__ __align__(16) float sq[];  // [0, d): q   [d, 2d): qr
+    constexpr int R = 8;  // rows per warp in flight
+    const int g = blockIdx.y;
+    const int64_t row = (int64_t)g * nq + blockIdx.x;
+    for (int j = threadIdx.x; j < d; j += blockDim.x) sq[j] = load_f32(q, row * d + j);
+    __syncthreads();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const float* M = (pass == 0 ? Pi : S) + (size_t)g * d * d;
+        const float* v = sq + pass * d;
+        float* outg = (pass == 0 ? qr : u) + row * d;
+        for (int i0 = warp * R; i0 < d; i0 += nw * R) {
+            float acc[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) acc[r] = 0.f;
+            for (int f = lane; f < d / 4; f += 32) {
+                const float4 b = *reinterpret_cast<const float4*>(v + 4 * f);
+                float4 a[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    a[r] = __ldg(reinterpret_cast<const float4*>(M + (size_t)(i0 + r) * d) + f);
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    acc[r] = fmaf(a[r].x, b.x, acc[r]);
+                    acc[r] = fmaf(a[r].y, b.y, acc[r]);
+                    acc[r] = fmaf(a[r].z, b.z, acc[r]);
+                    acc[r] = fmaf(a[r].w, b.w, acc[r]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], o);
+            }
+            if (lane < R) {
+                float a = acc[0];
+#pragma unroll
+                for (int r = 1; r < R; ++r) a = (lane == r) ? acc[r] : a;
+                outg[i0 + lane] = a;
+                if (pass == 0) sq[d + i0 + lane] = a;
+            }
+        }
+        __syncthreads();
     }
 }
 
-// qr = Q Pi^T, u = qr S^T for every group (fp32 SIMT GEMM).
+// qr = Q Pi^T, u = qr S^T for every group: one fused launch for few queries,
+// else two fp32 SIMT GEMMs per group.
 int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const void* d_q,
                int q_dtype, float* qr, float* u, cudaStream_t s) {
     const size_t dd = (size_t)d * d;
     const size_t esz = (q_dtype == TQ_F32) ? 4 : 2;
+    if (nq <= 32) {
+        dim3 grid((unsigned)nq, (unsigned)G);
+        const size_t smem = (size_t)2 * d * sizeof(float);
+        if (q_dtype == TQ_F32) {
+            TQ_TRY_CUDA(cudaFuncSetAttribute(k_query_prep<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+            k_query_prep<float><<<grid, 512, smem, s>>>(d_Pi, d_S, d, nq, (const float*)d_q, qr, u);
+        } else {
+            TQ_TRY_CUDA(cudaFuncSetAttribute(k_query_prep<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+            k_query_prep<__nv_bfloat16><<<grid, 512, smem, s>>>(
+                d_Pi, d_S, d, nq, (const __nv_bfloat16*)d_q, qr, u);
+        }
+        TQ_CHECK_LAUNCH();
+        return TQ_OK;
+    }
     for (int g = 0; g < G; ++g) {
         const void* qg = (const char*)d_q + (size_t)g * nq * d * esz;
         int rc = launch_sgemm(nq, d, d, qg, q_dtype, d, d_Pi + g * dd, true, d,

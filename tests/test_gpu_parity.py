@@ -220,3 +220,35 @@ def test_errors_on_device(quant, tq_lib, cuda):
     with pytest.raises(ValueError):
         tq.encode(torch.zeros(10, 64, device=cuda))
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- tensor-core encode (d = 128, bf16)
+@pytest.mark.parametrize("G,n,b", [(1, 64, 1), (3, 640, 4), (1, 5, 2), (160, 100, 4), (8, 4097, 3)])
+def test_encode_tc_bf16_shapes(quant, oparams, tq_lib, G, n, b):
+    """Shapes of the fused tensor-core kernel: exact tiles, a 5-row tile, more
+    groups than SMs (whole groups per CTA, weights reloaded into tensor
+    memory at each group), ragged tails; device status word stays clean."""
+    x = synth.kv_keys(G, n, 128, seed=11)
+    tq = quant(128, b, 0, G)
+    codes = tq.encode(x.cuda())
+    B = tq_lib.binding
+    assert B.tq_device_status(tq.ws.buf.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+    for g in sorted({0, G // 2, G - 1}):
+        P = oparams(128, b, g)
+        ora = O.encode(P, x[g].to(torch.float64).numpy(), diagnostics=True)
+        gpu = (_np(codes.codes[g]).view(np.uint32), _np(codes.xnorm[g]), _np(codes.rnorm[g]))
+        PT.compare_encode(128, b, P.beta, gpu, ora, bound_flags=(n * 128 >= 10 ** 5))
+
+
+def test_encode_tc_matches_portable_path(quant, tq_lib):
+    """The tensor-core kernel (bf16 input) and the SIMT path (the same values
+    given as fp32) produce the same records up to boundary flips."""
+    G, n, b = 2, 2000, 4
+    x = synth.kv_keys(G, n, 128, seed=12)
+    tq = quant(128, b, 0, G)
+    c_tc = tq.encode(x.cuda())
+    c_pt = tq.encode(x.float().cuda())
+    torch.cuda.synchronize()
+    same = (c_tc.codes == c_pt.codes).all(dim=2).float().mean().item()
+    assert same > 0.995
+    assert torch.allclose(c_tc.xnorm, c_pt.xnorm, rtol=1e-6)
