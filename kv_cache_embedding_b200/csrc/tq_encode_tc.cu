@@ -17,14 +17,16 @@
 //  * A tile of 64 bf16 key vectors arrives by TMA (128-byte swizzle) and is
 //    the B operand as is: bf16 x bf16 products are exact, so the rotation
 //    D1 = Pi X^T is fp32-accurate after 3 passes.
-//  * Epilogue warps (thread = output coordinate) work in units scaled by 2^10
-//    (exact: 1/|x|, boundaries and centroids are pre-multiplied): y' = 2^10 y,
-//    bucketize, r' = y' - c'[idx], |r|^2, and r' as two fp16 pieces written
-//    coordinate-major (one 128-byte row per coordinate, vectors contiguous):
-//    the MN-major B operand of D2 = S R^T (3 passes: s1 h1 + s1 h2 + s2 h1).
-//    Only the sign of D2 is kept.
+//  * Epilogue warps (thread = output coordinate, kVpw vectors per warp) work
+//    in units scaled by 2^10 (exact: 1/|x|, boundaries and centroids are
+//    pre-multiplied): y' = 2^10 y, bucketize, r' = y' - c'[idx], |r|^2, and r'
+//    as two fp16 pieces written coordinate-major (one 128-byte row per
+//    coordinate, vectors contiguous): the MN-major B operand of D2 = S R^T
+//    (3 passes: s1 h1 + s1 h2 + s2 h1).  Only the sign of D2 is kept.  The
+//    second half of a tile (signs, packing, stores) runs after the first half
+//    of the next tile so the QJL MMA overlaps epilogue work.
 //  * Warp roles: 0 TMA producer, 1 TMEM owner + MMA issuer, 2-3 norms,
-//    4..11 epilogue (two warps per TMEM lane quarter, 32 vectors each).
+//    4.. epilogue (kEpi warps; kEpi / 4 per TMEM lane quarter).
 //  * Every wait is bounded (1 s); a warp that gives up sets the abort flag and
 //    the device status word, all roles leave their loops, in-flight TMA loads
 //    and MMAs are drained (again bounded) and TMEM is released.
@@ -45,22 +47,24 @@ using namespace sm100;
 constexpr int kD = 128;
 constexpr int kTN = 64;                      // vectors per tile (MMA N)
 constexpr int kXS = 4;                       // key-tile stages
-constexpr int kThreads = 384;
+constexpr int kVpw = 16;                     // vectors per epilogue warp
+constexpr int kNH = kTN / kVpw;              // epilogue warps per TMEM lane quarter
+constexpr int kEpi = 4 * kNH;                // epilogue warps
+constexpr int kThreads = 32 * (4 + kEpi);
 constexpr uint32_t kColPi = 0, kColS = 192, kColD1 = 320, kColD2 = 448, kTmemCols = 512;
 constexpr uint32_t kStageBytes = kTN * kD * 2;   // two 8 KB swizzled regions (k < 64, k >= 64)
 constexpr uint64_t kWaitNs = 1000000000ull;      // 1 s per wait
 constexpr float kRScale = 1024.f;                // r * 2^10 keeps fp16 pieces normal
-constexpr uint32_t kIdescRot = idesc_f16(1, 128, kTN);  // bf16 x bf16 -> f32
-constexpr uint32_t kIdescQjl = idesc_f16(0, 128, kTN) | (1u << 16);  // fp16 x fp16, B MN-major
+constexpr uint32_t kIdescRot = idesc_f16(1, 128, kTN);                // bf16 x bf16 -> f32
+constexpr uint32_t kIdescQjl = idesc_f16(0, 128, kTN) | (1u << 16);   // fp16 x fp16, B MN-major
 
 struct Smem {
     uint8_t x[kXS][kStageBytes];   // 1024-aligned (first member)
     uint8_t r[2][2][kStageBytes];  // [tile parity][piece h1, h2]: B operand of the QJL MMA
-    uint32_t codes[kTN][16];       // packed records of the tile (W <= 16 words)
-    float inv[kXS][kTN];           // 1/|x| per stage
-    float rr[2][4][kTN];           // [tile parity][lane quarter] |r|^2 partial sums
-    float c[8];
-    float beta[8];
+    float inv[kXS][kTN];           // 2^10 / |x| per stage
+    float rr[2][4][kTN];           // [tile parity][lane quarter] |r'|^2 partial sums
+    float c[8];                    // 2^10 c
+    float beta[8];                 // 2^10 beta
     uint64_t full_x[kXS], empty_x[kXS], norm_full[kXS];
     uint64_t d1_full[2], d1_empty[2], r_full, d2_full, d2_empty, w_ready, epi_bar, mma_done;
     uint32_t tmem_base;
@@ -108,161 +112,199 @@ __device__ __forceinline__ uint32_t pack_f16(__half lo, __half hi) {
     return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
 }
 
-// Row `row` of Pi (3 bf16 pieces) or S (2 fp16 pieces) into TMEM lane `row`:
-// column c of a piece holds k = 2c (low half) and k = 2c + 1 (high half).
-__device__ void load_weights(const float* __restrict__ Pi, const float* __restrict__ S, int g,
-                             int row, int h, uint32_t taddr_lane) {
-    if (h == 0) {
-        const float* src = Pi + ((size_t)g * kD + row) * kD;
-        for (int half = 0; half < 2; ++half) {
-            uint32_t p1[32], p2[32], p3[32];
+// 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp gets lane
+// (warp's quarter base + t), columns [taddr.col, +16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+template <int V>
+__device__ __forceinline__ void tmem_ldv(uint32_t taddr, uint32_t (&r)[V]) {
+    if constexpr (V == 16) tmem_ld16(taddr, r);
+    else tmem_ld32(taddr, r);
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+// Copy the d x d fp32 matrix M (row-major) transposed into shared memory,
+// stage[k][m] = M[m][k], by the epilogue warps (te = 0 .. 32 kEpi - 1): lane
+// = row m within a quarter, so the shared stores of a warp are contiguous;
+// each thread keeps its 8 row loads in flight together.
+__device__ __forceinline__ void stage_transposed(const float* __restrict__ M, float* stage, int te) {
+    const int m = 32 * ((te >> 5) & 3) + (te & 31);
+    const int kg = te >> 7;  // 0..3: which quarter of the 32 float4 of the row
+    float4 v[8];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float2 v = __ldg(reinterpret_cast<const float2*>(src + 64 * half + 2 * c));
-                __nv_bfloat16 a1 = __float2bfloat16_rn(v.x);
-                float ra = v.x - __bfloat162float(a1);
-                __nv_bfloat16 a2 = __float2bfloat16_rn(ra);
-                __nv_bfloat16 a3 = __float2bfloat16_rn(ra - __bfloat162float(a2));
-                __nv_bfloat16 b1 = __float2bfloat16_rn(v.y);
-                float rb = v.y - __bfloat162float(b1);
-                __nv_bfloat16 b2 = __float2bfloat16_rn(rb);
-                __nv_bfloat16 b3 = __float2bfloat16_rn(rb - __bfloat162float(b2));
-                p1[c] = pack_bf16(a1, b1);
-                p2[c] = pack_bf16(a2, b2);
-                p3[c] = pack_bf16(a3, b3);
+    for (int j = 0; j < 8; ++j)
+        v[j] = __ldg(reinterpret_cast<const float4*>(M + (size_t)m * kD) + 8 * kg + j);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int k = 4 * (8 * kg + j);
+        stage[(k + 0) * kD + m] = v[j].x;
+        stage[(k + 1) * kD + m] = v[j].y;
+        stage[(k + 2) * kD + m] = v[j].z;
+        stage[(k + 3) * kD + m] = v[j].w;
+    }
+}
+
+// Pieces of row `row` of the staged matrix (stage[k][row]) into TMEM lane
+// `row`: Pi as bf16 pieces 0-2 (bits 0-2 of `mask`), S as fp16 pieces 0-1
+// (bit 3).  Column c of a piece holds k = 2c (low half) and k = 2c + 1 (high
+// half); written 8 columns at a time.
+__device__ void pieces_to_tmem(const float* stage, bool is_pi, int row, int mask,
+                               uint32_t taddr_lane) {
+#pragma unroll 1
+    for (int piece = 0; piece < 3; ++piece) {
+        if (is_pi ? !(mask & (1 << piece)) : (piece == 2 || !(mask & 8))) continue;
+        const uint32_t col0 = is_pi ? kColPi + 64u * piece : kColS + 64u * piece;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float vx = stage[(2 * (c0 + c)) * kD + row];
+                const float vy = stage[(2 * (c0 + c) + 1) * kD + row];
+                if (is_pi) {  // Pi = p1 + p2 + p3 (bf16)
+                    __nv_bfloat16 a = __float2bfloat16_rn(vx), bb = __float2bfloat16_rn(vy);
+                    float ra = vx - __bfloat162float(a), rb = vy - __bfloat162float(bb);
+                    if (piece >= 1) {
+                        a = __float2bfloat16_rn(ra);
+                        bb = __float2bfloat16_rn(rb);
+                        ra -= __bfloat162float(a);
+                        rb -= __bfloat162float(bb);
+                    }
+                    if (piece == 2) {
+                        a = __float2bfloat16_rn(ra);
+                        bb = __float2bfloat16_rn(rb);
+                    }
+                    w[c] = pack_bf16(a, bb);
+                } else {  // S = s1 + s2 (fp16)
+                    __half a = __float2half_rn(vx), bb = __float2half_rn(vy);
+                    if (piece == 1) {
+                        a = __float2half_rn(vx - __half2float(a));
+                        bb = __float2half_rn(vy - __half2float(bb));
+                    }
+                    w[c] = pack_f16(a, bb);
+                }
             }
-            tmem_st32(taddr_lane + kColPi + 0 + 32 * half, p1);
-            tmem_st32(taddr_lane + kColPi + 64 + 32 * half, p2);
-            tmem_st32(taddr_lane + kColPi + 128 + 32 * half, p3);
+            tmem_st8(taddr_lane + col0 + (uint32_t)c0, w);
         }
+    }
+}
+
+// One halving round of a transposed butterfly: lane keeps half of its n
+// values (selected by `up`), sends the other half to lane ^ m and combines.
+template <int N, class Op, class T>
+__device__ __forceinline__ void halve(T (&v)[N], bool up, int m, Op op) {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+        const T lo = v[2 * i], hi = v[2 * i + 1];
+        v[i] = op(up ? hi : lo, __shfl_xor_sync(0xffffffffu, up ? lo : hi, m));
+    }
+}
+
+// Sum over the 32 lanes of v[j], for every j < V (V = 16 or 32).  Rounds pair
+// lanes by bits 0.. of the lane index against bits 0.. of j; lane l ends with
+// the sum for j = l % V (lanes l and l + 16 agree when V = 16).
+template <int V>
+__device__ __forceinline__ float transpose_reduce(const float (&v)[V], int lane) {
+    float cur[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) cur[i] = v[i];
+    auto add = [](float a, float b) { return a + b; };
+    halve<V>(cur, lane & 1, 1, add);
+    halve<V / 2>(reinterpret_cast<float(&)[V / 2]>(cur), lane & 2, 2, add);
+    halve<V / 4>(reinterpret_cast<float(&)[V / 4]>(cur), lane & 4, 4, add);
+    halve<V / 8>(reinterpret_cast<float(&)[V / 8]>(cur), lane & 8, 8, add);
+    float t;
+    if constexpr (V == 32) {
+        halve<2>(reinterpret_cast<float(&)[2]>(cur), lane & 16, 16, add);
+        t = cur[0];
     } else {
-        const float* src = S + ((size_t)g * kD + row) * kD;
-        for (int half = 0; half < 2; ++half) {
-            uint32_t s1[32], s2[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float2 v = __ldg(reinterpret_cast<const float2*>(src + 64 * half + 2 * c));
-                __half a1 = __float2half_rn(v.x);
-                __half a2 = __float2half_rn(v.x - __half2float(a1));
-                __half b1 = __float2half_rn(v.y);
-                __half b2 = __float2half_rn(v.y - __half2float(b1));
-                s1[c] = pack_f16(a1, b1);
-                s2[c] = pack_f16(a2, b2);
-            }
-            tmem_st32(taddr_lane + kColS + 0 + 32 * half, s1);
-            tmem_st32(taddr_lane + kColS + 64 + 32 * half, s2);
-        }
+        t = cur[0] + __shfl_xor_sync(0xffffffffu, cur[0], 16);
     }
+    return t;
 }
 
-// Sum of v[j] over the 32 lanes for every j; lane l returns the sum for j = l.
-__device__ __forceinline__ float transpose_reduce32(const float (&v)[32], int lane) {
-    float a[16], b[8], c[4], d[2];
+// OR-combine fields of F lanes (F = 8 or 16, already shifted into place) for
+// V vectors: afterwards lane e (= lane % F) holds the finished words of
+// vectors j = e + F*i, i < V/F.
+template <int F, int V>
+__device__ __forceinline__ void transpose_or(const uint32_t (&v)[V], int lane,
+                                             uint32_t (&out)[V / F]) {
+    uint32_t cur[V];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const bool up = lane & 16;
-        const float keep = up ? v[i + 16] : v[i], send = up ? v[i] : v[i + 16];
-        a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
+    for (int i = 0; i < V; ++i) cur[i] = v[i];
+    auto orr = [](uint32_t a, uint32_t b) { return a | b; };
+    halve<V>(cur, lane & 1, 1, orr);
+    halve<V / 2>(reinterpret_cast<uint32_t(&)[V / 2]>(cur), lane & 2, 2, orr);
+    halve<V / 4>(reinterpret_cast<uint32_t(&)[V / 4]>(cur), lane & 4, 4, orr);
+    if constexpr (F == 16) halve<V / 8>(reinterpret_cast<uint32_t(&)[V / 8]>(cur), lane & 8, 8, orr);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 8;
-        const float keep = up ? a[i + 8] : a[i], send = up ? a[i] : a[i + 8];
-        b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 4;
-        const float keep = up ? b[i + 4] : b[i], send = up ? b[i] : b[i + 4];
-        c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const bool up = lane & 2;
-        const float keep = up ? c[i + 2] : c[i], send = up ? c[i] : c[i + 2];
-        d[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-    const bool up = lane & 1;
-    const float keep = up ? d[1] : d[0], send = up ? d[0] : d[1];
-    return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    for (int i = 0; i < V / F; ++i) out[i] = cur[i];
 }
 
-// OR-combine fields of F lanes (F = 8 or 16, fields already shifted into
-// place) for 32 vectors: afterwards lane e (= lane % F) holds the finished
-// words of vectors j = e + F*i, i < 32/F.
-template <int F>
-__device__ __forceinline__ void transpose_or(const uint32_t (&v)[32], int lane,
-                                             uint32_t (&out)[32 / F]) {
-    uint32_t a[16], b[8], c[4], d[2];
-    const int e = lane % F;
+// Pack the fields of this lane's coordinate (block q, position `lane`) for
+// the warp's V vectors (rows V*h .. V*h + V - 1 of the tile) and store the
+// finished words of block q straight to the tile's records `dst` (W words per
+// record); rows at or beyond `valid` are not written.
+template <int B, int V>
+__device__ __forceinline__ void pack_store(const uint32_t (&cellw)[V / 8],
+                                           const uint32_t (&pbits)[V], int lane, int q, int h,
+                                           uint32_t* __restrict__ dst, int valid) {
+    constexpr int W = B * kD / 32;
+    uint32_t z[V];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const bool up = e & 1;
-        const uint32_t lo = v[2 * i], hi = v[2 * i + 1];
-        a[i] = (up ? hi : lo) | __shfl_xor_sync(0xffffffffu, up ? lo : hi, 1);
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool up = e & 2;
-        const uint32_t lo = a[2 * i], hi = a[2 * i + 1];
-        b[i] = (up ? hi : lo) | __shfl_xor_sync(0xffffffffu, up ? lo : hi, 2);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool up = e & 4;
-        const uint32_t lo = b[2 * i], hi = b[2 * i + 1];
-        c[i] = (up ? hi : lo) | __shfl_xor_sync(0xffffffffu, up ? lo : hi, 4);
-    }
-    if (F == 8) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) out[i] = c[i];
-    } else {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const bool up = e & 8;
-            const uint32_t lo = c[2 * i], hi = c[2 * i + 1];
-            d[i] = (up ? hi : lo) | __shfl_xor_sync(0xffffffffu, up ? lo : hi, 8);
-        }
-#pragma unroll
-        for (int i = 0; i < 32 / F; ++i) out[i] = d[i];
-    }
-}
-
-// Pack the fields of this lane's coordinate (block q, position `lane`) for the
-// warp's 32 vectors into sm.codes rows [32h, 32h + 32).
-template <int B>
-__device__ __forceinline__ void pack_tile(const int (&cell)[32], const uint32_t (&pbits)[32],
-                                          int lane, int q, int h, uint32_t (*codes)[16]) {
-    uint32_t z[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) z[j] = (__uint_as_float(pbits[j]) >= 0.f) ? 1u : 0u;
+    for (int j = 0; j < V; ++j) z[j] = (__uint_as_float(pbits[j]) >= 0.f) ? 1u : 0u;
     if (B == 1 || B == 3) {
         uint32_t mine = 0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < V; ++j) {
             const uint32_t w = __ballot_sync(0xffffffffu, z[j] != 0u);
             if (lane == j) mine = w;
         }
-        codes[32 * h + lane][B * q + (B == 1 ? 0 : 2)] = mine;
+        if (lane < V && V * h + lane < valid)
+            dst[(V * h + lane) * W + B * q + (B == 1 ? 0 : 2)] = mine;
     }
     if (B == 4) {
-        uint32_t v[32], out[4];
+        uint32_t v[V], out[V / 8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = ((uint32_t)cell[j] | (z[j] << 3)) << (4 * (lane & 7));
-        transpose_or<8>(v, lane, out);
+        for (int j = 0; j < V; ++j) {
+            const uint32_t cell = (cellw[j >> 3] >> (4 * (j & 7))) & 15u;
+            v[j] = (cell | (z[j] << 3)) << (4 * (lane & 7));
+        }
+        transpose_or<8, V>(v, lane, out);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) codes[32 * h + (lane & 7) + 8 * i][4 * q + (lane >> 3)] = out[i];
+        for (int i = 0; i < V / 8; ++i) {
+            const int row = V * h + (lane & 7) + 8 * i;
+            if (row < valid) dst[row * W + 4 * q + (lane >> 3)] = out[i];
+        }
     }
     if (B == 2 || B == 3) {
-        uint32_t v[32], out[2];
+        uint32_t v[V], out[V / 16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const uint32_t f = (B == 2) ? ((uint32_t)cell[j] | (z[j] << 1)) : (uint32_t)cell[j];
+        for (int j = 0; j < V; ++j) {
+            const uint32_t cell = (cellw[j >> 3] >> (4 * (j & 7))) & 15u;
+            const uint32_t f = (B == 2) ? (cell | (z[j] << 1)) : cell;
             v[j] = f << (2 * (lane & 15));
         }
-        transpose_or<16>(v, lane, out);
+        transpose_or<16, V>(v, lane, out);
 #pragma unroll
-        for (int i = 0; i < 2; ++i) codes[32 * h + (lane & 15) + 16 * i][B * q + (lane >> 4)] = out[i];
+        for (int i = 0; i < V / 16; ++i) {
+            const int row = V * h + (lane & 15) + 16 * i;
+            if (row < valid) dst[row * W + B * q + (lane >> 4)] = out[i];
+        }
     }
 }
 
@@ -274,27 +316,30 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             int* __restrict__ err) {
     constexpr int L = (B == 1) ? 1 : (1 << (B - 1));
     constexpr int W = B * kD / 32;
-    extern __shared__ uint8_t smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                        ~uintptr_t(1023));
+    constexpr int V = kVpw;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment by pointer arithmetic on the shared array itself, so
+    // every access below stays a shared-memory (not generic) access
+    const uint32_t sbase = smem_u32(smem_raw);
+    Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     volatile int* abort = &sm.abort;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kXS; ++s) {
             mbar_init(&sm.full_x[s], 1);
-            mbar_init(&sm.empty_x[s], 11);  // MMA commit + 2 norm warps + 8 epilogue warps
+            mbar_init(&sm.empty_x[s], 1 + 2 + kEpi);  // MMA commit + norm warps + epilogue
             mbar_init(&sm.norm_full[s], 2);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.d1_full[b], 1);
-            mbar_init(&sm.d1_empty[b], 8);
+            mbar_init(&sm.d1_empty[b], kEpi);
         }
-        mbar_init(&sm.r_full, 8);
+        mbar_init(&sm.r_full, kEpi);
         mbar_init(&sm.d2_full, 1);
-        mbar_init(&sm.d2_empty, 8);
-        mbar_init(&sm.w_ready, 8);
-        mbar_init(&sm.epi_bar, 8);
+        mbar_init(&sm.d2_empty, kEpi);
+        mbar_init(&sm.w_ready, kEpi);
+        mbar_init(&sm.epi_bar, kEpi);
         mbar_init(&sm.mma_done, 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // static indices: the codebook stays out of local memory
@@ -426,57 +471,60 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
         });
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
-        const int q = warp & 3, h = (warp - 4) >> 2;
+        const int q = warp & 3, h = (warp - 4) >> 2;  // lane quarter, vector slice
         const int coord = q * 32 + lane;
         const uint32_t lane_addr = tbase + ((uint32_t)(q * 32) << 16);
         // residual row of this coordinate: 128 bytes, 16-byte chunk c (vectors
-        // 8c..8c+7) at position c ^ (coord % 8); this warp writes chunks 4h..4h+3
-        uint32_t roff[4];
+        // 8c..8c+7) at position c ^ (coord % 8); this warp writes chunks
+        // (V/8) h .. (V/8) h + V/8 - 1
+        uint32_t roff[V / 8];
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii)
-            roff[ii] = (uint32_t)coord * 128u + ((((uint32_t)(4 * h + ii)) ^ (uint32_t)(coord & 7)) << 4);
+        for (int ii = 0; ii < V / 8; ++ii)
+            roff[ii] = (uint32_t)coord * 128u +
+                       ((((uint32_t)(V / 8 * h + ii)) ^ (uint32_t)(coord & 7)) << 4);
         float bt[7];
 #pragma unroll
         for (int k = 0; k < 7; ++k) bt[k] = sm.beta[k];
+        // weight pieces this warp loads into TMEM at each group start
+        const int wmask = (kNH == 4) ? (1 << h) : (h == 0 ? 7 : 8);
         uint32_t i = 0, eb = 0;
-        const int te = threadIdx.x - 128;  // 0..255 over the epilogue warps
-        auto epi_sync = [&]() -> bool {
+        const int te = threadIdx.x - 128;  // 0 .. 32*kEpi - 1 over the epilogue warps
+        auto epi_sync = [&]() -> bool {  // all epilogue warps
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.epi_bar);
             const bool ok = warp_wait(&sm.epi_bar, eb & 1, abort);
             ++eb;
             return ok;
         };
+        float* stage = reinterpret_cast<float*>(&sm.r[0][0][0]);  // 64 KB, free at group start
         // The second half of a tile (sign bits, packing, stores) runs after the
-        // first half of the next tile, so the QJL MMA of a tile overlaps the
-        // epilogue work of its successor.  State of the pending tile:
+        // first half of the next tile.  State of the pending tile:
         bool pend = false;
         int pg = 0, pt = 0;
         uint32_t pidx = 0;
-        uint32_t pcell[4] = {0u, 0u, 0u, 0u};
+        uint32_t pcell[V / 8];
+#pragma unroll
+        for (int u = 0; u < V / 8; ++u) pcell[u] = 0u;
         auto finish = [&]() -> bool {
             if (!warp_wait(&sm.d2_full, pidx & 1, abort)) return give_up(abort, err, 9);
             tc_fence_after();
-            uint32_t pb[32];
-            tmem_ld32(lane_addr + kColD2 + 32u * h, pb);
+            uint32_t pb[V];
+            tmem_ldv<V>(lane_addr + kColD2 + (uint32_t)(V * h), pb);
             tmem_wait_ld();
+            const int64_t v0 = (int64_t)pt * kTN;
+            const int valid = (int)((n - v0) < kTN ? (n - v0) : kTN);
+            // |r|^2 of the tile is complete: every epilogue warp stored its part
+            // before arriving on r_full, which the QJL MMA behind d2_full waited for
+            if (q == 0 && lane < V && V * h + lane < valid) {
+                const float (*rrb)[kTN] = sm.rr[pidx & 1];
+                const int vv = V * h + lane;
+                rnorm[(int64_t)pg * n + v0 + vv] =
+                    sqrtf(rrb[0][vv] + rrb[1][vv] + rrb[2][vv] + rrb[3][vv]) * (1.f / kRScale);
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.d2_empty);
-            int cell[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) cell[j] = (int)((pcell[j >> 3] >> (4 * (j & 7))) & 15u);
-            pack_tile<B>(cell, pb, lane, q, h, sm.codes);
-            if (!epi_sync()) return give_up(abort, err, 10);
-            const int64_t v0 = (int64_t)pt * kTN;
-            const int valid = (int)((n - v0) < kTN ? (n - v0) : kTN);
-            uint32_t* dst = codes + ((int64_t)pg * n + v0) * W;
-            for (int e = te; e < valid * W; e += 256) dst[e] = sm.codes[e / W][e % W];
-            const float (*rrb)[kTN] = sm.rr[pidx & 1];
-            if (te < valid)
-                rnorm[(int64_t)pg * n + v0 + te] =
-                    sqrtf(rrb[0][te] + rrb[1][te] + rrb[2][te] + rrb[3][te]) * (1.f / kRScale);
-            if (!epi_sync()) return give_up(abort, err, 11);
+            pack_store<B, V>(pcell, pb, lane, q, h, codes + ((int64_t)pg * n + v0) * W, valid);
             pend = false;
             return true;
         };
@@ -485,7 +533,14 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             if (first) {
                 // every MMA of the previous group must be done before its weights go
                 if (pend && !finish()) return running = false;
-                load_weights(Pi, S, g, coord, h, lane_addr);
+                // Pi, then S, staged transposed through shared memory
+                for (int mat = 0; mat < 2; ++mat) {
+                    if (!epi_sync()) return running = give_up(abort, err, 13);
+                    stage_transposed((mat == 0 ? Pi : S) + (size_t)g * kD * kD, stage, te);
+                    if (!epi_sync()) return running = give_up(abort, err, 14);
+                    pieces_to_tmem(stage, mat == 0, coord, wmask, lane_addr);
+                }
+                if (!epi_sync()) return running = give_up(abort, err, 15);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -495,18 +550,18 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             if (!warp_wait(&sm.d1_full[b], (i >> 1) & 1, abort))
                 return running = give_up(abort, err, 7);
             tc_fence_after();
-            uint32_t acc[32];
-            tmem_ld32(lane_addr + kColD1 + 64u * b + 32u * h, acc);
+            uint32_t acc[V];
+            tmem_ldv<V>(lane_addr + kColD1 + 64u * b + (uint32_t)(V * h), acc);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.d1_empty[b]);
             if (!warp_wait(&sm.norm_full[s], (i / kXS) & 1, abort))
                 return running = give_up(abort, err, 8);
-            float inv[32];
+            float inv[V];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 t4 = *reinterpret_cast<const float4*>(&sm.inv[s][32 * h + j]);
+            for (int j = 0; j < V; j += 4) {
+                const float4 t4 = *reinterpret_cast<const float4*>(&sm.inv[s][V * h + j]);
                 inv[j] = t4.x;
                 inv[j + 1] = t4.y;
                 inv[j + 2] = t4.z;
@@ -515,11 +570,13 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty_x[s]);
 
-            uint32_t ccur[4] = {0u, 0u, 0u, 0u};
-            float rr[32];
-            uint32_t hp1[16], hp2[16];
+            uint32_t ccur[V / 8];
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
+            for (int u = 0; u < V / 8; ++u) ccur[u] = 0u;
+            float rr[V];
+            uint32_t hp1[V / 2], hp2[V / 2];
+#pragma unroll
+            for (int j = 0; j < V; j += 2) {
                 float sr[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
@@ -549,16 +606,17 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             uint8_t* r0 = sm.r[b][0];
             uint8_t* r1 = sm.r[b][1];
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
+            for (int ii = 0; ii < V / 8; ++ii) {
                 *reinterpret_cast<uint4*>(r0 + roff[ii]) =
                     make_uint4(hp1[4 * ii], hp1[4 * ii + 1], hp1[4 * ii + 2], hp1[4 * ii + 3]);
                 *reinterpret_cast<uint4*>(r1 + roff[ii]) =
                     make_uint4(hp2[4 * ii], hp2[4 * ii + 1], hp2[4 * ii + 2], hp2[4 * ii + 3]);
             }
+            const float tot = transpose_reduce<V>(rr, lane);
+            if (lane < V) sm.rr[b][q][V * h + lane] = tot;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.r_full);
-            sm.rr[b][q][32 * h + lane] = transpose_reduce32(rr, lane);
 
             if (pend && !finish()) return running = false;
             pend = true;
@@ -566,7 +624,7 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             pt = t;
             pidx = i;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) pcell[u] = ccur[u];
+            for (int u = 0; u < V / 8; ++u) pcell[u] = ccur[u];
             ++i;
             return true;
         });
