@@ -91,54 +91,129 @@ def make_inputs(cfg, device, seed_offset=0, max_rows=None):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling every 50 ms in the background."""
+    """SM clock and clock-event (throttle) reasons sampled every 5 ms in a
+    background thread through NVML (the library behind nvidia-smi); falls back
+    to `nvidia-smi -lms 50` when NVML is unavailable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index):
-        self.index = index
-        self.rows = []
+    def __init__(self, device):
+        self.device = device
+        self.rows = []        # (time, sm_mhz, sm_max_mhz, reason names)
         self.proc = None
         self.t = None
+        self.stop_ev = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            idx = self.device.index if self.device.index is not None else 0
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                idx = int(vis.split(",")[idx])
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(idx)
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def loop():
+                while not self.stop_ev.is_set():
+                    try:
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        bits = int(get_reasons(h))
+                    except Exception:
+                        break
+                    names = [n for b, n in self.REASONS.items() if bits & b]
+                    self.rows.append((time.time(), sm, mx, names))
+                    self.stop_ev.wait(0.005)
+
+            self.source = "nvml 5 ms"
+            self.t = threading.Thread(target=loop, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.device.index or 0), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
-        self.t = threading.Thread(target=self._read, daemon=True)
+        self.source = "nvidia-smi 50 ms"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+        def read():
+            for line in self.proc.stdout:
+                r = [c.strip() for c in line.split(",")]
+                if len(r) < 9 or not r[1].replace(".", "").isdigit():
+                    continue
+                self.rows.append((time.time(), float(r[1]),
+                                  float(r[2]) if r[2].replace(".", "").isdigit() else None,
+                                  [names[i] for i in range(4) if r[5 + i] == "Active"]))
+
+        self.t = threading.Thread(target=read, daemon=True)
         self.t.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+    def wait_first(self, timeout=5.0):
+        """Block until the first sample is in (so the timed region is covered)."""
+        t_end = time.time() + timeout
+        while not self.rows and time.time() < t_end and (self.t and self.t.is_alive()):
+            time.sleep(0.01)
 
     def stop(self):
+        self.stop_ev.set()
         if self.proc:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.t:
-                self.t.join(timeout=2)
+        if self.t:
+            self.t.join(timeout=2)
 
     def summary(self, t0, t1):
-        rows = [r for (ts, r) in self.rows if t0 <= ts <= t1 and len(r) >= 9]
+        rows = [r for r in self.rows if t0 <= r[0] <= t1]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "source": self.source}
+        sm = [r[1] for r in rows]
+        mx = [r[2] for r in rows if r[2] is not None]
+        reasons = sorted({n for r in rows for n in r[3]})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "source": self.source,
+                "window": "timed region"}
+
+
+# ---------------------------------------------------------------- ranks
+def rank_max(dist, values, device):
+    """Max over ranks of each value: a multi-GPU time is the slowest rank's."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank, world, steps, total_ms):
+    """Whole-job Mvec/s: the units every rank processed over `steps` steps,
+    divided by the (max-over-ranks) device time."""
+    return units_per_rank * world * steps / (total_ms / 1e3) / 1e6
 
 
 # ---------------------------------------------------------------- our arm
@@ -225,10 +300,9 @@ def run_ours(args, cfg, rank, world, dist):
 
     nlaunch, kernel_names = count_launches(step) if not args.no_count else (None, [])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler = ClockSampler(dev)
     sampler.start()
-    time.sleep(0.2)
-    tw = time.time()  # clocks are summarised over warm-up + timed steps (GPU under load)
+    sampler.wait_first()
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
@@ -249,16 +323,11 @@ def run_ours(args, cfg, rank, world, dist):
     sco = [e[1].elapsed_time(e[2]) for e in evs]
     tpk = [e[2].elapsed_time(e[3]) for e in evs]
     tot_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
-    if dist:
-        t = torch.tensor([tot_ms, sum(enc), sum(sco), sum(tpk)], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        tot_ms, se, ss, st = t.tolist()
-    else:
-        se, ss, st = sum(enc), sum(sco), sum(tpk)
+    tot_ms, se, ss, st = rank_max(dist, [tot_ms, sum(enc), sum(sco), sum(tpk)], dev)
     K_ = args.steps
     ms_step = tot_ms / K_
     units = cfg["G"] * cfg["n"] * world
-    value = units * K_ / (tot_ms / 1e3) / 1e6
+    value = job_throughput(cfg["G"] * cfg["n"], world, K_, tot_ms)
 
     # e2e: host (pinned) inputs -> device, the same path through the public API,
     # results back to pinned host buffers, every step.
@@ -300,11 +369,7 @@ def run_ours(args, cfg, rank, world, dist):
         e2e_once()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = rank_max(dist, [e0.elapsed_time(e1) / e2e_steps], dev)[0]
     h2d = xh.numel() * xh.element_size() + qh.numel() * qh.element_size()
     d2h = sum(t.numel() * t.element_size() for t in (ch, xnh, rnh, sh, tvh, tih) if t is not None)
 
@@ -352,7 +417,7 @@ def run_ours(args, cfg, rank, world, dist):
         "gpu_launches": (nlaunch * K_) if nlaunch is not None else None,
         "gpu_launches_per_step": nlaunch,
         "kernels": kernel_names,
-        "clocks": sampler.summary(tw, t1),
+        "clocks": sampler.summary(t0, t1),
         "peaks": pk,
     }
     if score_ms is not None:
@@ -453,7 +518,7 @@ def run_reference(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="kv", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

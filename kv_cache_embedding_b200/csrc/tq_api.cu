@@ -35,6 +35,10 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
         case TQ_OP_SCORE:
             return 2 * qbuf;
         case TQ_OP_TOPK:
+            if (topk_materialized(G, n, nq))  // scores, chunk maxima, counters, candidates
+                return 2 * qbuf + align256((size_t)G * nq * n * 4) +
+                       align256((size_t)G * nq * ntiles * 4) + align256((size_t)G * nq * 8) +
+                       2 * align256((size_t)G * nq * kTopkCandidates * 4);
             return 2 * qbuf + parts;
         case TQ_OP_DECODE:
             return 2 * align256((size_t)chunk * d * 4);

@@ -47,6 +47,15 @@ __device__ __forceinline__ bool better(float va, int64_t ia, float vb, int64_t i
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// tq_topk writes the whole score matrix (and per-chunk maxima) to its
+// workspace when it has at most this many scores, then selects per row; larger
+// searches run the fused score + running-list kernel instead.
+constexpr int64_t kTopkMaterialize = (int64_t)1 << 24;
+constexpr int kTopkCandidates = 4096;  // gathered candidates per row on that path
+inline bool topk_materialized(int G, int64_t n, int nq) {
+    return (int64_t)G * nq * n <= kTopkMaterialize;
+}
+
 inline bool valid_db(int d, int b) {
     return d >= kMinD && d <= kMaxD && d % 128 == 0 && b >= 1 && b <= 4;
 }

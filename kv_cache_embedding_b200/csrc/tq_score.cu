@@ -172,9 +172,12 @@ __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ cod
                                                 const float* __restrict__ rnorm, int64_t n, int d,
                                                 int nq, const float* __restrict__ qr,
                                                 const float* __restrict__ u, KCodebook cb,
-                                                float* __restrict__ scores) {
+                                                float* __restrict__ scores,
+                                                float* __restrict__ cmax, int nchunks,
+                                                int* __restrict__ zero_cnt) {
     extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d] pairs (qr_i, u_i)
     __shared__ float2 s_tab[16];
+    __shared__ float s_max[4][NQ];
     const int g = blockIdx.y;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
@@ -199,6 +202,9 @@ __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ cod
 
     score_keys<B, NQ, KP, F2>(rec, d, s_qu, s_tab, acc);
     const float k0 = kSqrtHalfPi / (float)d;
+    float mx[NQ];
+#pragma unroll
+    for (int qq = 0; qq < NQ; ++qq) mx[qq] = -INFINITY;
 #pragma unroll
     for (int k = 0; k < KP; ++k) {
         if (!ok[k]) continue;
@@ -207,9 +213,30 @@ __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ cod
         const float kap = k0 * rnorm[gv];
 #pragma unroll
         for (int qq = 0; qq < NQ; ++qq)
-            if (qq < qn)
-                scores[((int64_t)g * nq + q0 + qq) * n + v[k]] =
-                    xn * (acc[k][qq].x + kap * acc[k][qq].y);
+            if (qq < qn) {
+                const float sc = xn * (acc[k][qq].x + kap * acc[k][qq].y);
+                scores[((int64_t)g * nq + q0 + qq) * n + v[k]] = sc;
+                mx[qq] = fmaxf(mx[qq], sc);
+            }
+    }
+    if (zero_cnt && blockIdx.x == 0 && threadIdx.x < 2 * qn)  // top-k counters of these rows
+        zero_cnt[(threadIdx.x & 1) * (int64_t)gridDim.y * nq + (int64_t)g * nq + q0 +
+                 (threadIdx.x >> 1)] = 0;
+    if (cmax) {  // the block's 128 KP keys form one chunk: its maximum per query
+        const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                mx[qq] = fmaxf(mx[qq], __shfl_xor_sync(0xffffffffu, mx[qq], o));
+            if (lane == 0) s_max[warp][qq] = mx[qq];
+        }
+        __syncthreads();
+        if (threadIdx.x < qn) {
+            const int qq = threadIdx.x;
+            const float m = fmaxf(fmaxf(s_max[0][qq], s_max[1][qq]), fmaxf(s_max[2][qq], s_max[3][qq]));
+            cmax[((int64_t)g * nq + q0 + qq) * nchunks + blockIdx.x] = m;
+        }
     }
 }
 
@@ -248,63 +275,249 @@ __device__ void warp_select(float* s, int count, int64_t id0, int K, float* vals
     }
 }
 
-// grid: (tiles of kTopkTile keys, G, query passes of NQ <= 8); 256 threads,
-// KP = 4 keys each.  Scores of the tile go to shared memory, then warp q
-// selects the tile's best K for query q0 + q into part_vals/part_ids
-// [G][nq][ntiles][K].
+// ---- running top-k lists ---------------------------------------------------
+// A warp keeps a sorted list of the best K (K <= 32) (value, id) pairs seen so
+// far in registers: lane r holds the r-th best by (value desc, id asc); empty
+// slots hold (-inf, none).  New entries are screened against the K-th best with
+// one ballot; the rare ones that beat it are inserted one at a time.
+constexpr int kCandTile = 256;  // keys scored per pass of a block (thread = key)
+static_assert(kCandTile == kTopkTile, "key ranges are bounded by the top-k workspace tiles");
+
+template <typename Id>
+__device__ __forceinline__ bool better_t(float va, Id ia, float vb, Id ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+template <typename Id>
+__device__ __forceinline__ Id id_none() {
+    // INT64_MAX, INT32_MAX, UINT32_MAX
+    return (Id)(~(uint64_t)0 >> (sizeof(Id) == 8 ? 1 : ((Id)-1 < (Id)0 ? 33 : 32)));
+}
+
+template <typename Id>
+struct WarpList {
+    float v;     // this lane's slot
+    Id id;
+    float kv;    // the K-th best (same on every lane)
+    Id kid;
+
+    __device__ __forceinline__ void init() {
+        v = -INFINITY;
+        id = id_none<Id>();
+        kv = -INFINITY;
+        kid = id_none<Id>();
+    }
+    // Offer every lane's (cv, cid) where `want`; warp-uniform call.
+    __device__ __forceinline__ void offer(bool want, float cv, Id cid, int K, int lane) {
+        uint32_t m = __ballot_sync(0xffffffffu, want && better_t(cv, cid, kv, kid));
+        while (m) {
+            const int src = __ffs(m) - 1;
+            m &= m - 1;
+            const float nv = __shfl_sync(0xffffffffu, cv, src);
+            const Id nid = __shfl_sync(0xffffffffu, cid, src);
+            if (!better_t(nv, nid, kv, kid)) continue;  // the list moved on meanwhile
+            // position = number of kept entries better than the new one
+            const int p = __popc(__ballot_sync(0xffffffffu, lane < K && better_t(v, id, nv, nid)));
+            const float uv = __shfl_up_sync(0xffffffffu, v, 1);
+            const Id uid = __shfl_up_sync(0xffffffffu, id, 1);
+            if (lane == p) {
+                v = nv;
+                id = nid;
+            } else if (lane > p && lane < K) {
+                v = uv;
+                id = uid;
+            }
+            kv = __shfl_sync(0xffffffffu, v, K - 1);
+            kid = __shfl_sync(0xffffffffu, id, K - 1);
+        }
+    }
+};
+
+// grid: (nblk key ranges of `span` keys, G, query passes of NQ <= 8); 256
+// threads, thread = key.  Each warp keeps a running best-K list per query
+// over the keys it scores; at the end the block's 8 lists per query are
+// combined in shared memory.  Output: the range's best K per query (value,
+// global key id; -inf / INT64_MAX where the range has fewer) in
+// part_vals/part_ids [G][nq][nblk][K].
 template <int B, int NQ, bool F2>
-__global__ __launch_bounds__(256) void k_score_topk_tile(
+__global__ __launch_bounds__(256) void k_score_topk(
     const uint32_t* __restrict__ codes, const float* __restrict__ xnorm,
     const float* __restrict__ rnorm, int64_t n, int d, int nq, const float* __restrict__ qr,
-    const float* __restrict__ u, KCodebook cb, int K, int ntiles, float* __restrict__ part_vals,
-    int64_t* __restrict__ part_ids) {
-    constexpr int KP = kTopkTile / 256;
-    extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d], then scores [NQ][kTopkTile]
-    float* s_sc = reinterpret_cast<float*>(s_qu + NQ * d);
+    const float* __restrict__ u, KCodebook cb, int K, int nblk, int64_t span,
+    float* __restrict__ part_vals, int64_t* __restrict__ part_ids) {
+    extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d]
     __shared__ float2 s_tab[16];
+    __shared__ float s_lv[NQ][8][kMaxK];
+    __shared__ uint32_t s_li[NQ][8][kMaxK];
     const int g = blockIdx.y;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
-    const int64_t t0 = (int64_t)blockIdx.x * kTopkTile;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t kb0 = (int64_t)blockIdx.x * span;
+    const int64_t kb1 = min(n, kb0 + span);
     load_score_smem<B, NQ>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
     __syncthreads();
     const int W = words_per_vector(d, B);
-    int64_t v[KP];
-    bool ok[KP];
-    const uint32_t* rec[KP];
-#pragma unroll
-    for (int k = 0; k < KP; ++k) {
-        v[k] = t0 + k * 256 + threadIdx.x;
-        ok[k] = v[k] < n;
-        rec[k] = codes + ((int64_t)g * n + (ok[k] ? v[k] : 0)) * W;
-    }
-    float2 acc[KP][NQ];
-#pragma unroll
-    for (int k = 0; k < KP; ++k)
-#pragma unroll
-        for (int qq = 0; qq < NQ; ++qq) acc[k][qq] = make_float2(0.f, 0.f);
-    score_keys<B, NQ, KP, F2>(rec, d, s_qu, s_tab, acc);
     const float k0 = kSqrtHalfPi / (float)d;
+    WarpList<uint32_t> L[NQ];
 #pragma unroll
-    for (int k = 0; k < KP; ++k) {
-        const int e = k * 256 + threadIdx.x;
-        if (ok[k]) {
-            const int64_t gv = (int64_t)g * n + v[k];
-            const float xn = xnorm[gv];
-            const float kap = k0 * rnorm[gv];
+    for (int qq = 0; qq < NQ; ++qq) L[qq].init();
+    for (int64_t t0 = kb0; t0 < kb1; t0 += kCandTile) {
+        const int64_t v = t0 + threadIdx.x;
+        const bool ok = v < kb1;
+        const int64_t gv = (int64_t)g * n + (ok ? v : kb0);
+        const uint32_t* rec[1] = {codes + gv * W};
+        float2 acc[1][NQ];
 #pragma unroll
-            for (int qq = 0; qq < NQ; ++qq)
-                s_sc[qq * kTopkTile + e] = xn * (acc[k][qq].x + kap * acc[k][qq].y);
-        } else {
+        for (int qq = 0; qq < NQ; ++qq) acc[0][qq] = make_float2(0.f, 0.f);
+        score_keys<B, NQ, 1, F2>(rec, d, s_qu, s_tab, acc);
+        const float xn = xnorm[gv];
+        const float kap = k0 * rnorm[gv];
 #pragma unroll
-            for (int qq = 0; qq < NQ; ++qq) s_sc[qq * kTopkTile + e] = -INFINITY;
+        for (int qq = 0; qq < NQ; ++qq)
+            L[qq].offer(ok && qq < qn, xn * (acc[0][qq].x + kap * acc[0][qq].y),
+                        (uint32_t)(v - kb0), K, lane);
+    }
+#pragma unroll
+    for (int qq = 0; qq < NQ; ++qq)
+        if (lane < K) {
+            s_lv[qq][warp][lane] = L[qq].v;
+            s_li[qq][warp][lane] = L[qq].id;
+        }
+    __syncthreads();
+    if (warp < qn) {
+        WarpList<uint32_t> M;
+        M.init();
+        for (int w = 0; w < 8; ++w)
+            M.offer(lane < K, s_lv[warp][w][lane], s_li[warp][w][lane], K, lane);
+        const int64_t o = (((int64_t)g * nq + q0 + warp) * nblk + blockIdx.x) * K;
+        if (lane < K) {
+            const bool have = M.id != id_none<uint32_t>();
+            part_vals[o + lane] = have ? M.v : -INFINITY;
+            part_ids[o + lane] = have ? kb0 + (int64_t)M.id : INT64_MAX;
         }
     }
+}
+
+// Top-K of rows of materialised scores.  grid: (P blocks per row, rows); 256
+// threads.  Every warp derives the same threshold t on its own: the chunk
+// maxima (one per kTopkTile keys) are folded by max into 64 slots (two per
+// lane), sorted across the warp, and t is the K-th largest slot -- K slots,
+// hence K scores, are >= t, so the whole top K is.  Each block then scans its
+// share of the row and appends the scores >= t to the row's candidate list in
+// global memory.  The last block of a row to finish (a counter, no waiting)
+// selects the best K from the list, or from the whole row if the list
+// overflowed (massive ties).  The counters are zeroed by the score kernel that
+// writes the row.
+constexpr int kCandCapG = kTopkCandidates;  // candidate entries per row
+
+// Descending bitonic sort of 64 values held two per lane (slot 2 * lane + h
+// in v[h]).
+__device__ __forceinline__ void warp_sort64_desc(float (&v)[2], int lane) {
+    for (int k = 2; k <= 64; k <<= 1) {
+        const bool desc = ((2 * lane) & k) == 0;  // direction of this slot's run
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j == 1) {  // partner slot in the same lane
+                const float hi = fmaxf(v[0], v[1]), lo = fminf(v[0], v[1]);
+                v[0] = desc ? hi : lo;
+                v[1] = desc ? lo : hi;
+            } else {
+                const bool lower = (lane & (j >> 1)) == 0;  // bit j of the slot index
+                const bool keep_max = lower == desc;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[h], j >> 1);
+                    v[h] = keep_max ? fmaxf(v[h], o) : fminf(v[h], o);
+                }
+            }
+        }
+    }
+}
+
+__global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict__ scores,
+                                                      const float* __restrict__ cmax, int64_t n,
+                                                      int nchunks, int K, int* cand_cnt, int* done,
+                                                      float* cand_v, int* cand_i,
+                                                      float* __restrict__ vals,
+                                                      int64_t* __restrict__ ids) {
+    __shared__ int s_last;
+    const int64_t row = blockIdx.y;
+    const int P = gridDim.x;
+    const int lane = threadIdx.x % 32;
+    const float* sr = scores + row * n;
+    const float* cm = cmax + row * nchunks;
+    float f[2] = {-INFINITY, -INFINITY};
+    for (int c = lane; c < nchunks; c += 64) {
+        f[0] = fmaxf(f[0], cm[c]);
+        if (c + 32 < nchunks) f[1] = fmaxf(f[1], cm[c + 32]);
+    }
+    warp_sort64_desc(f, lane);
+    // the K-th largest slot (-inf when fewer than K chunks)
+    const float thr = __shfl_sync(0xffffffffu, ((K - 1) & 1) ? f[1] : f[0], (K - 1) >> 1);
+    const int64_t per = (n + P - 1) / P;
+    const int64_t e0 = (int64_t)blockIdx.x * per;
+    const int64_t e1 = min(n, e0 + per);
+    float* cv = cand_v + row * kCandCapG;
+    int* ci = cand_i + row * kCandCapG;
+    constexpr int U = 16;
+    for (int64_t base = e0; base < e1; base += (int64_t)U * blockDim.x) {
+        float v[U];
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int64_t e = base + (int64_t)j * blockDim.x + threadIdx.x;
+            v[j] = e < e1 ? sr[e] : -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int64_t e = base + (int64_t)j * blockDim.x + threadIdx.x;
+            const bool pass = e < e1 && v[j] >= thr;
+            const uint32_t m = __ballot_sync(0xffffffffu, pass);
+            if (m) {
+                const int leader = __ffs(m) - 1;
+                int pos0 = 0;
+                if (lane == leader) pos0 = atomicAdd(&cand_cnt[row], __popc(m));
+                pos0 = __shfl_sync(0xffffffffu, pos0, leader);
+                const int pos = pos0 + __popc(m & ((1u << lane) - 1u));
+                if (pass && pos < kCandCapG) {
+                    cv[pos] = v[j];
+                    ci[pos] = (int)e;
+                }
+            }
+        }
+    }
+    // the last block of the row selects
+    __threadfence();
     __syncthreads();
-    const int warp = threadIdx.x / 32;
-    if (warp < qn) {
-        const int64_t o = (((int64_t)g * nq + q0 + warp) * ntiles + blockIdx.x) * K;
-        warp_select(s_sc + warp * kTopkTile, kTopkTile, t0, K, part_vals + o, part_ids + o);
+    if (threadIdx.x == 0) s_last = (atomicAdd(&done[row], 1) == P - 1);
+    __syncthreads();
+    if (!s_last || threadIdx.x >= 32) return;
+    __threadfence();
+    const int cnt = __ldcg(&cand_cnt[row]);
+    WarpList<int> L;
+    L.init();
+    if (cnt <= kCandCapG) {
+        constexpr int C = 8;
+        for (int c0 = 0; c0 < cnt; c0 += 32 * C) {
+            float cvv[C];
+            int cii[C];
+#pragma unroll
+            for (int j = 0; j < C; ++j) {
+                const int c = c0 + 32 * j + lane;
+                cvv[j] = c < cnt ? __ldcg(&cv[c]) : -INFINITY;
+                cii[j] = c < cnt ? __ldcg(&ci[c]) : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < C; ++j) L.offer(c0 + 32 * j + lane < cnt, cvv[j], cii[j], K, lane);
+        }
+    } else {
+        for (int64_t f0 = 0; f0 < n; f0 += 32) {
+            const int64_t e = f0 + lane;
+            L.offer(e < n, e < n ? sr[e] : -INFINITY, (int)e, K, lane);
+        }
+    }
+    if (lane < K) {
+        const bool have = L.id != id_none<int>();
+        vals[row * K + lane] = have ? L.v : -INFINITY;
+        ids[row * K + lane] = have ? (int64_t)L.id : INT64_MAX;
     }
 }
 
@@ -327,64 +540,38 @@ __global__ __launch_bounds__(256) void k_rows_topk_tile(const float* __restrict_
     }
 }
 
-// Merge [rows][ntiles][K] partial lists into the final K per row.
-// One block (256 threads) per row; K rounds of block-wide arg-max.
-__global__ __launch_bounds__(256) void k_topk_merge(float* __restrict__ part_vals,
-                                                    int64_t* __restrict__ part_ids, int ntiles,
-                                                    int K, float* __restrict__ vals,
+// Merge [rows][nparts][K] partial lists (missing entries: id INT64_MAX) into
+// the final K per row.  One warp per row (4 rows per 128-thread block): the
+// entries stream through a running best-K list, 16 per lane loaded ahead.
+__global__ __launch_bounds__(128) void k_topk_merge(const float* __restrict__ part_vals,
+                                                    const int64_t* __restrict__ part_ids,
+                                                    int64_t rows, int nparts, int K,
+                                                    float* __restrict__ vals,
                                                     int64_t* __restrict__ ids) {
-    __shared__ float s_v[8];
-    __shared__ int64_t s_i[8];
-    __shared__ int64_t s_pos[8];
-    const int64_t row = blockIdx.x;
-    float* pv = part_vals + row * ntiles * K;
-    int64_t* pi = part_ids + row * ntiles * K;
-    const int count = ntiles * K;
-    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
-    for (int r = 0; r < K; ++r) {
-        float bv = -INFINITY;
-        int64_t bid = INT64_MAX, bpos = -1;
-        for (int e = threadIdx.x; e < count; e += blockDim.x) {
-            const int64_t id = pi[e];
-            if (id == INT64_MAX) continue;
-            const float v = pv[e];
-            if (better(v, id, bv, bid)) {
-                bv = v;
-                bid = id;
-                bpos = e;
-            }
+    constexpr int C = 16;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+    if (row >= rows) return;
+    const float* pv = part_vals + row * nparts * K;
+    const int64_t* pi = part_ids + row * nparts * K;
+    const int64_t count = (int64_t)nparts * K;
+    WarpList<int64_t> L;
+    L.init();
+    for (int64_t base = 0; base < count; base += 32 * C) {
+        float v[C];
+        int64_t id[C];
+#pragma unroll
+        for (int j = 0; j < C; ++j) {
+            const int64_t e = base + 32 * j + lane;
+            v[j] = e < count ? pv[e] : -INFINITY;
+            id[j] = e < count ? pi[e] : INT64_MAX;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int64_t oid = __shfl_xor_sync(0xffffffffu, bid, o);
-            const int64_t op = __shfl_xor_sync(0xffffffffu, bpos, o);
-            if (better(ov, oid, bv, bid)) {
-                bv = ov;
-                bid = oid;
-                bpos = op;
-            }
-        }
-        if (lane == 0) {
-            s_v[warp] = bv;
-            s_i[warp] = bid;
-            s_pos[warp] = bpos;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            float v = s_v[0];
-            int64_t id = s_i[0], pos = s_pos[0];
-            for (int w = 1; w < 8; ++w)
-                if (better(s_v[w], s_i[w], v, id)) {
-                    v = s_v[w];
-                    id = s_i[w];
-                    pos = s_pos[w];
-                }
-            vals[row * K + r] = v;
-            ids[row * K + r] = id;
-            if (pos >= 0) pi[pos] = INT64_MAX;
-        }
-        __syncthreads();
+        for (int j = 0; j < C; ++j) L.offer(id[j] != INT64_MAX, v[j], id[j], K, lane);
+    }
+    if (lane < K) {
+        vals[row * K + lane] = L.v;
+        ids[row * K + lane] = L.id;
     }
 }
 
@@ -485,14 +672,16 @@ __global__ __launch_bounds__(256) void k_logits_fp32(const float* __restrict__ k
 template <int B, int NQ, bool F2>
 int launch_score2_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                     int G, int nq, const float* qr, const float* u, const KCodebook& kc,
-                    float* scores, cudaStream_t s) {
+                    float* scores, float* cmax, int* zero_cnt, cudaStream_t s) {
     constexpr int KP = 2;
+    static_assert(128 * KP == kTopkTile, "one score block per top-k chunk");
     const size_t smem = (size_t)NQ * d * sizeof(float2);
     TQ_TRY_CUDA(cudaFuncSetAttribute(k_score2<B, NQ, KP, F2>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    dim3 grid((unsigned)((n + 128 * KP - 1) / (128 * KP)), (unsigned)G,
-              (unsigned)((nq + NQ - 1) / NQ));
-    k_score2<B, NQ, KP, F2><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores);
+    const int nchunks = (int)((n + 128 * KP - 1) / (128 * KP));
+    dim3 grid((unsigned)nchunks, (unsigned)G, (unsigned)((nq + NQ - 1) / NQ));
+    k_score2<B, NQ, KP, F2><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores,
+                                                    cmax, nchunks, zero_cnt);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -505,21 +694,13 @@ int score_nq(int d, int nq) {
     return p;
 }
 
-// packed f32x2 accumulation (sm_100 fma.rn.f32x2); TQ_SCORE_FFMA2=0 selects plain FFMA
-const bool g_score_f2 = [] {
-    const char* e = getenv("TQ_SCORE_FFMA2");
-    return !(e && e[0] == '0');
-}();
-
 template <int B>
 int launch_score_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                    int G, int nq, const float* qr, const float* u, const KCodebook& kc,
-                   float* scores, cudaStream_t s) {
-#define TQ_SC(NQV)                                                                          \
-    return g_score_f2 ? launch_score2_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
-                                                      scores, s)                            \
-                      : launch_score2_t<B, NQV, false>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
-                                                       scores, s)
+                   float* scores, float* cmax, int* zero_cnt, cudaStream_t s) {
+#define TQ_SC(NQV) \
+    return launch_score2_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, cmax, \
+                                         zero_cnt, s)
     switch (score_nq(d, nq)) {
         case 1: TQ_SC(1);
         case 2: TQ_SC(2);
@@ -529,16 +710,35 @@ int launch_score_b(const uint32_t* codes, const float* xn, const float* rn, int6
 #undef TQ_SC
 }
 
+// Key ranges per (group, query pass) for k_score_topk: enough blocks for one
+// full wave of the device, each range a whole number of kCandTile passes.
+struct TopkGrid {
+    int nblk;
+    int64_t span;
+};
+
 template <int B, int NQ, bool F2>
 int launch_topk_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
-                  int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
-    const size_t smem = (size_t)NQ * d * sizeof(float2) + (size_t)NQ * kTopkTile * sizeof(float);
-    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score_topk_tile<B, NQ, F2>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    dim3 grid((unsigned)ntiles, (unsigned)G, (unsigned)((nq + NQ - 1) / NQ));
-    k_score_topk_tile<B, NQ, F2><<<grid, 256, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, K,
-                                                          ntiles, pv, pi);
+                  float* pv, int64_t* pi, TopkGrid* out, cudaStream_t s) {
+    const size_t smem = (size_t)NQ * d * sizeof(float2);
+    auto kern = k_score_topk<B, NQ, F2>;
+    TQ_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    int dev = 0, nsm = 0, occ = 0;
+    TQ_TRY_CUDA(cudaGetDevice(&dev));
+    TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    TQ_TRY_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 256, smem));
+    const int npass = (nq + NQ - 1) / NQ;
+    const int64_t passes = (n + kCandTile - 1) / kCandTile;  // kCandTile-key passes per group
+    int64_t want = (int64_t)nsm * (occ > 0 ? occ : 1) / ((int64_t)G * npass);
+    want = want < 1 ? 1 : (want > passes ? passes : want);
+    const int64_t per = (passes + want - 1) / want;  // passes per block
+    TopkGrid tg;
+    tg.span = per * kCandTile;
+    tg.nblk = (int)((n + tg.span - 1) / tg.span);
+    *out = tg;
+    dim3 grid((unsigned)tg.nblk, (unsigned)G, (unsigned)npass);
+    kern<<<grid, 256, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, K, tg.nblk, tg.span, pv, pi);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -546,12 +746,9 @@ int launch_topk_t(const uint32_t* codes, const float* xn, const float* rn, int64
 template <int B>
 int launch_topk_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
-                  int ntiles, float* pv, int64_t* pi, cudaStream_t s) {
-#define TQ_TK(NQV)                                                                              \
-    return g_score_f2 ? launch_topk_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, K,    \
-                                                    ntiles, pv, pi, s)                          \
-                      : launch_topk_t<B, NQV, false>(codes, xn, rn, n, d, G, nq, qr, u, kc, K,   \
-                                                     ntiles, pv, pi, s)
+                  float* pv, int64_t* pi, TopkGrid* tg, cudaStream_t s) {
+#define TQ_TK(NQV) \
+    return launch_topk_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, pv, pi, tg, s)
     switch (score_nq(d, nq)) {
         case 1: TQ_TK(1);
         case 2: TQ_TK(2);
@@ -682,10 +879,10 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     if (rc) return rc;
     const KCodebook kc = make_kcodebook(cb);
     switch (b) {
-        case 1: return launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
-        case 2: return launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
-        case 3: return launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
-        default: return launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, s);
+        case 1: return launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
+        case 2: return launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
+        case 3: return launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
+        default: return launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
     }
 }
 
@@ -710,20 +907,57 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
     p += align256((size_t)G * nq * d * 4);
     float* u = (float*)p;
     p += align256((size_t)G * nq * d * 4);
-    float* pv = (float*)p;
-    p += align256((size_t)G * nq * ntiles * k * 4);
-    int64_t* pi = (int64_t*)p;
     rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
     if (rc) return rc;
     const KCodebook kc = make_kcodebook(cb);
+    const int64_t rows = (int64_t)G * nq;
+    if (topk_materialized(G, n, nq)) {
+        // scores [G][nq][n] and chunk maxima [G][nq][ntiles], then per-row selection
+        float* sc = (float*)p;
+        p += align256((size_t)rows * n * 4);
+        float* cm = (float*)p;
+        p += align256((size_t)rows * ntiles * 4);
+        int* cnt = (int*)p;  // [2][rows]: candidate counts, finished blocks
+        p += align256((size_t)rows * 2 * 4);
+        float* cv = (float*)p;
+        p += align256((size_t)rows * kCandCapG * 4);
+        int* ci = (int*)p;
+        switch (b) {
+            case 1: rc = launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+            case 2: rc = launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+            case 3: rc = launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+            default: rc = launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+        }
+        if (rc) return rc;
+        int nsm = 0, dev = 0;
+        TQ_TRY_CUDA(cudaGetDevice(&dev));
+        TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+        // blocks per row: 16 scores per thread (one pass of loads), more when
+        // the rows alone would leave most SMs idle
+        int64_t P = (n + 256 * 16 - 1) / (256 * 16);
+        const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
+        const int64_t pmax = (n + 255) / 256;
+        P = P < pmin ? pmin : P;
+        P = P > pmax ? pmax : P;
+        dim3 grid((unsigned)P, (unsigned)rows);
+        k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, n, ntiles, k, cnt, cnt + rows, cv, ci, d_vals,
+                                             d_ids);
+        TQ_CHECK_LAUNCH();
+        return TQ_OK;
+    }
+    // fused: per-range best-K lists [G][nq][nblk][K], then the merge
+    float* pv = (float*)p;
+    p += align256((size_t)rows * ntiles * k * 4);
+    int64_t* pi = (int64_t*)p;
+    TopkGrid tg;
     switch (b) {
-        case 1: rc = launch_topk_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
-        case 2: rc = launch_topk_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
-        case 3: rc = launch_topk_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
-        default: rc = launch_topk_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, ntiles, pv, pi, s); break;
+        case 1: rc = launch_topk_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, pv, pi, &tg, s); break;
+        case 2: rc = launch_topk_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, pv, pi, &tg, s); break;
+        case 3: rc = launch_topk_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, pv, pi, &tg, s); break;
+        default: rc = launch_topk_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, pv, pi, &tg, s); break;
     }
     if (rc) return rc;
-    k_topk_merge<<<(unsigned)(G * nq), 256, 0, s>>>(pv, pi, ntiles, k, d_vals, d_ids);
+    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, tg.nblk, k, d_vals, d_ids);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -854,7 +1088,8 @@ extern "C" int tq_exact_topk(int d, int G, int64_t n, const float* d_x, int nq, 
             TQ_CHECK_LAUNCH();
         }
     }
-    k_topk_merge<<<(unsigned)(G * nq), 256, 0, s>>>(pv, pi, ntiles, k, d_vals, d_ids);
+    const int64_t rows = (int64_t)G * nq;
+    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, ntiles, k, d_vals, d_ids);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }

@@ -76,3 +76,18 @@ def sample_rows(n, count, seed=3):
     g = _gen(seed, "cpu")
     count = min(count, n)
     return torch.randperm(n, generator=g)[:count].sort().values
+
+
+def random_records(n, words, seed=11, norm_range=(0.5, 2.0), rnorm_range=(0.0, 0.5)):
+    """Uniformly random code records for search tests that need no encoder:
+    `words` uint32 words per record (every bit pattern is a valid record of
+    the packed layouts), plus per-record norms.  Returns (codes [n, words]
+    uint32 numpy, xnorm [n] fp32, rnorm [n] fp32) on the CPU."""
+    g = _gen(seed, "cpu")
+    w = torch.randint(0, 1 << 32, (n, words), generator=g, dtype=torch.int64)
+    lo, hi = norm_range
+    xn = torch.rand(n, generator=g) * (hi - lo) + lo
+    rlo, rhi = rnorm_range
+    rn = torch.rand(n, generator=g) * (rhi - rlo) + rlo
+    return (w.to(torch.int64).numpy().astype("uint32"), xn.numpy().astype("float32"),
+            rn.numpy().astype("float32"))

@@ -178,6 +178,66 @@ def test_topk(quant, oparams, tq_lib, cuda, n, k, nq):
                     float(xn.max()))
 
 
+@pytest.mark.parametrize("G,n,k,b", [(1, 400_000, 10, 4), (1, 400_000, 32, 2), (3, 150_001, 10, 3)])
+def test_topk_long_ranges(quant, oparams, tq_lib, cuda, G, n, k, b):
+    """Key ranges of many passes per block: the running threshold and the
+    candidate-buffer cuts of the fused score + top-k kernel are exercised."""
+    d, nq = 128, 4
+    W = b * d // 32
+    qs = synth.gaussian_rows(G * nq, d, seed=21, norm_range=None).reshape(G, nq, d)
+    recs = [synth.random_records(n, W, seed=30 + g) for g in range(G)]
+    codes = tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+    vals, ids = quant(d, b, 0, G).topk(codes, qs.cuda(), k)
+    for g in range(G):
+        c, xn, rn = recs[g]
+        s_ora = O.score(oparams(d, b, g), c, xn, rn, _f64(qs[g]))
+        PT.compare_topk(_np(vals[g]), _np(ids[g]), s_ora, k, np.linalg.norm(_f64(qs[g]), axis=1),
+                        float(xn.max()))
+
+
+@pytest.mark.parametrize("copies", [41, 5000])
+def test_topk_equal_scores_take_smallest_ids(quant, oparams, tq_lib, cuda, copies):
+    """Copies of the best record score exactly alike; the top-k keeps the
+    smallest ids among them (ties: id ascending).  5000 copies overflow the
+    gathered candidate set and take the full-row selection."""
+    d, b, n, nq, k = 128, 4, 300_000, 2, 10
+    c, xn, rn = synth.random_records(n, b * d // 32, seed=40)
+    q = synth.gaussian_rows(nq, d, seed=41, norm_range=None)
+    best = int(np.argmax(O.score(oparams(d, b, 0), c, xn, rn, _f64(q))[0]))
+    pos = np.sort(synth.sample_rows(n, copies, seed=42).numpy())
+    pos = pos[pos != best]
+    c[pos], xn[pos], rn[pos] = c[best], xn[best], rn[best]
+    copies = np.sort(np.append(pos, best))
+    vals, ids = quant(d, b).topk(_to_codes(tq_lib, c, xn, rn, cuda), q.cuda()[None], k)
+    np.testing.assert_array_equal(_np(ids[0])[0], copies[:k])
+    assert np.all(_np(vals[0])[0] == _np(vals[0])[0][0])
+
+
+def test_topk_fused_path(quant, oparams, tq_lib, cuda):
+    """More than 2^24 scores: the fused score + running-list kernel and the
+    merge of its per-range lists (instead of materialised scores)."""
+    d, b, n, nq, k = 128, 2, 2_200_000, 8, 10
+    c, xn, rn = synth.random_records(n, b * d // 32, seed=45)
+    q = synth.gaussian_rows(nq, d, seed=46, norm_range=None)
+    vals, ids = quant(d, b).topk(_to_codes(tq_lib, c, xn, rn, cuda), q.cuda()[None], k)
+    s_ora = O.score(oparams(d, b, 0), c, xn, rn, _f64(q))
+    PT.compare_topk(_np(vals[0]), _np(ids[0]), s_ora, k, np.linalg.norm(_f64(q), axis=1),
+                    float(xn.max()))
+
+
+def test_exact_topk_many_tiles(tq_lib, cuda):
+    """Thousands of partial lists per row through the merge."""
+    n, d, nq, k = 200_000, 128, 3, 10
+    x = synth.gaussian_rows(n, d, seed=43, unit=True)
+    q = synth.gaussian_rows(nq, d, seed=44, unit=True)
+    vals, ids = tq_lib.exact_topk(x.cuda()[None], q.cuda()[None], k)
+    ex = O.exact_scores(_f64(x), _f64(q))
+    PT.compare_topk(_np(vals[0]), _np(ids[0]), ex, k, np.ones(nq), 1.0)
+
+
 @pytest.mark.parametrize("b", [1, 3, 4])
 def test_decode(quant, oparams, tq_lib, cuda, b):
     d = 128
