@@ -55,6 +55,31 @@ CONFIGS = {
 
 FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 CUDA-core peak at max SM clock
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the dominant kernel, from one ncu capture of `python bench.py --steps 2
+# --warmup 3 --no-cpu-baseline --no-count` (summary under profiles/).  It is
+# reported only while the kernel's sources still hash to what was captured.
+NCU_TRAFFIC = {
+    ("kv", "k_encode_tc"): {
+        "sources": ["kv_cache_embedding_b200/csrc/tq_encode_tc.cu",
+                    "kv_cache_embedding_b200/csrc/tq_sm100.cuh"],
+        "sha1": "ab4b8235cd9123f4999844520f1ab4bc37aea169",
+        "bytes": 68257280 + 2632192,
+    },
+}
+
+
+def ncu_traffic(config, kernel):
+    import hashlib
+    rec = NCU_TRAFFIC.get((config, kernel))
+    if rec is None:
+        return None
+    h = hashlib.sha1()
+    for rel in rec["sources"]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return rec["bytes"] if h.hexdigest() == rec["sha1"] else None
+
 
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -386,7 +411,9 @@ def run_ours(args, cfg, rank, world, dist):
     if tc:
         peak = pk["bf16"] / 3.0
         roofline = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
-                    "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                    "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                    "traffic": ncu_traffic(args.config, "k_encode_tc"),
+                    "alg_bytes": ab["enc_bytes"],
                     "kernel": "k_encode_tc (tq_encode: rotation + QJL on tcgen05, 3 x 16-bit "
                               "passes per fp32-accurate product, fused epilogue)",
                     "peak_source": "measured bf16 burst (MEASURED_PEAKS.json) / 3 passes",
