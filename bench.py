@@ -61,9 +61,8 @@ FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 CUDA-core peak at max 
 # reported only while the kernel's sources still hash to what was captured.
 NCU_TRAFFIC = {
     ("kv", "k_encode_tc"): {
-        "sources": ["kv_cache_embedding_b200/csrc/tq_encode_tc.cu",
-                    "kv_cache_embedding_b200/csrc/tq_sm100.cuh"],
-        "sha1": "ab4b8235cd9123f4999844520f1ab4bc37aea169",
+        "sources": ["kv_cache_embedding_b200/csrc/tq_encode_tc.cu"],
+        "sha1": "2f7dc64a57a4d0a8d4f7a0c0e91ca5ece4ef7c49",
         "bytes": 68257280 + 2632192,
     },
 }

@@ -135,12 +135,20 @@ TQ_API int tq_encode(const tq_codebook_t *cb, const float *d_Pi, const float *d_
               uint32_t *d_codes, float *d_xnorm, float *d_rnorm,
               void *d_ws, size_t ws_bytes, void *stream);
 
-/* Device status of the last tq_encode that used d_ws (its first 4 bytes):
- * TQ_OK, or TQ_ERR_DEVICE_TIMEOUT when a bounded device-side wait of the
- * tensor-core encode gave up (the kernel then drains its in-flight copies,
- * releases tensor memory and exits; its outputs are undefined).  Copies the
- * word to the host and synchronises `stream`. */
+/* Device status of the last tq_encode, tq_score or tq_topk that used d_ws
+ * (its first 4 bytes): TQ_OK, or TQ_ERR_DEVICE_TIMEOUT when a bounded
+ * device-side wait of a tensor-core kernel gave up (the kernel then drains its
+ * in-flight copies and MMAs, releases tensor memory and exits; its outputs are
+ * undefined).  Copies the word to the host and synchronises `stream`. */
 TQ_API int tq_device_status(const void *d_ws, void *stream);
+
+/* Self-test of the device-side time-out path (no counterpart on the pages):
+ * one thread waits, with the same bounded wait the tensor-core kernels use,
+ * on a barrier that nothing completes.  After limit_ns (1 .. 2e9) it gives up
+ * and records TQ_ERR_DEVICE_TIMEOUT in the first 4 bytes of d_ws (>= 256
+ * bytes), which tq_device_status(d_ws, stream) then reports; the context
+ * stays usable.  TQ_ERR_ARG for a null d_ws or a limit out of range. */
+TQ_API int tq_selftest_wait_timeout(void *d_ws, uint64_t limit_ns, void *stream);
 
 /* S0 + S1, scores (quant_prune_distill #674: inner-product quantization with
  * an unbiased estimate; comuna.ru "8x faster attention logits"):

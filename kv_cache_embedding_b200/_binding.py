@@ -2,7 +2,7 @@
 names, arguments marshalled as plain integers (device pointers), sizes and
 the stream handle.  No computation happens here.
 
-The library must be built (``python -m kv_cache_embedding_b200.build``);
+The library must be built (``python kv_cache_embedding_b200/build.py``);
 importing this module without it raises, there is no fallback.
 """
 import ctypes as C
@@ -28,7 +28,7 @@ TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT = 
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
-           "tq_device_status")
+           "tq_device_status", "tq_selftest_wait_timeout")
 
 
 class tq_codebook_t(C.Structure):
@@ -53,7 +53,7 @@ class TQError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"libtq.so not built at {LIB_PATH}; run `python -m kv_cache_embedding_b200.build`")
+            f"libtq.so not built at {LIB_PATH}; run `python kv_cache_embedding_b200/build.py`")
     L = C.CDLL(LIB_PATH)
     P, i32, i64, u64, sz = C.c_void_p, C.c_int, C.c_int64, C.c_uint64, C.c_size_t
     cbp = C.POINTER(tq_codebook_t)
@@ -73,6 +73,8 @@ def _load():
     L.tq_topk_noalloc.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P]
     L.tq_device_status.restype = i32
     L.tq_device_status.argtypes = [P, P]
+    L.tq_selftest_wait_timeout.restype = i32
+    L.tq_selftest_wait_timeout.argtypes = [P, u64, P]
     L.tq_decode.restype = i32
     L.tq_decode.argtypes = [cbp, P, P, i32, i64, P, P, P, P, P, sz, P]
     L.tq_logits_fp32.restype = i32
@@ -111,8 +113,13 @@ def tq_encode(cb, d_Pi, d_S, G, n, d_x, x_dtype, d_codes, d_xnorm, d_rnorm, d_ws
 
 
 def tq_device_status(d_ws, stream):
-    """Status word the last tq_encode left in d_ws (synchronises the stream)."""
+    """Status word the last tq_encode / tq_score / tq_topk left in d_ws
+    (synchronises the stream)."""
     return lib.tq_device_status(d_ws, stream)
+
+
+def tq_selftest_wait_timeout(d_ws, limit_ns, stream):
+    return _ok("tq_selftest_wait_timeout", lib.tq_selftest_wait_timeout(d_ws, limit_ns, stream))
 
 
 def tq_score(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, d_scores, d_ws,

@@ -32,14 +32,10 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
         case TQ_OP_ENCODE:
             if (b < 1 || b > 4) return (size_t)-1;
             return 256 + 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
-        case TQ_OP_SCORE:
-            return 2 * qbuf;
+        case TQ_OP_SCORE:  // status word, transformed queries
+            return 256 + 2 * qbuf;
         case TQ_OP_TOPK:
-            if (topk_materialized(G, n, nq))  // scores, chunk maxima, counters, candidates
-                return 2 * qbuf + align256((size_t)G * nq * n * 4) +
-                       align256((size_t)G * nq * ntiles * 4) + align256((size_t)G * nq * 8) +
-                       2 * align256((size_t)G * nq * kTopkCandidates * 4);
-            return 2 * qbuf + parts;
+            return tq::topk_workspace_bytes(d, b, G, n, nq, k, topk_materialized(G, n, nq));
         case TQ_OP_DECODE:
             return 2 * align256((size_t)chunk * d * 4);
         case TQ_OP_EXACT:
@@ -48,6 +44,23 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
             return (size_t)-1;
     }
 }
+
+namespace tq {
+size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize) {
+    (void)b;
+    const size_t qbuf = align256((size_t)G * nq * d * 4);
+    if (materialize) {
+        // scores, maxima per 128-key tile, counters, candidate lists
+        const int64_t ntm = (n + 127) / 128;
+        return 256 + 2 * qbuf + align256((size_t)G * nq * n * 4) +
+               align256((size_t)G * nq * ntm * 4) + align256((size_t)G * nq * 8) +
+               2 * align256((size_t)G * nq * kTopkCandidates * 4);
+    }
+    const int64_t ntiles = (n + kTopkTile - 1) / kTopkTile;
+    return 256 + 2 * qbuf + align256((size_t)G * nq * ntiles * k * 4) +
+           align256((size_t)G * nq * ntiles * k * 8);
+}
+}  // namespace tq
 
 extern "C" int tq_device_status(const void* d_ws, void* stream) {
     if (!d_ws) return TQ_ERR_ARG;

@@ -76,6 +76,24 @@ int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const
                  bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
                  cudaStream_t s);
 bool encode_tc_supported(int d, int x_dtype, int G, int64_t n);
+bool score_tc_supported(int d, int b, int G, int64_t n, int nq);
+int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
+                    const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,
+                    const float* u, float* d_scores, float* tmax, int* zero_cnt, int* d_err,
+                    cudaStream_t s);
+// Top-k with the path chosen by the caller: materialised scores (`materialize`)
+// or the fused running-list kernel.
+int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
+             const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
+             const void* d_q, int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
+             size_t ws_bytes, bool materialize, cudaStream_t s);
+size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize);
+// tq_topk's argument checks: TQ_OK to run, kTopkNothing when there is nothing
+// to compute (a successful no-op), else the error status.
+constexpr int kTopkNothing = 1;
+int topk_validate(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
+                  const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
+                  const void* d_q, int q_dtype, int k, const float* d_vals, const int64_t* d_ids);
 int launch_encode_tc(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
                      int64_t n, const void* d_x, uint32_t* d_codes, float* d_xnorm,
                      float* d_rnorm, int* d_err, cudaStream_t s);

@@ -41,13 +41,19 @@ extern "C" int tq_topk_noalloc(const tq_codebook_t* cb, const float* d_Pi, const
                                int G, int64_t n, const uint32_t* d_codes, const float* d_xnorm,
                                const float* d_rnorm, int nq, const void* d_q, int q_dtype, int k,
                                float* d_vals, int64_t* d_ids, void* stream) {
-    if (!cb) return TQ_ERR_ARG;
+    const int v = tq::topk_validate(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q,
+                                    q_dtype, k, d_vals, d_ids);
+    if (v) return v == tq::kTopkNothing ? TQ_OK : v;
     const size_t need = tq_workspace_bytes(TQ_OP_TOPK, cb->d, cb->b, G, n, nq, k);
-    // (size_t)-1 marks an unsupported shape: tq_topk reports the precise error.
-    if (need != (size_t)-1 && need > (size_t)TQ_NOALLOC_SCRATCH_BYTES) return TQ_ERR_SCRATCH_LIMIT;
+    // The materialised-score path when its scratch fits, else the fused path.
+    bool materialize = tq::topk_materialized(G, n, nq) && need <= (size_t)TQ_NOALLOC_SCRATCH_BYTES;
+    if (!materialize && tq::topk_workspace_bytes(cb->d, cb->b, G, n, nq, k, false) >
+                            (size_t)TQ_NOALLOC_SCRATCH_BYTES)
+        return TQ_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;
     const int rc = scratch_address(&scratch);
     if (rc) return rc;
-    return tq_topk(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
-                   d_ids, scratch, (size_t)TQ_NOALLOC_SCRATCH_BYTES, stream);
+    return tq::topk_run(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k,
+                        d_vals, d_ids, scratch, (size_t)TQ_NOALLOC_SCRATCH_BYTES, materialize,
+                        (cudaStream_t)stream);
 }

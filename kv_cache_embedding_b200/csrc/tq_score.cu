@@ -873,10 +873,16 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_SCORE, d, b, G, n, nq, 0))
         return TQ_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
-    float* qr = (float*)d_ws;
-    float* u = (float*)((char*)d_ws + align256((size_t)G * nq * d * 4));
+    // [status word (256 B) | qr | u]
+    int* err = (int*)d_ws;
+    float* qr = (float*)((char*)d_ws + 256);
+    float* u = (float*)((char*)qr + align256((size_t)G * nq * d * 4));
     rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
     if (rc) return rc;
+    if (score_tc_supported(d, b, G, n, nq))
+        return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
+                               nullptr, err, s);
+    TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
     const KCodebook kc = make_kcodebook(cb);
     switch (b) {
         case 1: return launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
@@ -886,23 +892,19 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     }
 }
 
-extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
-                       int64_t n, const uint32_t* d_codes, const float* d_xnorm,
-                       const float* d_rnorm, int nq, const void* d_q, int q_dtype, int k,
-                       float* d_vals, int64_t* d_ids, void* d_ws, size_t ws_bytes,
-                       void* stream) {
-    int rc = check_common(cb, G, n, nq, q_dtype);
-    if (rc) return rc;
-    if (k < 1 || k > kMaxK || (int64_t)k > n) return (n == 0 && nq == 0) ? TQ_OK : TQ_ERR_ARG;
-    if (nq == 0) return TQ_OK;
-    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_vals || !d_ids)
-        return TQ_ERR_ARG;
+namespace tq {
+int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
+             const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
+             const void* d_q, int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
+             size_t ws_bytes, bool materialize, cudaStream_t s) {
     const int d = cb->d, b = cb->b;
-    if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_TOPK, d, b, G, n, nq, k))
+    if (!d_ws || ws_bytes < topk_workspace_bytes(d, b, G, n, nq, k, materialize))
         return TQ_ERR_WORKSPACE;
-    cudaStream_t s = (cudaStream_t)stream;
+    int rc;
     const int ntiles = (int)((n + kTopkTile - 1) / kTopkTile);
-    char* p = (char*)d_ws;
+    // [status word (256 B) | qr | u | path-specific]
+    int* err = (int*)d_ws;
+    char* p = (char*)d_ws + 256;
     float* qr = (float*)p;
     p += align256((size_t)G * nq * d * 4);
     float* u = (float*)p;
@@ -911,22 +913,34 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
     if (rc) return rc;
     const KCodebook kc = make_kcodebook(cb);
     const int64_t rows = (int64_t)G * nq;
-    if (topk_materialized(G, n, nq)) {
-        // scores [G][nq][n] and chunk maxima [G][nq][ntiles], then per-row selection
+    if (materialize) {
+        // scores [G][nq][n], row maxima per chunk, counters, candidates; then
+        // the per-row selection
+        const bool tc = score_tc_supported(d, b, G, n, nq);
+        const int64_t ntm = (n + 127) / 128;
         float* sc = (float*)p;
         p += align256((size_t)rows * n * 4);
         float* cm = (float*)p;
-        p += align256((size_t)rows * ntiles * 4);
+        p += align256((size_t)rows * ntm * 4);
         int* cnt = (int*)p;  // [2][rows]: candidate counts, finished blocks
         p += align256((size_t)rows * 2 * 4);
         float* cv = (float*)p;
         p += align256((size_t)rows * kCandCapG * 4);
         int* ci = (int*)p;
-        switch (b) {
-            case 1: rc = launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
-            case 2: rc = launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
-            case 3: rc = launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
-            default: rc = launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+        int nchunks;
+        if (tc) {  // maxima per 128-key tile
+            rc = launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt, err,
+                                 s);
+            nchunks = (int)ntm;
+        } else {  // maxima per 256-key block
+            TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
+            switch (b) {
+                case 1: rc = launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+                case 2: rc = launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+                case 3: rc = launch_score_b<3>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+                default: rc = launch_score_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
+            }
+            nchunks = ntiles;
         }
         if (rc) return rc;
         int nsm = 0, dev = 0;
@@ -940,12 +954,13 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
         P = P < pmin ? pmin : P;
         P = P > pmax ? pmax : P;
         dim3 grid((unsigned)P, (unsigned)rows);
-        k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, n, ntiles, k, cnt, cnt + rows, cv, ci, d_vals,
-                                             d_ids);
+        k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, n, nchunks, k, cnt, cnt + rows, cv, ci, d_vals,
+                                            d_ids);
         TQ_CHECK_LAUNCH();
         return TQ_OK;
     }
     // fused: per-range best-K lists [G][nq][nblk][K], then the merge
+    TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
     float* pv = (float*)p;
     p += align256((size_t)rows * ntiles * k * 4);
     int64_t* pi = (int64_t*)p;
@@ -960,6 +975,34 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
     k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, tg.nblk, k, d_vals, d_ids);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
+}
+}  // namespace tq
+
+namespace tq {
+int topk_validate(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
+                  const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
+                  const void* d_q, int q_dtype, int k, const float* d_vals,
+                  const int64_t* d_ids) {
+    int rc = check_common(cb, G, n, nq, q_dtype);
+    if (rc) return rc;
+    if (k < 1 || k > kMaxK || (int64_t)k > n) return (n == 0 && nq == 0) ? kTopkNothing : TQ_ERR_ARG;
+    if (nq == 0) return kTopkNothing;
+    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_vals || !d_ids)
+        return TQ_ERR_ARG;
+    return TQ_OK;
+}
+}  // namespace tq
+
+extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                       int64_t n, const uint32_t* d_codes, const float* d_xnorm,
+                       const float* d_rnorm, int nq, const void* d_q, int q_dtype, int k,
+                       float* d_vals, int64_t* d_ids, void* d_ws, size_t ws_bytes,
+                       void* stream) {
+    const int rc = topk_validate(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype,
+                                 k, d_vals, d_ids);
+    if (rc) return rc == kTopkNothing ? TQ_OK : rc;
+    return topk_run(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
+                    d_ids, d_ws, ws_bytes, topk_materialized(G, n, nq), (cudaStream_t)stream);
 }
 
 extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,

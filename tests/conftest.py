@@ -21,8 +21,14 @@ def oracle_lib():
 
 @pytest.fixture(scope="session")
 def tq_lib():
-    """Build libtq.so in-tree (no-op when up to date) and return the binding."""
-    from kv_cache_embedding_b200 import build as kb
+    """Build libtq.so in-tree (no-op when up to date) and return the binding.
+    The build script is loaded by path: importing the package needs the
+    library it builds."""
+    import importlib.util
+    path = os.path.join(ROOT, "kv_cache_embedding_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_tq_build", path)
+    kb = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(kb)
     kb.build()
     import kv_cache_embedding_b200 as tq
     return tq

@@ -165,6 +165,25 @@ def test_score_gqa_bf16_groups(quant, oparams, tq_lib, cuda):
         PT.compare_scores(s_gpu[g], s_ora, np.linalg.norm(_f64(qs[g]), axis=1), xn.astype(np.float64))
 
 
+@pytest.mark.parametrize("G,n,nq,b", [(160, 300, 2, 4), (160, 300, 16, 4), (3, 1000, 37, 3), (2, 129, 16, 2)])
+def test_score_groups_and_query_passes(quant, oparams, tq_lib, cuda, G, n, nq, b):
+    """More groups than SMs (whole groups per CTA in turn), several query
+    passes per group, a ragged last tile of keys."""
+    d = 128
+    W = b * d // 32
+    qs = synth.gaussian_rows(G * nq, d, seed=50, norm_range=None).reshape(G, nq, d)
+    recs = [synth.random_records(n, W, seed=60 + g) for g in range(G)]
+    codes = tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+    s_gpu = _np(quant(d, b, 0, G).score(codes, qs.cuda()))
+    for g in range(G):
+        c, xn, rn = recs[g]
+        s_ora = O.score(oparams(d, b, g), c, xn, rn, _f64(qs[g]))
+        PT.compare_scores(s_gpu[g], s_ora, np.linalg.norm(_f64(qs[g]), axis=1), xn.astype(np.float64))
+
+
 @pytest.mark.parametrize("n,k,nq", [(4096, 10, 17), (2500, 1, 3), (2500, 32, 3), (33, 32, 2)])
 def test_topk(quant, oparams, tq_lib, cuda, n, k, nq):
     d, b = 128, 4
@@ -280,6 +299,24 @@ def test_errors_on_device(quant, tq_lib, cuda):
     with pytest.raises(ValueError):
         tq.encode(torch.zeros(10, 64, device=cuda))
     torch.cuda.synchronize()
+
+
+def test_device_wait_times_out_and_context_survives(quant, oparams, tq_lib, cuda):
+    """The bounded device-side wait gives up on a barrier nothing completes,
+    the status word reports TQ_ERR_DEVICE_TIMEOUT, and the next calls on the
+    same context run and are correct (status clean again)."""
+    B = tq_lib.binding
+    stream = torch.cuda.current_stream().cuda_stream
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda)
+    B.tq_selftest_wait_timeout(ws.data_ptr(), 20_000_000, stream)  # 20 ms
+    assert B.tq_device_status(ws.data_ptr(), stream) == B.TQ_ERR_DEVICE_TIMEOUT
+    with pytest.raises(B.TQError):
+        B.tq_selftest_wait_timeout(ws.data_ptr(), 0, stream)
+    # the context is still usable: an encode through the tensor-core kernel
+    x = synth.kv_keys(1, 300, 128, seed=12)
+    for gpu, ora, P in _encode_both(quant, oparams, x, 128, 4):
+        PT.compare_encode(128, 4, P.beta, gpu, ora)
+    assert B.tq_device_status(quant(128, 4).ws.buf.data_ptr(), stream) == B.TQ_OK
 
 
 # ---------------------------------------------------------------- tensor-core encode (d = 128, bf16)
