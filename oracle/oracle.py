@@ -44,6 +44,9 @@ def lib():
         L.tqo_topk.argtypes = [i64, i64, P, i32, P, P]
         L.tqo_exact_scores.argtypes = [i32, i64, P, i64, P, P]
         L.tqo_mse_estimate.argtypes = [i32, i32, P, P, P, P, P, P]
+        L.tqo_mse_encode.argtypes = [i32, i32, P, P, P, i64, P, P, P, P, P, P]
+        L.tqo_mse_score.argtypes = [i32, i32, P, i64, P, P, i64, P, P]
+        L.tqo_mse_decode.argtypes = [i32, i32, P, P, i64, P, P, P]
         _lib = L
     return _lib
 
@@ -222,3 +225,58 @@ def mse_estimate(d, bits, seed, x, q):
     _check(lib().tqo_mse_estimate(d, bits, _p(c), _p(beta), _p(Pi), _p(_f64(x)), _p(_f64(q)),
                                   _p(est)), "mse_estimate")
     return float(est[0])
+
+
+# ---------------------------------------------------------------- MSE-only variant
+class MseParams:
+    """The oracle's parameters of the MSE-only quantizer for (d, b, seed): the
+    b-bit Lloyd-Max tables (2^b levels) and Pi (the same Pi as the
+    inner-product quantizer of that seed)."""
+
+    def __init__(self, d, b, seed):
+        self.d, self.b, self.seed = d, b, seed
+        self.c, self.beta = codebook(d, b + 1)
+        self.Pi = rotation(d, seed)
+
+
+def mse_encode(params, x, diagnostics=False):
+    """Records of the MSE-only quantizer: codes [n, b*d/32] uint32 (R7 layout,
+    index top bit in the z position), xnorm, rnorm; with diagnostics also y
+    [n, d] float64 and the full b-bit index [n, d] int32."""
+    d, b = params.d, params.b
+    x = _f64(x).reshape(-1, d)
+    n = x.shape[0]
+    codes = np.empty((n, words_per_vector(d, b)), dtype=np.uint32)
+    xn = np.empty(n, dtype=np.float32)
+    rn = np.empty(n, dtype=np.float32)
+    y = np.empty((n, d), np.float64) if diagnostics else None
+    idx = np.empty((n, d), np.int32) if diagnostics else None
+    _check(lib().tqo_mse_encode(d, b, _p(params.c), _p(params.beta), _p(params.Pi), n, _p(x),
+                                _p(codes), _p(xn), _p(rn), _p(y), _p(idx)), "mse_encode")
+    if diagnostics:
+        return codes, xn, rn, y, idx
+    return codes, xn, rn
+
+
+def mse_score(params, codes, xnorm, q):
+    """|x| <Pi q, c[idx]> for every query row and record: [nq, n]."""
+    d, b = params.d, params.b
+    q = _f64(q).reshape(-1, d)
+    qr = (q @ params.Pi.astype(np.float64).T)  # Pi q in double from fp32 Pi
+    qr = np.ascontiguousarray(qr)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32).reshape(-1, words_per_vector(d, b))
+    n = codes.shape[0]
+    out = np.empty((q.shape[0], n), np.float64)
+    _check(lib().tqo_mse_score(d, b, _p(params.c), n, _p(codes), _p(_f32(xnorm)), q.shape[0],
+                               _p(qr), _p(out)), "mse_score")
+    return out
+
+
+def mse_decode(params, codes, xnorm):
+    d, b = params.d, params.b
+    codes = np.ascontiguousarray(codes, dtype=np.uint32).reshape(-1, words_per_vector(d, b))
+    n = codes.shape[0]
+    out = np.empty((n, d), np.float64)
+    _check(lib().tqo_mse_decode(d, b, _p(params.c), _p(params.Pi), n, _p(codes),
+                                _p(_f32(xnorm)), _p(out)), "mse_decode")
+    return out

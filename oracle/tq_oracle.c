@@ -603,3 +603,112 @@ int tqo_mse_estimate(int d, int bits, const float *c, const float *beta,
     *estimate = nx * acc;
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The MSE-only quantizer as a stored code ([QPD] "for MSE-optimised          */
+/* TurboQuant": all b bits go to the Lloyd-Max index, no QJL).  Steps 1-4 of  */
+/* tqo_encode with 2^b levels (c, beta: the b-bit tables, i.e. tqo_codebook  */
+/* at b + 1).  R11: the record keeps the layout of R7, the b-bit index split  */
+/* into its low b-1 bits (the idx field) and its top bit (the z position);   */
+/* |r| = |y - c[idx]| is stored as well.                                     */
+/* ------------------------------------------------------------------------ */
+static int32_t tqo_mse_index(int b, int32_t idx, int32_t z)
+{
+    return (b == 1) ? z : (idx | (z << (b - 1)));
+}
+
+int tqo_mse_encode(int d, int b, const float *c, const float *beta, const float *Pi,
+                   int64_t n, const double *x, uint32_t *codes, float *xnorm, float *rnorm,
+                   double *y_out, int32_t *idx_out)
+{
+    int L = 1 << b;
+    int64_t wpv, v;
+    if (tqo_check_db(d, b)) return -1;
+    wpv = tqo_words_per_vector(d, b);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (v = 0; v < n; v++) {
+        const double *xv = x + (size_t)v * d;
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+        int32_t *lo = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        int32_t *top = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        int32_t *full = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        double nx = 0.0, nr = 0.0;
+        int i, j, w;
+        for (j = 0; j < d; j++) nx += xv[j] * xv[j];
+        nx = sqrt(nx);
+        for (i = 0; i < d; i++) {
+            double acc = 0.0;
+            for (j = 0; j < d; j++) acc += (double)Pi[(size_t)i * d + j] * xv[j];
+            y[i] = (nx > 0.0) ? acc / nx : 0.0;
+        }
+        for (i = 0; i < d; i++) {
+            int cnt = 0;
+            double r;
+            for (j = 0; j + 1 < L; j++)
+                if ((double)beta[j] <= y[i]) cnt++;
+            full[i] = cnt;
+            lo[i] = (b == 1) ? 0 : (cnt & ((1 << (b - 1)) - 1));
+            top[i] = (b == 1) ? cnt : (cnt >> (b - 1));
+            r = y[i] - (double)c[cnt];
+            nr += r * r;
+        }
+        for (w = 0; w < d / 32; w++)
+            tqo_pack_block(b, lo + 32 * w, top + 32 * w, codes + (size_t)v * wpv + (size_t)w * b);
+        xnorm[v] = (float)nx;
+        rnorm[v] = (float)sqrt(nr);
+        if (y_out) memcpy(y_out + (size_t)v * d, y, sizeof(double) * (size_t)d);
+        if (idx_out) memcpy(idx_out + (size_t)v * d, full, sizeof(int32_t) * (size_t)d);
+        free(y); free(lo); free(top); free(full);
+    }
+    return 0;
+}
+
+/* The MSE estimate from stored records: s = |x| sum_i qr_i c[idx_i]
+ * (qr = Pi q from tqo_query; [QPD]: biased, the contrast to the QJL one). */
+int tqo_mse_score(int d, int b, const float *c, int64_t n, const uint32_t *codes,
+                  const float *xnorm, int64_t nq, const double *qr, double *scores)
+{
+    int64_t wpv, v;
+    if (tqo_check_db(d, b)) return -1;
+    wpv = tqo_words_per_vector(d, b);
+#pragma omp parallel for schedule(dynamic, 64)
+    for (v = 0; v < n; v++) {
+        int32_t idx[32], z[32];
+        for (int64_t t = 0; t < nq; t++) {
+            const double *a = qr + (size_t)t * d;
+            double acc = 0.0;
+            for (int w = 0; w < d / 32; w++) {
+                tqo_unpack_block(b, codes + (size_t)v * wpv + (size_t)w * b, idx, z);
+                for (int j = 0; j < 32; j++)
+                    acc += a[32 * w + j] * (double)c[tqo_mse_index(b, idx[j], z[j])];
+            }
+            scores[(size_t)t * n + v] = (double)xnorm[v] * acc;
+        }
+    }
+    return 0;
+}
+
+/* MSE dequantization: xhat = |x| Pi^T c[idx]. */
+int tqo_mse_decode(int d, int b, const float *c, const float *Pi, int64_t n,
+                   const uint32_t *codes, const float *xnorm, double *out)
+{
+    int64_t wpv, v;
+    if (tqo_check_db(d, b)) return -1;
+    wpv = tqo_words_per_vector(d, b);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (v = 0; v < n; v++) {
+        int32_t idx[32], z[32];
+        double *yh = (double *)malloc(sizeof(double) * (size_t)d);
+        for (int w = 0; w < d / 32; w++) {
+            tqo_unpack_block(b, codes + (size_t)v * wpv + (size_t)w * b, idx, z);
+            for (int j = 0; j < 32; j++) yh[32 * w + j] = (double)c[tqo_mse_index(b, idx[j], z[j])];
+        }
+        for (int i = 0; i < d; i++) {
+            double acc = 0.0;
+            for (int j = 0; j < d; j++) acc += (double)Pi[(size_t)j * d + i] * yh[j];
+            out[(size_t)v * d + i] = (double)xnorm[v] * acc;
+        }
+        free(yh);
+    }
+    return 0;
+}

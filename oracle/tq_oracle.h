@@ -69,7 +69,17 @@ int tqo_mse_estimate(int d, int bits, const float *c, const float *beta,
                      const float *Pi, const double *x, const double *q,
                      double *estimate);
 
+/* MSE-only quantizer stored as a code (b-bit Lloyd-Max index, no QJL). */
+int tqo_mse_encode(int d, int b, const float *c, const float *beta, const float *Pi,
+                   int64_t n, const double *x, uint32_t *codes, float *xnorm, float *rnorm,
+                   double *y_out, int32_t *idx_out);
+int tqo_mse_score(int d, int b, const float *c, int64_t n, const uint32_t *codes,
+                  const float *xnorm, int64_t nq, const double *qr, double *scores);
+int tqo_mse_decode(int d, int b, const float *c, const float *Pi, int64_t n,
+                   const uint32_t *codes, const float *xnorm, double *out);
+
 #ifdef __cplusplus
 }
 #endif
+
 #endif
