@@ -40,6 +40,10 @@ CONFIGS = {
     "kv": dict(G=8, n=32768, d=128, b=4, x="kv", nq=4, q="kv", k=10, score=True, topk=True,
                desc="KV keys bf16 [1,8,32768,128] (4 outlier channels x20 per head), b=4; "
                     "decode queries bf16 32 heads GQA 4:1"),
+    "kv_mse": dict(G=8, n=32768, d=128, b=4, x="kv", nq=4, q="kv", k=10, score=True, topk=True,
+                   variant="mse",
+                   desc="KV keys bf16 [1,8,32768,128] as kv, MSE-only variant (4-bit Lloyd-Max "
+                        "index, no QJL); decode queries bf16 32 heads GQA 4:1"),
     "decode": dict(G=8, n=131072, d=128, b=4, x="kv", nq=4, q="kv", k=10, score=True, topk=True,
                    desc="decode attention logits, Llama-3.1-8B-shaped: 32 q heads / 8 KV heads, "
                         "head_dim 128, context 131072, bf16, b=4"),
@@ -317,7 +321,8 @@ def run_ours(args, cfg, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     x, q = make_inputs(cfg, dev, seed_offset=rank)
-    tq = K.TurboQuant(cfg["d"], cfg["b"], seed=0, groups=cfg["G"], device=dev)
+    tq = K.TurboQuant(cfg["d"], cfg["b"], seed=0, groups=cfg["G"], device=dev,
+                      variant=cfg.get("variant", "prod"))
     step = Step(tq, cfg, x, q)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize()
@@ -406,7 +411,7 @@ def run_ours(args, cfg, rank, world, dist):
     # tcgen05 kernel whose contractions run as 3 half-precision passes per
     # fp32-accurate product, so its peak is the measured bf16 peak / 3.
     ach = ab["enc_flops"] / (enc_ms / 1e3) / 1e12
-    tc = cfg["d"] == 128 and cfg["x"] == "kv"
+    tc = cfg["d"] == 128 and cfg["x"] == "kv" and cfg.get("variant", "prod") == "prod"
     if tc:
         peak = pk["bf16"] / 3.0
         roofline = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
@@ -489,14 +494,20 @@ def oracle_sample(cfg, target_s=10.0, max_units=None):
     G, n, d, b, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
     x, q = make_inputs(cfg, "cpu", max_rows=65536)
     n = min(n, x.shape[1])
-    params = O.Params(d, b, 0)  # one group's parameters (built outside the timing)
+    mse = cfg.get("variant", "prod") == "mse"
+    # one group's parameters (built outside the timing)
+    params = O.MseParams(d, b, 0) if mse else O.Params(d, b, 0)
 
     def run(rows):
         xs = x[0, :rows].to(torch.float64).numpy()
         qs = q[0].to(torch.float64).numpy()
         t = time.perf_counter()
-        codes, xn, rn = O.encode(params, xs)
-        s = O.score(params, codes, xn, rn, qs)
+        if mse:
+            codes, xn, rn = O.mse_encode(params, xs)
+            s = O.mse_score(params, codes, xn, qs)
+        else:
+            codes, xn, rn = O.encode(params, xs)
+            s = O.score(params, codes, xn, rn, qs)
         O.topk(s, min(k, rows))
         return time.perf_counter() - t
 

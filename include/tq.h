@@ -82,21 +82,34 @@ extern "C" {
 #define TQ_OP_DECODE  4
 #define TQ_OP_EXACT   5
 
+/* codebook variants */
+#define TQ_VARIANT_PROD 0  /* inner-product quantizer: (b-1)-bit Lloyd-Max index
+                              + 1 QJL sign bit per coordinate (unbiased)        */
+#define TQ_VARIANT_MSE  1  /* MSE-only quantizer: b-bit Lloyd-Max index, no QJL
+                              (quant_prune_distill #674 "MSE-optimised";
+                              biased inner products)                           */
+
 /* Host-side codebook (quant_prune_distill #674: Lloyd-Max grid for the
  * target bit width; RecSysChannel #256 item 1: thresholds computed in
- * advance).  Filled by tq_build_codebook; plain data, caller-owned, may be
+ * advance).  Filled by tq_build_codebook (TQ_VARIANT_PROD) or
+ * tq_build_codebook_mse (TQ_VARIANT_MSE); plain data, caller-owned, may be
  * copied.  centroids[j] / boundaries[j] are the Lloyd-Max centroids and cell
- * boundaries of N(0,1) for 2^(b-1) levels, multiplied by 1/sqrt(d) and
- * rounded to fp32; unused entries are 0.  For b = 1 there are no levels. */
+ * boundaries of N(0,1) for `levels` levels, multiplied by 1/sqrt(d) and
+ * rounded to fp32; unused entries are 0.  PROD: levels = 2^(b-1) (none for
+ * b = 1).  MSE: levels = 2^b; its records use the layout below with the
+ * b-bit index split into its low b-1 bits (the idx field) and its top bit
+ * (the position of z), and store |r| = |y - c[idx]|. */
 typedef struct tq_codebook {
-    int32_t  d;            /* vector dimension                              */
-    int32_t  b;            /* total bits per coordinate (index bits b-1 + 1) */
-    int32_t  levels;       /* 2^(b-1), or 0 for b = 1                        */
-    int32_t  groups;       /* G: number of (Pi, S) pairs built               */
+    int32_t  d;            /* vector dimension                               */
+    int32_t  b;            /* total bits per coordinate                      */
+    int32_t  levels;       /* PROD: 2^(b-1), 0 for b = 1; MSE: 2^b           */
+    int32_t  groups;       /* G: number of (Pi, S) pairs (MSE: Pi only) built */
     uint64_t seed;         /* group g uses seed + g                          */
-    float    centroids[8];
-    float    boundaries[8];
+    float    centroids[16];
+    float    boundaries[16];
     double   distortion;   /* Lloyd-Max mean squared error for N(0,1)        */
+    int32_t  variant;      /* TQ_VARIANT_PROD or TQ_VARIANT_MSE              */
+    int32_t  reserved;     /* 0                                              */
 } tq_codebook_t;
 
 /* Bytes of device workspace an operation needs for the given sizes (0 when
@@ -123,6 +136,18 @@ TQ_API const char *tq_status_str(int status);
 TQ_API int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook_t *cb,
                       float *d_Pi, float *d_S, void *d_ws, size_t ws_bytes,
                       void *stream);
+
+/* E0 of the MSE-only quantizer (quant_prune_distill #674, "MSE-optimised
+ * TurboQuant": random rotation, then every bit on the Lloyd-Max index):
+ * Pi_g exactly as tq_build_codebook draws it (so a PROD and an MSE codebook of
+ * one seed share their rotation) and the b-bit (2^b-level) Lloyd-Max tables;
+ * no S.  cb->variant = TQ_VARIANT_MSE.  With such a codebook tq_encode,
+ * tq_score, tq_topk and tq_decode take d_S = NULL and compute
+ *   encode: idx_i = #{j : beta_j <= y_i} over 2^b levels, |r| = |y - c[idx]|;
+ *   score:  s = |x| <Pi_g q, c[idx]>;      decode: xhat = |x| Pi_g^T c[idx].
+ * Same arguments, sizes and errors as tq_build_codebook otherwise. */
+TQ_API int tq_build_codebook_mse(int d, int b, uint64_t seed, int G, tq_codebook_t *cb,
+                          float *d_Pi, void *d_ws, size_t ws_bytes, void *stream);
 
 /* E1-E6, encode (quant_prune_distill #674 inner-product quantizer;
  * RecSysChannel #256 caveat 1: normalise, multiply by a random matrix):

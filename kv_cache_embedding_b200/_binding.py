@@ -23,10 +23,13 @@ TQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 TQ_F32 = 0
 TQ_BF16 = 1
+TQ_VARIANT_PROD = 0
+TQ_VARIANT_MSE = 1
 
 TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT = range(6)
 
-EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_encode", "tq_score",
+EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_build_codebook_mse",
+           "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
            "tq_device_status", "tq_selftest_wait_timeout")
 
@@ -38,9 +41,11 @@ class tq_codebook_t(C.Structure):
         ("levels", C.c_int32),
         ("groups", C.c_int32),
         ("seed", C.c_uint64),
-        ("centroids", C.c_float * 8),
-        ("boundaries", C.c_float * 8),
+        ("centroids", C.c_float * 16),
+        ("boundaries", C.c_float * 16),
         ("distortion", C.c_double),
+        ("variant", C.c_int32),
+        ("reserved", C.c_int32),
     ]
 
 
@@ -63,6 +68,8 @@ def _load():
     L.tq_status_str.argtypes = [i32]
     L.tq_build_codebook.restype = i32
     L.tq_build_codebook.argtypes = [i32, i32, u64, i32, cbp, P, P, P, sz, P]
+    L.tq_build_codebook_mse.restype = i32
+    L.tq_build_codebook_mse.argtypes = [i32, i32, u64, i32, cbp, P, P, sz, P]
     L.tq_encode.restype = i32
     L.tq_encode.argtypes = [cbp, P, P, i32, i64, P, i32, P, P, P, P, sz, P]
     L.tq_score.restype = i32
@@ -104,6 +111,11 @@ def _ok(fn, status):
 def tq_build_codebook(d, b, seed, G, cb, d_Pi, d_S, d_ws, ws_bytes, stream):
     return _ok("tq_build_codebook",
                lib.tq_build_codebook(d, b, seed, G, C.byref(cb), d_Pi, d_S, d_ws, ws_bytes, stream))
+
+
+def tq_build_codebook_mse(d, b, seed, G, cb, d_Pi, d_ws, ws_bytes, stream):
+    return _ok("tq_build_codebook_mse",
+               lib.tq_build_codebook_mse(d, b, seed, G, C.byref(cb), d_Pi, d_ws, ws_bytes, stream))
 
 
 def tq_encode(cb, d_Pi, d_S, G, n, d_x, x_dtype, d_codes, d_xnorm, d_rnorm, d_ws, ws_bytes,

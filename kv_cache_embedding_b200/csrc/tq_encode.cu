@@ -6,7 +6,8 @@
 // matrix); seeallochnaya #3476 steps 1-2 (rotate; round every coordinate on
 // the precomputed grid; residual -> random matrix -> sign).
 //
-// Portable path (any supported d): per group and row chunk
+// Portable path (any supported d; the only path of the MSE-only variant): per
+// group and row chunk
 //   k_rownorm      |x| in fp64 accumulation                       (E1)
 //   sgemm          Y = X Pi^T / |x|                                (E2)
 //   k_quantize     idx = #{beta_j <= y}, r = y - c[idx], |r|       (E3, E4)
@@ -50,7 +51,7 @@ __global__ void k_quantize(float* __restrict__ yr, uint8_t* __restrict__ idx, in
         float r = v;
         if (cb.levels > 0) {
 #pragma unroll
-            for (int j = 0; j < 7; ++j)
+            for (int j = 0; j < 15; ++j)
                 if (j + 1 < cb.levels && cb.beta[j] <= v) ++cell;
             r = v - cb.c[cell];
         }
@@ -65,7 +66,9 @@ __global__ void k_quantize(float* __restrict__ yr, uint8_t* __restrict__ idx, in
 
 // One warp per row; lane j handles coordinate 32w + j of block w.  Fields of
 // neighbouring lanes are OR-combined with a butterfly inside each word's lanes.
-template <int B>
+// MSE: no projection; the b-bit cell is split into its low b-1 bits (idx
+// field) and its top bit (the z position).
+template <int B, bool MSE>
 __global__ void k_pack(const float* __restrict__ p, const uint8_t* __restrict__ idx, int64_t rows,
                        int d, uint32_t* __restrict__ codes) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
@@ -74,8 +77,9 @@ __global__ void k_pack(const float* __restrict__ p, const uint8_t* __restrict__ 
     const int W = words_per_vector(d, B);
     for (int w = 0; w < d / 32; ++w) {
         const int i = 32 * w + lane;
-        const uint32_t z = (p[row * d + i] >= 0.f) ? 1u : 0u;
-        const uint32_t iv = idx[row * d + i];
+        const uint32_t cell = idx[row * d + i];
+        const uint32_t z = MSE ? (cell >> (B - 1)) : ((p[row * d + i] >= 0.f) ? 1u : 0u);
+        const uint32_t iv = MSE ? (cell & ((1u << (B - 1)) - 1u)) : cell;
         uint32_t* out = codes + row * W + w * B;
         if (B == 1) {
             const uint32_t word = __ballot_sync(0xffffffffu, z != 0u);
@@ -111,12 +115,13 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     if (!valid_db(d, b)) return TQ_ERR_UNSUPPORTED;
     if (cb->groups < G) return TQ_ERR_MISMATCH;
     if (n == 0) return TQ_OK;
-    if (!d_Pi || !d_S || !d_x || !d_codes || !d_xnorm || !d_rnorm) return TQ_ERR_ARG;
+    const bool mse = is_mse(cb);
+    if (!d_Pi || (!mse && !d_S) || !d_x || !d_codes || !d_xnorm || !d_rnorm) return TQ_ERR_ARG;
     const size_t need = tq_workspace_bytes(TQ_OP_ENCODE, d, b, G, n, 0, 0);
     if (need > 0 && (!d_ws || ws_bytes < need)) return TQ_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     // the first 256 bytes of the workspace hold the device status word
-    if (encode_tc_supported(d, x_dtype, G, n))  // d = 128 bf16 keys: fused tensor-core kernel
+    if (!mse && encode_tc_supported(d, x_dtype, G, n))  // d = 128 bf16 keys: fused tensor-core kernel
         return launch_encode_tc(cb, d_Pi, d_S, G, n, d_x, d_codes, d_xnorm, d_rnorm,
                                 (int*)d_ws, s);
     TQ_TRY_CUDA(cudaMemsetAsync(d_ws, 0, sizeof(int), s));
@@ -147,15 +152,25 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
             if (rc) return rc;
             k_quantize<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rn);
             TQ_CHECK_LAUNCH();
+            uint32_t* cg = d_codes + (size_t)off * W;
+            if (mse) {  // no QJL projection
+                switch (b) {
+                    case 1: k_pack<1, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    case 2: k_pack<2, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    case 3: k_pack<3, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    default: k_pack<4, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                }
+                TQ_CHECK_LAUNCH();
+                continue;
+            }
             rc = launch_sgemm((int)rows, d, d, Y, TQ_F32, d, d_S + g * dd, true, d, P, d, nullptr,
                               0, s);
             if (rc) return rc;
-            uint32_t* cg = d_codes + (size_t)off * W;
             switch (b) {
-                case 1: k_pack<1><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                case 2: k_pack<2><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                case 3: k_pack<3><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                default: k_pack<4><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                case 1: k_pack<1, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                case 2: k_pack<2, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                case 3: k_pack<3, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                default: k_pack<4, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
             }
             TQ_CHECK_LAUNCH();
         }

@@ -18,20 +18,24 @@ constexpr int64_t kEncodeChunk = 65536;  // rows per encode/decode chunk
 
 // Codebook passed to kernels by value (kernel parameter space).
 struct KCodebook {
-    float c[8];
-    float beta[8];
-    int levels;   // 2^(b-1), 0 for b = 1
+    float c[16];
+    float beta[16];
+    int levels;   // PROD: 2^(b-1), 0 for b = 1; MSE: 2^b
+    int mse;      // 1: MSE-only variant (b-bit index, no QJL)
 };
 
 inline KCodebook make_kcodebook(const tq_codebook_t* cb) {
     KCodebook k;
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < 16; ++i) {
         k.c[i] = cb->centroids[i];
         k.beta[i] = cb->boundaries[i];
     }
     k.levels = cb->levels;
+    k.mse = cb->variant == TQ_VARIANT_MSE ? 1 : 0;
     return k;
 }
+
+inline bool is_mse(const tq_codebook_t* cb) { return cb->variant == TQ_VARIANT_MSE; }
 
 __host__ __device__ inline int words_per_vector(int d, int b) { return d / 32 * b; }
 

@@ -136,7 +136,7 @@ __global__ void k_finish_pi(const double* __restrict__ Q, const double* __restri
 // t_H = inf; centroid of [t_i, t_{i+1}) is (phi(t_i) - phi(t_{i+1})) /
 // (Q(t_i) - Q(t_{i+1})) with Q the upper tail; the negative half mirrors it.
 void lloyd_max_host(int L, double* c, double* beta, double* distortion) {
-    const int H = L / 2;
+    const int H = L / 2;  // L <= 16
     double p[8], t[9];
     for (int i = 0; i < H; ++i) p[i] = (i + 0.5) * (3.0 / H);
     auto phi = [](double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI); };
@@ -172,32 +172,13 @@ void lloyd_max_host(int L, double* c, double* beta, double* distortion) {
 }  // namespace
 }  // namespace tq
 
-extern "C" int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook_t* cb,
-                                 float* d_Pi, float* d_S, void* d_ws, size_t ws_bytes,
-                                 void* stream) {
-    using namespace tq;
-    if (!cb || G < 1) return TQ_ERR_ARG;
-    if (!valid_db(d, b)) return TQ_ERR_UNSUPPORTED;
-    if (!d_Pi || !d_S || !d_ws) return TQ_ERR_ARG;
-    if (ws_bytes < tq_workspace_bytes(TQ_OP_BUILD, d, b, G, 0, 0, 0)) return TQ_ERR_WORKSPACE;
-    cudaStream_t s = (cudaStream_t)stream;
+namespace tq {
+namespace {
 
-    tq_codebook_t out;
-    std::memset(&out, 0, sizeof(out));
-    out.d = d;
-    out.b = b;
-    out.groups = G;
-    out.seed = seed;
-    out.levels = (b == 1) ? 0 : (1 << (b - 1));
-    out.distortion = 1.0;
-    if (out.levels > 0) {
-        double c[8], beta[8];
-        lloyd_max_host(out.levels, c, beta, &out.distortion);
-        const double sigma = 1.0 / std::sqrt((double)d);
-        for (int i = 0; i < out.levels; ++i) out.centroids[i] = (float)(c[i] * sigma);
-        for (int i = 0; i + 1 < out.levels; ++i) out.boundaries[i] = (float)(beta[i] * sigma);
-    }
-
+// Pi_g (and, with d_S, S_g) of every group: Gaussian draws, Householder QR in
+// fp64 on the device, Pi = Q diag(sign R_jj).
+int build_matrices(int d, uint64_t seed, int G, float* d_Pi, float* d_S, void* d_ws,
+                   cudaStream_t s) {
     const size_t dd = (size_t)d * d;
     double* A = (double*)d_ws;
     double* Q = (double*)((char*)d_ws + align256(dd * sizeof(double)));
@@ -209,7 +190,7 @@ extern "C" int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook
         const uint64_t sg = seed + (uint64_t)g;
         const uint64_t key_pi = mix64_host(sg ^ (0ULL * kGamma));
         const uint64_t key_s = mix64_host(sg ^ (1ULL * kGamma));
-        k_gaussian<<<gblocks, gthreads, 0, s>>>(key_s, d, nullptr, d_S + (size_t)g * dd);
+        if (d_S) k_gaussian<<<gblocks, gthreads, 0, s>>>(key_s, d, nullptr, d_S + (size_t)g * dd);
         k_gaussian<<<gblocks, gthreads, 0, s>>>(key_pi, d, A, nullptr);
         TQ_CHECK_LAUNCH();
         for (int j = 0; j < d; ++j) {
@@ -222,6 +203,56 @@ extern "C" int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook
         k_finish_pi<<<(unsigned)((dd + 255) / 256), 256, 0, s>>>(Q, rd, d, d_Pi + (size_t)g * dd);
         TQ_CHECK_LAUNCH();
     }
-    *cb = out;
+    return TQ_OK;
+}
+
+// Host codebook: `levels` Lloyd-Max levels of N(0,1) scaled by 1/sqrt(d).
+tq_codebook_t make_codebook(int d, int b, uint64_t seed, int G, int levels, int variant) {
+    tq_codebook_t out;
+    std::memset(&out, 0, sizeof(out));
+    out.d = d;
+    out.b = b;
+    out.groups = G;
+    out.seed = seed;
+    out.levels = levels;
+    out.variant = variant;
+    out.distortion = 1.0;
+    if (levels > 0) {
+        double c[16], beta[16];
+        lloyd_max_host(levels, c, beta, &out.distortion);
+        const double sigma = 1.0 / std::sqrt((double)d);
+        for (int i = 0; i < levels; ++i) out.centroids[i] = (float)(c[i] * sigma);
+        for (int i = 0; i + 1 < levels; ++i) out.boundaries[i] = (float)(beta[i] * sigma);
+    }
+    return out;
+}
+
+}  // namespace
+}  // namespace tq
+
+extern "C" int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook_t* cb,
+                                 float* d_Pi, float* d_S, void* d_ws, size_t ws_bytes,
+                                 void* stream) {
+    using namespace tq;
+    if (!cb || G < 1) return TQ_ERR_ARG;
+    if (!valid_db(d, b)) return TQ_ERR_UNSUPPORTED;
+    if (!d_Pi || !d_S || !d_ws) return TQ_ERR_ARG;
+    if (ws_bytes < tq_workspace_bytes(TQ_OP_BUILD, d, b, G, 0, 0, 0)) return TQ_ERR_WORKSPACE;
+    const int rc = build_matrices(d, seed, G, d_Pi, d_S, d_ws, (cudaStream_t)stream);
+    if (rc) return rc;
+    *cb = make_codebook(d, b, seed, G, (b == 1) ? 0 : (1 << (b - 1)), TQ_VARIANT_PROD);
+    return TQ_OK;
+}
+
+extern "C" int tq_build_codebook_mse(int d, int b, uint64_t seed, int G, tq_codebook_t* cb,
+                                     float* d_Pi, void* d_ws, size_t ws_bytes, void* stream) {
+    using namespace tq;
+    if (!cb || G < 1) return TQ_ERR_ARG;
+    if (!valid_db(d, b)) return TQ_ERR_UNSUPPORTED;
+    if (!d_Pi || !d_ws) return TQ_ERR_ARG;
+    if (ws_bytes < tq_workspace_bytes(TQ_OP_BUILD, d, b, G, 0, 0, 0)) return TQ_ERR_WORKSPACE;
+    const int rc = build_matrices(d, seed, G, d_Pi, nullptr, d_ws, (cudaStream_t)stream);
+    if (rc) return rc;
+    *cb = make_codebook(d, b, seed, G, 1 << b, TQ_VARIANT_MSE);
     return TQ_OK;
 }

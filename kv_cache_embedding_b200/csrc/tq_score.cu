@@ -92,9 +92,11 @@ __device__ __forceinline__ uint32_t field_index(const uint32_t (&w)[4], int j) {
     return (w[j >> 3] >> (4 * (j & 7))) & 15u;
 }
 
-// Decode table entry f -> (c[idx], 2z - 1) for the field layouts above.
+// Decode table entry f -> (c[idx], 2z - 1) for the field layouts above; for
+// the MSE-only variant the field is the whole b-bit cell: (c[f], 0).
 template <int B>
 __device__ __forceinline__ float2 table_entry(const KCodebook& cb, int f) {
+    if (cb.mse) return make_float2(cb.c[f & ((1 << B) - 1)], 0.f);
     if (B == 1) return make_float2(0.f, (f & 1) ? 1.f : -1.f);
     if (B == 2) return make_float2(cb.c[f & 1], (f & 2) ? 1.f : -1.f);
     if (B == 3) return make_float2(cb.c[f & 3], (f & 4) ? 1.f : -1.f);
@@ -609,9 +611,13 @@ __global__ void k_combine(const uint32_t* __restrict__ codes, const float* __res
         int cell;
         uint32_t z;
         field<B>(w, j, cell, z);
-        const float yh = (B == 1) ? 0.f : cb.c[cell];
         float* p = E + row * d + blk * 32 + j;
-        *p = yh + kap * (*p);
+        if (cb.mse) {  // MSE-only variant: the b-bit cell is (idx | z << (b-1)); no QJL term
+            *p = cb.c[(B == 1) ? (int)z : (cell | (int)(z << (B - 1)))];
+        } else {
+            const float yh = (B == 1) ? 0.f : cb.c[cell];
+            *p = yh + kap * (*p);
+        }
     }
 }
 
@@ -776,9 +782,13 @@ __global__ __launch_bounds__(512) void k_query_prep(const float* __restrict__ Pi
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
+        float* outg = (pass == 0 ? qr : u) + row * d;
+        if (pass == 1 && !S) {  // MSE-only variant: no QJL vector
+            for (int j = threadIdx.x; j < d; j += blockDim.x) outg[j] = 0.f;
+            break;
+        }
         const float* M = (pass == 0 ? Pi : S) + (size_t)g * d * d;
         const float* v = sq + pass * d;
-        float* outg = (pass == 0 ? qr : u) + row * d;
         for (int i0 = warp * R; i0 < d; i0 += nw * R) {
             float acc[R];
 #pragma unroll
@@ -841,6 +851,10 @@ int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const 
         int rc = launch_sgemm(nq, d, d, qg, q_dtype, d, d_Pi + g * dd, true, d,
                               qr + (size_t)g * nq * d, d, nullptr, 0, s);
         if (rc) return rc;
+        if (!d_S) {  // MSE-only variant: no QJL vector
+            TQ_TRY_CUDA(cudaMemsetAsync(u + (size_t)g * nq * d, 0, (size_t)nq * d * 4, s));
+            continue;
+        }
         rc = launch_sgemm(nq, d, d, qr + (size_t)g * nq * d, TQ_F32, d, d_S + g * dd, true, d,
                           u + (size_t)g * nq * d, d, nullptr, 0, s);
         if (rc) return rc;
@@ -868,7 +882,9 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     int rc = check_common(cb, G, n, nq, q_dtype);
     if (rc) return rc;
     if (n == 0 || nq == 0) return TQ_OK;
-    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_scores) return TQ_ERR_ARG;
+    if (!d_Pi || (!is_mse(cb) && !d_S) || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_scores)
+        return TQ_ERR_ARG;
+    if (is_mse(cb)) d_S = nullptr;
     const int d = cb->d, b = cb->b;
     if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_SCORE, d, b, G, n, nq, 0))
         return TQ_ERR_WORKSPACE;
@@ -879,7 +895,7 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     float* u = (float*)((char*)qr + align256((size_t)G * nq * d * 4));
     rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
     if (rc) return rc;
-    if (score_tc_supported(d, b, G, n, nq))
+    if (!is_mse(cb) && score_tc_supported(d, b, G, n, nq))
         return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
     TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
@@ -909,14 +925,14 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
     p += align256((size_t)G * nq * d * 4);
     float* u = (float*)p;
     p += align256((size_t)G * nq * d * 4);
-    rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
+    rc = query_prep(d_Pi, is_mse(cb) ? nullptr : d_S, G, d, nq, d_q, q_dtype, qr, u, s);
     if (rc) return rc;
     const KCodebook kc = make_kcodebook(cb);
     const int64_t rows = (int64_t)G * nq;
     if (materialize) {
         // scores [G][nq][n], row maxima per chunk, counters, candidates; then
         // the per-row selection
-        const bool tc = score_tc_supported(d, b, G, n, nq);
+        const bool tc = !is_mse(cb) && score_tc_supported(d, b, G, n, nq);
         const int64_t ntm = (n + 127) / 128;
         float* sc = (float*)p;
         p += align256((size_t)rows * n * 4);
@@ -987,7 +1003,8 @@ int topk_validate(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, 
     if (rc) return rc;
     if (k < 1 || k > kMaxK || (int64_t)k > n) return (n == 0 && nq == 0) ? kTopkNothing : TQ_ERR_ARG;
     if (nq == 0) return kTopkNothing;
-    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_vals || !d_ids)
+    if (!d_Pi || (!is_mse(cb) && !d_S) || !d_codes || !d_xnorm || !d_rnorm || !d_q || !d_vals ||
+        !d_ids)
         return TQ_ERR_ARG;
     return TQ_OK;
 }
@@ -1012,7 +1029,8 @@ extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float
     int rc = check_common(cb, G, n, 0, TQ_F32);
     if (rc) return rc;
     if (n == 0) return TQ_OK;
-    if (!d_Pi || !d_S || !d_codes || !d_xnorm || !d_rnorm || !d_xhat) return TQ_ERR_ARG;
+    const bool mse = is_mse(cb);
+    if (!d_Pi || (!mse && !d_S) || !d_codes || !d_xnorm || !d_rnorm || !d_xhat) return TQ_ERR_ARG;
     const int d = cb->d, b = cb->b;
     if (!d_ws || ws_bytes < tq_workspace_bytes(TQ_OP_DECODE, d, b, G, n, 0, 0))
         return TQ_ERR_WORKSPACE;
@@ -1029,17 +1047,19 @@ extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float
             const int64_t off = (int64_t)g * n + r0;
             const uint32_t* cg = d_codes + off * W;
             const unsigned blocks = (unsigned)((rows * (d / 32) + 255) / 256);
-            switch (b) {
-                case 1: k_signs<1><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                case 2: k_signs<2><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                case 3: k_signs<3><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                default: k_signs<4><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+            if (!mse) {
+                switch (b) {
+                    case 1: k_signs<1><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                    case 2: k_signs<2><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                    case 3: k_signs<3><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                    default: k_signs<4><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                }
+                TQ_CHECK_LAUNCH();
+                // E = T S   (E[v][j] = sum_i T[v][i] S[i][j])
+                rc = launch_sgemm((int)rows, d, d, T, TQ_F32, d, d_S + g * dd, false, d, E, d,
+                                  nullptr, 0, s);
+                if (rc) return rc;
             }
-            TQ_CHECK_LAUNCH();
-            // E = T S   (E[v][j] = sum_i T[v][i] S[i][j])
-            rc = launch_sgemm((int)rows, d, d, T, TQ_F32, d, d_S + g * dd, false, d, E, d, nullptr,
-                              0, s);
-            if (rc) return rc;
             switch (b) {
                 case 1: k_combine<1><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
                 case 2: k_combine<2><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;

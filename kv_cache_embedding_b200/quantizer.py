@@ -54,21 +54,33 @@ class Workspace:
 
 
 class TurboQuant:
-    """TurboQuant inner-product quantizer with b total bits per coordinate
-    ((b-1)-bit Lloyd-Max index + 1 QJL sign bit) for dimension d and G groups
-    (KV heads), each group with its own Pi and S (seed + g)."""
+    """TurboQuant quantizer with b total bits per coordinate for dimension d and
+    G groups (KV heads), each group with its own Pi (and S) from seed + g.
 
-    def __init__(self, d, b, seed=0, groups=1, device="cuda"):
+    variant="prod" (default): the inner-product quantizer, (b-1)-bit
+    Lloyd-Max index + 1 QJL sign bit, unbiased inner products.
+    variant="mse": the MSE-only quantizer, b-bit Lloyd-Max index, no QJL
+    (no S; biased inner products)."""
+
+    def __init__(self, d, b, seed=0, groups=1, device="cuda", variant="prod"):
+        if variant not in ("prod", "mse"):
+            raise ValueError(f"variant must be 'prod' or 'mse', got {variant!r}")
         self.d, self.b, self.seed, self.G = int(d), int(b), int(seed), int(groups)
+        self.variant = variant
         self.device = torch.device(device)
         self.Pi = torch.empty(self.G, d, d, dtype=torch.float32, device=self.device)
-        self.S = torch.empty(self.G, d, d, dtype=torch.float32, device=self.device)
+        self.S = (torch.empty(self.G, d, d, dtype=torch.float32, device=self.device)
+                  if variant == "prod" else None)
         self.cb = B.tq_codebook_t()
         self.ws = Workspace(self.device)
         nbytes = B.tq_workspace_bytes(B.TQ_OP_BUILD, d, b, self.G, 0, 0, 0)
         wp, wn = self.ws.get(nbytes)
-        B.tq_build_codebook(self.d, self.b, self.seed, self.G, self.cb, _ptr(self.Pi),
-                            _ptr(self.S), wp, wn, _stream())
+        if variant == "prod":
+            B.tq_build_codebook(self.d, self.b, self.seed, self.G, self.cb, _ptr(self.Pi),
+                                _ptr(self.S), wp, wn, _stream())
+        else:
+            B.tq_build_codebook_mse(self.d, self.b, self.seed, self.G, self.cb, _ptr(self.Pi),
+                                    wp, wn, _stream())
 
     @property
     def words(self):

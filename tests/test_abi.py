@@ -4,6 +4,7 @@ device work (no GPU needed for these paths)."""
 import ctypes as C
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -37,11 +38,21 @@ def test_status_strings(tq_lib):
     assert B.tq_status_str(12345) == "unknown status"
 
 
-def test_codebook_struct_layout(tq_lib):
+def test_codebook_struct_layout(tq_lib, tmp_path):
+    """The binding's struct matches the header's, as a C compiler lays it out."""
     B = tq_lib.binding
-    assert C.sizeof(B.tq_codebook_t) == 96
-    assert B.tq_codebook_t.seed.offset == 16
-    assert B.tq_codebook_t.distortion.offset == 88
+    fields = [f for f, _ in B.tq_codebook_t._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text(
+        "#include <stdio.h>\n#include <stddef.h>\n#include \"tq.h\"\n"
+        "int main(void) {\n  printf(\"%zu\\n\", sizeof(tq_codebook_t));\n"
+        + "".join(f"  printf(\"%zu\\n\", offsetof(tq_codebook_t, {f}));\n" for f in fields)
+        + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
+    assert got[0] == C.sizeof(B.tq_codebook_t) == 168
+    assert got[1:] == [getattr(B.tq_codebook_t, f).offset for f in fields]
 
 
 def test_workspace_sizes(tq_lib):

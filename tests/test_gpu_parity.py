@@ -349,3 +349,103 @@ def test_encode_tc_matches_portable_path(quant, tq_lib):
     same = (c_tc.codes == c_pt.codes).all(dim=2).float().mean().item()
     assert same > 0.995
     assert torch.allclose(c_tc.xnorm, c_pt.xnorm, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- MSE-only variant
+@pytest.fixture(scope="module")
+def quant_mse(cuda, tq_lib):
+    cache = {}
+
+    def get(d, b, seed=0, groups=1):
+        key = (d, b, seed, groups)
+        if key not in cache:
+            cache[key] = tq_lib.TurboQuant(d, b, seed=seed, groups=groups, device=cuda,
+                                           variant="mse")
+            torch.cuda.synchronize()
+        return cache[key]
+    return get
+
+
+def _mse_full_index(d, b, codes):
+    idx, z = PT.read_layout(d, b, codes)
+    return z if b == 1 else idx | (z << (b - 1))
+
+
+def _mse_compare(d, b, gpu, ora, beta, bound_flags=True):
+    """Cells bit-exact except within 1e-5 sigma of a boundary (counted, at most
+    1e-4 of all coordinates); norms to 1e-4; |r| on records whose cells all
+    agree."""
+    g_codes, g_xn, g_rn = gpu
+    o_codes, o_xn, o_rn, y, o_idx = ora
+    g_idx = _mse_full_index(d, b, g_codes)
+    assert np.array_equal(_mse_full_index(d, b, o_codes), o_idx)
+    sigma = 1.0 / math.sqrt(d)
+    if beta.size:
+        near = np.min(np.abs(y[:, :, None] - beta.astype(np.float64)[None, None, :]), axis=2) \
+            < 1e-5 * sigma
+    else:
+        near = np.zeros_like(y, dtype=bool)
+    mism = g_idx != o_idx
+    assert not np.any(mism & ~near), int(np.sum(mism & ~near))
+    if bound_flags:
+        assert near.mean() <= 1e-4, near.mean()
+    np.testing.assert_allclose(g_xn, o_xn, rtol=1e-4, atol=1e-30)
+    same = ~np.any(mism, axis=1)
+    np.testing.assert_allclose(g_rn[same], o_rn[same], rtol=1e-4, atol=1e-6)
+
+
+def test_mse_and_prod_share_the_rotation(quant, quant_mse):
+    a, m = quant(128, 3, 5), quant_mse(128, 3, 5)
+    assert torch.equal(a.Pi, m.Pi)
+    assert m.S is None and m.cb.variant == 1 and m.cb.levels == 8
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_mse_encode_tiny_config(quant_mse, b):
+    d = 128
+    x = synth.gaussian_rows(4096, d, seed=1)
+    P = O.MseParams(d, b, 0)
+    codes = quant_mse(d, b).encode(x.cuda()[None])
+    ora = O.mse_encode(P, x.numpy(), diagnostics=True)
+    gpu = (_np(codes.codes[0]).view(np.uint32), _np(codes.xnorm[0]), _np(codes.rnorm[0]))
+    _mse_compare(d, b, gpu, ora, P.beta)
+
+
+@pytest.mark.parametrize("d,b,G", [(128, 4, 2), (256, 2, 1), (1536, 3, 1)])
+def test_mse_encode_bf16_and_large_d(quant_mse, d, b, G):
+    x = synth.kv_keys(G, 1001, d, seed=2)
+    codes = quant_mse(d, b, 0, G).encode(x.cuda())
+    for g in range(G):
+        P = O.MseParams(d, b, g)
+        ora = O.mse_encode(P, x[g].to(torch.float64).numpy(), diagnostics=True)
+        gpu = (_np(codes.codes[g]).view(np.uint32), _np(codes.xnorm[g]), _np(codes.rnorm[g]))
+        _mse_compare(d, b, gpu, ora, P.beta)
+
+
+@pytest.mark.parametrize("b,nq", [(4, 64), (2, 3), (1, 5)])
+def test_mse_score_and_topk(quant_mse, tq_lib, cuda, b, nq):
+    d, n, k = 128, 3000, 10
+    x = synth.gaussian_rows(n, d, seed=3)
+    q = synth.gaussian_rows(nq, d, seed=4, norm_range=None)
+    P = O.MseParams(d, b, 0)
+    c, xn, rn = O.mse_encode(P, x.numpy())
+    codes = _to_codes(tq_lib, c, xn, rn, cuda)
+    tq = quant_mse(d, b)
+    s_gpu = _np(tq.score(codes, q.cuda()[None])[0])
+    s_ora = O.mse_score(P, c, xn, q.numpy())
+    qn = np.linalg.norm(_f64(q), axis=1)
+    PT.compare_scores(s_gpu, s_ora, qn, xn.astype(np.float64))
+    vals, ids = tq.topk(codes, q.cuda()[None], k)
+    PT.compare_topk(_np(vals[0]), _np(ids[0]), s_ora, k, qn, float(xn.max()))
+
+
+@pytest.mark.parametrize("b", [1, 4])
+def test_mse_decode(quant_mse, tq_lib, cuda, b):
+    d = 128
+    x = synth.gaussian_rows(700, d, seed=6)
+    P = O.MseParams(d, b, 0)
+    c, xn, rn = O.mse_encode(P, x.numpy())
+    ref = O.mse_decode(P, c, xn)
+    got = _np(quant_mse(d, b).decode(_to_codes(tq_lib, c, xn, rn, cuda))[0]).astype(np.float64)
+    err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
+    assert err.max() <= 1e-4, err.max()
