@@ -338,29 +338,60 @@ def run_ours(args, cfg, rank, world, dist):
 
     nlaunch, kernel_names = count_launches(step) if not args.no_count else (None, [])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    sampler = ClockSampler(dev)
-    sampler.start()
-    sampler.wait_first()
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
+    # The step as one CUDA graph (the same public calls, captured once): its
+    # replays are the timed steps.  Per-call times come from a second timed
+    # pass of plain stream launches.
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step.run()
+            torch.cuda.synchronize()
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture unsupported: plain launches
+            print(f"graph capture failed ({e}); timing plain launches", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    sampler.start()
+    sampler.wait_first()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     for i in range(args.steps):
         flush.zero_()
-        step.run(evs[i])
+        if graph is not None:
+            gev[i][0].record()
+            graph.replay()
+            gev[i][1].record()
+        else:
+            step.run(evs[i])
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     t1 = time.time()
+    if graph is not None:  # per-call breakdown, plain launches
+        for i in range(args.steps):
+            flush.zero_()
+            step.run(evs[i])
+        torch.cuda.synchronize()
     time.sleep(0.3)
     sampler.stop()
     enc = [e[0].elapsed_time(e[1]) for e in evs]
     sco = [e[1].elapsed_time(e[2]) for e in evs]
     tpk = [e[2].elapsed_time(e[3]) for e in evs]
-    tot_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
+    if graph is not None:
+        tot_ms = sum(e[0].elapsed_time(e[1]) for e in gev)
+    else:
+        tot_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
     tot_ms, se, ss, st = rank_max(dist, [tot_ms, sum(enc), sum(sco), sum(tpk)], dev)
     K_ = args.steps
     ms_step = tot_ms / K_
@@ -461,6 +492,7 @@ def run_ours(args, cfg, rank, world, dist):
         "config": {"workload": f"{args.config}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
                    "d": cfg["d"], "b": cfg["b"], "queries_per_group": cfg["nq"], "k": cfg["k"],
                    "l2": "flushed (256 MB write) between timed steps",
+                   "launch": "CUDA graph of the step" if graph is not None else "stream launches",
                    "parallelism": f"dp{world} (independent batches per GPU)"},
         "encode": {"ms": round(enc_ms, 5),
                    "mvec_s": round(cfg["G"] * cfg["n"] / enc_ms / 1e3, 3),
@@ -585,6 +617,8 @@ def main():
     ap.add_argument("--config", default="kv", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain stream launches instead of replays of the step's CUDA graph")
     ap.add_argument("--no-count", action="store_true",
                     help="skip the profiler-based launch count (for runs under ncu)")
     args = ap.parse_args()

@@ -772,7 +772,10 @@ __global__ __launch_bounds__(512) void k_query_prep(const float* __restrict__ Pi
                                                     const float* __restrict__ S, int d, int nq,
                                                     const TQ* __restrict__ q,
                                                     float* __restrict__ qr,
-                                                    float* __restrict__ u) {
+                                                    float* __restrict__ u, int* err) {
+    // the call's device status word starts clean (the scoring kernels after
+    // this one on the stream may record a time-out in it)
+    if (err && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err = 0;
     extern __shared__ __align__(16) float sq[];  // [0, d): q   [d, 2d): qr
     constexpr int R = 8;  // rows per warp in flight
     const int g = blockIdx.y;
@@ -827,7 +830,7 @@ __global__ __launch_bounds__(512) void k_query_prep(const float* __restrict__ Pi
 // qr = Q Pi^T, u = qr S^T for every group: one fused launch for few queries,
 // else two fp32 SIMT GEMMs per group.
 int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const void* d_q,
-               int q_dtype, float* qr, float* u, cudaStream_t s) {
+               int q_dtype, float* qr, float* u, int* err, cudaStream_t s) {
     const size_t dd = (size_t)d * d;
     const size_t esz = (q_dtype == TQ_F32) ? 4 : 2;
     if (nq <= 32) {
@@ -836,16 +839,18 @@ int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const 
         if (q_dtype == TQ_F32) {
             TQ_TRY_CUDA(cudaFuncSetAttribute(k_query_prep<float>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-            k_query_prep<float><<<grid, 512, smem, s>>>(d_Pi, d_S, d, nq, (const float*)d_q, qr, u);
+            k_query_prep<float><<<grid, 512, smem, s>>>(d_Pi, d_S, d, nq, (const float*)d_q, qr, u,
+                                                        err);
         } else {
             TQ_TRY_CUDA(cudaFuncSetAttribute(k_query_prep<__nv_bfloat16>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
             k_query_prep<__nv_bfloat16><<<grid, 512, smem, s>>>(
-                d_Pi, d_S, d, nq, (const __nv_bfloat16*)d_q, qr, u);
+                d_Pi, d_S, d, nq, (const __nv_bfloat16*)d_q, qr, u, err);
         }
         TQ_CHECK_LAUNCH();
         return TQ_OK;
     }
+    if (err) TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
     for (int g = 0; g < G; ++g) {
         const void* qg = (const char*)d_q + (size_t)g * nq * d * esz;
         int rc = launch_sgemm(nq, d, d, qg, q_dtype, d, d_Pi + g * dd, true, d,
@@ -893,12 +898,11 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     int* err = (int*)d_ws;
     float* qr = (float*)((char*)d_ws + 256);
     float* u = (float*)((char*)qr + align256((size_t)G * nq * d * 4));
-    rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, s);
+    rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, err, s);
     if (rc) return rc;
     if (!is_mse(cb) && score_tc_supported(d, b, G, n, nq))
         return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
-    TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
     const KCodebook kc = make_kcodebook(cb);
     switch (b) {
         case 1: return launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, d_scores, nullptr, nullptr, s);
@@ -925,7 +929,7 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
     p += align256((size_t)G * nq * d * 4);
     float* u = (float*)p;
     p += align256((size_t)G * nq * d * 4);
-    rc = query_prep(d_Pi, is_mse(cb) ? nullptr : d_S, G, d, nq, d_q, q_dtype, qr, u, s);
+    rc = query_prep(d_Pi, is_mse(cb) ? nullptr : d_S, G, d, nq, d_q, q_dtype, qr, u, err, s);
     if (rc) return rc;
     const KCodebook kc = make_kcodebook(cb);
     const int64_t rows = (int64_t)G * nq;
@@ -949,7 +953,6 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
                                  s);
             nchunks = (int)ntm;
         } else {  // maxima per 256-key block
-            TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
             switch (b) {
                 case 1: rc = launch_score_b<1>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
                 case 2: rc = launch_score_b<2>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, sc, cm, cnt, s); break;
@@ -976,7 +979,6 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         return TQ_OK;
     }
     // fused: per-range best-K lists [G][nq][nblk][K], then the merge
-    TQ_TRY_CUDA(cudaMemsetAsync(err, 0, sizeof(int), s));
     float* pv = (float*)p;
     p += align256((size_t)rows * ntiles * k * 4);
     int64_t* pi = (int64_t*)p;

@@ -662,7 +662,7 @@ int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d
         ec = 14 - ec;
     }
     const float cscale = ldexpf(1.f, ec);
-    TQ_TRY_CUDA(cudaMemsetAsync(d_err, 0, sizeof(int), s));
+    // d_err was cleared by the query transform that precedes this kernel
     const KCodebook kc = make_kcodebook(cb);
     const int nqp = nq < kMaxNQ ? nq : kMaxNQ;
     const int ntm = (int)score_tc_tiles(n);
