@@ -35,6 +35,7 @@
 #include <cuda_fp16.h>
 
 #include "tq_internal.cuh"
+#include "tq_codes.cuh"
 #include "tq_sm100.cuh"
 
 namespace tq {
@@ -164,38 +165,6 @@ __device__ __forceinline__ float order_val(uint32_t k) {
 
 // 2^e for |e| < 127 (exact).
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
-
-// (w >> s) for s >= 0, (w << -s) for s < 0; s is a compile-time constant.
-template <int S>
-__device__ __forceinline__ uint32_t shr(uint32_t w) {
-    if constexpr (S >= 0) return w >> S;
-    else return w << (-S);
-}
-
-// Byte offset (pair field * 128) of the table entry of coordinates 2m, 2m + 1
-// (M < 16) of a 32-coordinate block; the layouts are those of pair_field.
-template <int B, int M>
-__device__ __forceinline__ uint32_t lut_offset_m(const uint32_t (&w)[4]) {
-    if constexpr (B == 4) {
-        return shr<8 * (M & 3) - 7>(w[M >> 2]) & (0xFFu << 7);
-    } else if constexpr (B == 2) {
-        return shr<4 * (M & 7) - 7>(w[M >> 3]) & (0xFu << 7);
-    } else {  // B == 3: 2-bit cell pair, then the two sign bits
-        return (shr<4 * (M & 7) - 7>(w[M >> 3]) & (0xFu << 7)) |
-               (shr<2 * M - 11>(w[2]) & (0x3u << 11));
-    }
-}
-
-template <int B>
-__device__ __forceinline__ uint32_t lut_offset(const uint32_t (&w)[4], int m) {
-    switch (m) {
-#define TQ_LO(M) case M: return lut_offset_m<B, M>(w);
-        TQ_LO(0) TQ_LO(1) TQ_LO(2) TQ_LO(3) TQ_LO(4) TQ_LO(5) TQ_LO(6) TQ_LO(7)
-        TQ_LO(8) TQ_LO(9) TQ_LO(10) TQ_LO(11) TQ_LO(12) TQ_LO(13) TQ_LO(14) TQ_LO(15)
-#undef TQ_LO
-    }
-    return 0u;
-}
 
 // Pair field of coordinates 2m, 2m + 1 (m < 16) of a 32-coordinate block.
 template <int B>
@@ -495,7 +464,7 @@ k_score_tc(const uint32_t* __restrict__ codes, const float* __restrict__ xnorm,
                     uint32_t chi[8], clo[8], sgn[8];
 #pragma unroll
                     for (int m = 0; m < 8; ++m) {
-                        const uint4 e = lds128(lut_s + (lut_offset<B>(wb, 8 * h + m) | lane16));
+                        const uint4 e = lds128(lut_s + (pair_offset<B>(wb, 8 * h + m) | lane16));
                         chi[m] = e.x;
                         clo[m] = e.y;
                         sgn[m] = e.z;
