@@ -29,9 +29,15 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
     switch (op) {
         case TQ_OP_BUILD:
             return 2 * align256(dd * 8) + 2 * align256((size_t)d * 8);
-        case TQ_OP_ENCODE:
+        case TQ_OP_ENCODE: {
             if (b < 1 || b > 4) return (size_t)-1;
-            return 256 + 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
+            // status word, Y, P, cell bytes; for the tensor-core GEMMs the bf16
+            // pieces of Pi, S and one operand chunk
+            size_t bytes = 256 + 2 * align256((size_t)chunk * d * 4) + align256((size_t)chunk * d);
+            if (encode_gemm_tc(d))
+                bytes += 2 * align256(3 * dd * 2) + align256((size_t)3 * chunk * d * 2);
+            return bytes;
+        }
         case TQ_OP_SCORE:  // status word, transformed queries
             return 256 + 2 * qbuf;
         case TQ_OP_TOPK:

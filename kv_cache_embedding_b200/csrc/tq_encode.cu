@@ -9,10 +9,12 @@
 // Portable path (any supported d; the only path of the MSE-only variant): per
 // group and row chunk
 //   k_rownorm      |x| in fp64 accumulation                       (E1)
-//   sgemm          Y = X Pi^T / |x|                                (E2)
+//   GEMM           Y = X Pi^T / |x|                                (E2)
 //   k_quantize     idx = #{beta_j <= y}, r = y - c[idx], |r|       (E3, E4)
-//   sgemm          P = R S^T                                       (E5)
+//   GEMM           P = R S^T                                       (E5)
 //   k_pack         fields idx | z -> code words                    (E3, E6)
+// The GEMMs run on the tensor cores (split bf16 pieces, tq_gemm_tc.cu) for
+// d >= 256, else as fp32 SIMT GEMMs (tq_gemm.cu).
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -125,6 +127,7 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
         return launch_encode_tc(cb, d_Pi, d_S, G, n, d_x, d_codes, d_xnorm, d_rnorm,
                                 (int*)d_ws, s);
     TQ_TRY_CUDA(cudaMemsetAsync(d_ws, 0, sizeof(int), s));
+    int* err = (int*)d_ws;
     const KCodebook kc = make_kcodebook(cb);
     const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;
     float* Y = (float*)((char*)d_ws + 256);
@@ -133,7 +136,20 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     const int W = words_per_vector(d, b);
     const size_t esz = (x_dtype == TQ_F32) ? 4 : 2;
     const size_t dd = (size_t)d * d;
+    // tensor-core GEMMs: bf16 pieces of Pi_g, S_g and of the chunk's operand
+    const bool tcg = encode_gemm_tc(d) && gemm_tc_supported(d, d);
+    __nv_bfloat16* PiP = (__nv_bfloat16*)(IX + align256((size_t)chunk * d));
+    __nv_bfloat16* SP = (__nv_bfloat16*)((char*)PiP + align256(3 * dd * 2));
+    __nv_bfloat16* AP = (__nv_bfloat16*)((char*)SP + align256(3 * dd * 2));
     for (int g = 0; g < G; ++g) {
+        if (tcg) {
+            int rc = split_bf16x3(d_Pi + g * dd, (int64_t)dd, PiP, s);
+            if (rc) return rc;
+            if (!mse) {
+                rc = split_bf16x3(d_S + g * dd, (int64_t)dd, SP, s);
+                if (rc) return rc;
+            }
+        }
         for (int64_t r0 = 0; r0 < n; r0 += chunk) {
             const int64_t rows = (n - r0) < chunk ? (n - r0) : chunk;
             const int64_t off = (int64_t)g * n + r0;
@@ -147,8 +163,21 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                 k_rownorm<__nv_bfloat16><<<wblocks, 256, 0, s>>>((const __nv_bfloat16*)xg, rows,
                                                                  d, xn);
             TQ_CHECK_LAUNCH();
-            int rc = launch_sgemm((int)rows, d, d, xg, x_dtype, d, d_Pi + g * dd, true, d, Y, d,
+            int rc;
+            if (tcg) {  // Y = X Pi^T / |x| on the tensor cores
+                const __nv_bfloat16* A = (const __nv_bfloat16*)xg;  // bf16 keys: one exact piece
+                int pa = 1;
+                if (x_dtype == TQ_F32) {
+                    rc = split_bf16x3((const float*)xg, rows * d, AP, s);
+                    if (rc) return rc;
+                    A = AP;
+                    pa = 3;
+                }
+                rc = launch_gemm_tc((int)rows, d, d, A, pa, PiP, Y, d, xn, 1, err, s);
+            } else {
+                rc = launch_sgemm((int)rows, d, d, xg, x_dtype, d, d_Pi + g * dd, true, d, Y, d,
                                   xn, 1, s);
+            }
             if (rc) return rc;
             k_quantize<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rn);
             TQ_CHECK_LAUNCH();
@@ -163,8 +192,14 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                 TQ_CHECK_LAUNCH();
                 continue;
             }
-            rc = launch_sgemm((int)rows, d, d, Y, TQ_F32, d, d_S + g * dd, true, d, P, d, nullptr,
-                              0, s);
+            if (tcg) {  // P = R S^T on the tensor cores
+                rc = split_bf16x3(Y, rows * d, AP, s);
+                if (rc) return rc;
+                rc = launch_gemm_tc((int)rows, d, d, AP, 3, SP, P, d, nullptr, 0, err, s);
+            } else {
+                rc = launch_sgemm((int)rows, d, d, Y, TQ_F32, d, d_S + g * dd, true, d, P, d,
+                                  nullptr, 0, s);
+            }
             if (rc) return rc;
             switch (b) {
                 case 1: k_pack<1, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;

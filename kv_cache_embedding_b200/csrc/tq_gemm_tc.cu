@@ -1,0 +1,330 @@
+// FP32-accurate dense products of the encode path on the sm_100a tensor
+// cores, for the dimensions the fused d = 128 kernel does not cover (E2 the
+// rotation, E5 the QJL projection):
+//
+//   C[m][n] = scale(m) * sum_k A[m][k] * B[n][k]     (A [M][K], B [N][K], K-contiguous)
+//   scale(m) = 1 (mode 0), 1/row_scale[m] or 0 if row_scale[m] == 0 (mode 1)
+//
+// Pages: quant_prune_distill #674 (rotate by a random orthogonal matrix; QJL:
+// multiply the residual by a random matrix, keep the sign); RecSysChannel #256
+// caveat 1 (normalise, multiply by a random matrix).
+//
+// Precision: both operands are split into bf16 pieces, A = a1 + a2 + a3 (one
+// piece when A is bf16 already) and B = b1 + b2 + b3 (each to ~2^-24 of the
+// value); the MMAs sum a1 b1 + a1 b2 + a2 b1 + a1 b3 + a2 b2 + a3 b1 (bf16 x
+// bf16 products are exact in fp32).  The accumulator in tensor memory is
+// restarted every 128 of K and the chunk sums are added in fp32 registers,
+// so the rounding of an output stays near that of a 128-term fp32 sum for
+// any K, as in the SIMT path.
+//
+// Tiles: 128 rows (MMA M) x 128 columns (MMA N), K in blocks of 64 staged by
+// TMA with the 128-byte swizzle (two stages).  Warp 0 issues the TMA loads,
+// warp 1 owns tensor memory and issues the MMAs, warps 2-5 (one per TMEM lane
+// quarter) add up the chunk sums and store the tile.  Every wait is bounded
+// (1 s); a warp that gives up sets the abort flag and the status word.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "tq_internal.cuh"
+#include "tq_sm100.cuh"
+
+namespace tq {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTM = 128, kTN = 128, kKB = 64;        // tile rows, columns, K block
+constexpr int kPieceBytes = kTM * kKB * 2;            // one bf16 piece of a tile (16 KB)
+constexpr int kStages = 2;
+constexpr int kThreads = 32 * 6;
+constexpr uint32_t kTmemCols = 2 * kTN;               // two chunk accumulators
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t kIdesc = idesc_f16(1, kTM, kTN);   // bf16 x bf16 -> f32, K-major A and B
+
+struct SmemG {
+    uint8_t a[kStages][3][kPieceBytes];  // A pieces (1024-aligned, first)
+    uint8_t b[kStages][3][kPieceBytes];  // B pieces
+    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], mma_done;
+    uint32_t tmem_base;
+    int abort;
+    int zero;
+};
+constexpr size_t kSmemBytes = sizeof(SmemG) + 1024;
+
+__device__ __forceinline__ bool give_up(volatile int* abort, int* err, int site) {
+    *abort = 1;
+    atomicCAS(err, 0, TQ_ERR_DEVICE_TIMEOUT * 1000 - site);
+    return false;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort, kWaitNs);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, int32_t z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, one CTA.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+          int M, int N, int K, int pa, float* __restrict__ C, int64_t ldc,
+          const float* __restrict__ row_scale, int scale_mode, int* __restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    SmemG& sm = *reinterpret_cast<SmemG*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    volatile int* abort = &sm.abort;
+    const int tm = (M + kTM - 1) / kTM, tn = N / kTN;
+    const int tiles = tm * tn;
+    const int nkb = K / kKB;            // K blocks per tile
+    const int nch = nkb / 2;            // 128-wide K chunks per tile
+    const uint32_t stage_tx = (uint32_t)(pa + 3) * kPieceBytes;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.acc_full[i], 1);
+            mbar_init(&sm.acc_empty[i], 4);
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.abort = 0;
+        sm.zero = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer ----------------
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int m0 = (t / tn) * kTM, n0 = (t % tn) * kTN;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % kStages;
+                if (it >= (uint32_t)kStages &&
+                    !mbar_wait(&sm.empty[s], ((it / kStages) - 1) & 1, abort, kWaitNs)) {
+                    ok = give_up(abort, err, 41);
+                    break;
+                }
+                mbar_arrive_expect_tx(&sm.full[s], stage_tx);
+                for (int p = 0; p < pa; ++p)
+                    tma_load_3d(sm.a[s][p], &tmap_a, kb * kKB, m0, p, &sm.full[s]);
+                for (int p = 0; p < 3; ++p)
+                    tma_load_3d(sm.b[s][p], &tmap_b, kb * kKB, n0, p, &sm.full[s]);
+            }
+        }
+        // no TMA write may still be in flight when the CTA exits
+        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0); j < it; ++j)
+            mbar_wait(&sm.full[j % kStages], (j / kStages) & 1, &sm.zero, kWaitNs);
+    } else if (warp == 1 && lane == 0) {
+        // ---------------- MMA issuer ----------------
+        // products in order: a1 b1, a1 b2, a2 b1, a1 b3, a2 b2, a3 b1 (pa = 3);
+        // a1 b1, a1 b2, a1 b3 (pa = 1)
+        const int np = (pa == 3) ? 6 : 3;
+        const int pa_of[6] = {0, 0, 1, 0, 1, 2}, pb_of6[6] = {0, 1, 0, 2, 1, 0};
+        const int pb_of3[3] = {0, 1, 2};
+        uint32_t it = 0, cc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int c = 0; c < nch && ok; ++c, ++cc) {
+                const uint32_t ab = cc & 1;
+                if (cc >= 2 && !mbar_wait(&sm.acc_empty[ab], ((cc >> 1) - 1) & 1, abort, kWaitNs)) {
+                    ok = give_up(abort, err, 42);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tbase + ab * kTN;
+                for (int h = 0; h < 2; ++h, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&sm.full[s], (it / kStages) & 1, abort, kWaitNs)) {
+                        ok = give_up(abort, err, 43);
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int q = 0; q < np; ++q) {
+                        const int ia = (pa == 3) ? pa_of[q] : 0;
+                        const int ib = (pa == 3) ? pb_of6[q] : pb_of3[q];
+                        const uint32_t as = smem_u32(sm.a[s][ia]), bs = smem_u32(sm.b[s][ib]);
+#pragma unroll
+                        for (int ks = 0; ks < kKB / 16; ++ks)
+                            mma_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
+                                   smem_desc_kmajor_sw128(bs + ks * 32), kIdesc,
+                                   (h | q | ks) != 0);
+                    }
+                    tc_commit(&sm.empty[s]);
+                }
+                if (ok) tc_commit(&sm.acc_full[ab]);
+            }
+        }
+        // every issued MMA completes before tensor memory is released
+        tc_commit(&sm.mma_done);
+        mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
+    } else if (warp >= 2) {
+        // ---------------- chunk sums and stores ----------------
+        const int q = warp & 3;  // TMEM lane quarter: tile rows 32 q .. 32 q + 31
+        const uint32_t lane_addr = tbase + ((uint32_t)(32 * q) << 16);
+        uint32_t cc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int m0 = (t / tn) * kTM, n0 = (t % tn) * kTN;
+            float sum[kTN];
+#pragma unroll
+            for (int j = 0; j < kTN; ++j) sum[j] = 0.f;
+            for (int c = 0; c < nch; ++c, ++cc) {
+                const uint32_t ab = cc & 1;
+                if (!warp_wait(&sm.acc_full[ab], (cc >> 1) & 1, abort)) {
+                    ok = give_up(abort, err, 44);
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int j0 = 0; j0 < kTN; j0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + ab * kTN + (uint32_t)j0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sum[j0 + j] += __uint_as_float(v[j]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
+            }
+            if (!ok) break;
+            const int64_t row = (int64_t)m0 + 32 * q + lane;
+            if (row < M) {
+                float sc = 1.f;
+                if (scale_mode == 1) {
+                    const float r = row_scale[row];
+                    sc = (r != 0.f) ? 1.f / r : 0.f;
+                }
+                float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
+#pragma unroll
+                for (int j = 0; j < kTN; j += 4)
+                    dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
+                                             sum[j + 3] * sc);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tbase, kTmemCols);
+}
+
+// out[p][r][k]: the bf16 pieces of x (fp32), x = out[0] + out[1] + out[2] to
+// ~2^-24 of |x| (each piece the bf16 rounding of what the previous ones left).
+__global__ void k_split3(const float* __restrict__ x, int64_t count, __nv_bfloat16* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= count) return;
+    const float v = x[i];
+    const __nv_bfloat16 p1 = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(p1);
+    const __nv_bfloat16 p2 = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 p3 = __float2bfloat16_rn(r1 - __bfloat162float(p2));
+    out[i] = p1;
+    out[count + i] = p2;
+    out[2 * count + i] = p3;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tiled_encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D map over bf16 pieces [pieces][rows][K] (K contiguous), box 64 x 128 x 1,
+// 128-byte swizzle; rows beyond `rows` read as zeros.
+bool make_piece_map(CUtensorMap* map, const void* base, int pieces, int64_t rows, int K) {
+    EncodeTiledFn enc = tiled_encoder();
+    if (!enc) return false;
+    const cuuint64_t gdim[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)pieces};
+    const cuuint64_t gstride[2] = {(cuuint64_t)K * 2, (cuuint64_t)rows * K * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kKB, (cuuint32_t)kTM, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gdim, gstride, box,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int N, int K) {
+    return N > 0 && K > 0 && N % kTN == 0 && K % 128 == 0 && tiled_encoder() != nullptr;
+}
+
+int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t s) {
+    if (count <= 0) return TQ_OK;
+    k_split3<<<(unsigned)((count + 255) / 256), 256, 0, s>>>(x, count, out);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
+                   float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
+                   cudaStream_t s) {
+    if (M <= 0) return TQ_OK;
+    if (!gemm_tc_supported(N, K) || (pa != 1 && pa != 3) || ldc % 4) return TQ_ERR_ARG;
+    CUtensorMap ma, mb;
+    if (!make_piece_map(&ma, A, pa, M, K) || !make_piece_map(&mb, B, 3, N, K)) return TQ_ERR_CUDA;
+    int dev = 0, nsm = 0;
+    TQ_TRY_CUDA(cudaGetDevice(&dev));
+    TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    const int64_t tiles = (int64_t)((M + kTM - 1) / kTM) * (N / kTN);
+    const int nctas = (int)(tiles < nsm ? tiles : nsm);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes));
+    k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, C, ldc, row_scale,
+                                                  scale_mode, d_err);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+}  // namespace tq

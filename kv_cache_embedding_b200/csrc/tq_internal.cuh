@@ -80,6 +80,16 @@ int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const
                  bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
                  cudaStream_t s);
 bool encode_tc_supported(int d, int x_dtype, int G, int64_t n);
+// Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from bf16
+// pieces of A ([pa][M][K], pa = 1 or 3) and B ([3][N][K]); d_err as the
+// encode kernels' status word.
+bool gemm_tc_supported(int N, int K);
+int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t s);
+int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
+                   float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
+                   cudaStream_t s);
+// The encode path's dense products run on the tensor-core GEMM for d >= 256.
+inline bool encode_gemm_tc(int d) { return d >= 256; }
 bool score_tc_supported(int d, int b, int G, int64_t n, int nq);
 int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
                     const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,

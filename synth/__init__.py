@@ -83,11 +83,16 @@ def random_records(n, words, seed=11, norm_range=(0.5, 2.0), rnorm_range=(0.0, 0
     `words` uint32 words per record (every bit pattern is a valid record of
     the packed layouts), plus per-record norms.  Returns (codes [n, words]
     uint32 numpy, xnorm [n] fp32, rnorm [n] fp32) on the CPU."""
+    import numpy as np
     g = _gen(seed, "cpu")
-    w = torch.randint(0, 1 << 32, (n, words), generator=g, dtype=torch.int64)
+    w = np.empty((n, words), dtype=np.uint32)
+    step = max(1, (1 << 22) // max(words, 1))  # rows per draw (bounded host memory)
+    for r0 in range(0, n, step):
+        r1 = min(n, r0 + step)
+        w[r0:r1] = torch.randint(0, 1 << 32, (r1 - r0, words), generator=g,
+                                 dtype=torch.int64).numpy().astype(np.uint32)
     lo, hi = norm_range
     xn = torch.rand(n, generator=g) * (hi - lo) + lo
     rlo, rhi = rnorm_range
     rn = torch.rand(n, generator=g) * (rhi - rlo) + rlo
-    return (w.to(torch.int64).numpy().astype("uint32"), xn.numpy().astype("float32"),
-            rn.numpy().astype("float32"))
+    return w, xn.numpy().astype("float32"), rn.numpy().astype("float32")

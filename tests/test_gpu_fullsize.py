@@ -1,0 +1,120 @@
+"""Parity at the workloads' full sizes, in the launch configuration the
+benchmark times: the whole workload runs on the GPU, and the oracle checks a
+seeded sample of encoded rows (codes, norms) it computes from the same
+inputs.  Scoring and top-k at full size run over seeded random records (the
+oracle takes no input from the CUDA path); the oracle checks sampled scores
+and the top-k of a few queries over every record.
+
+Workloads (shapes of the pages'): KV keys bf16 [8, 32768, 128] (b = 2, 3, 4),
+decode-shaped scoring over 131072 tokens, embedding search 1e6 x 1536 fp32
+unit rows (b = 2, 4; top-10), large-d 1e6 x 3072 (b = 1..4 encode)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import oracle as O
+from tests import parity as PT
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _check_sampled_encode(tq_lib, quant, x_dev, d, b, G, n, rows, seed_base=0):
+    codes = quant.encode(x_dev)
+    torch.cuda.synchronize()
+    for g in range(G):
+        P = O.Params(d, b, seed_base + g)
+        xs = x_dev[g, rows].float().cpu().to(torch.float64).numpy()
+        ora = O.encode(P, xs, diagnostics=True)
+        gpu = (_np(codes.codes[g, rows]).view(np.uint32), _np(codes.xnorm[g, rows]),
+               _np(codes.rnorm[g, rows]))
+        PT.compare_encode(d, b, P.beta, gpu, ora)
+    return codes
+
+
+@pytest.mark.parametrize("b", [2, 3, 4])
+def test_kv_keys_full_size(tq_lib, cuda, b):
+    """[8, 32768, 128] bf16 through the fused tensor-core kernel (148 CTAs)."""
+    G, n, d = 8, 32768, 128
+    x = synth.kv_keys(G, n, d, seed=1, device=cuda)
+    quant = tq_lib.TurboQuant(d, b, seed=0, groups=G, device=cuda)
+    rows = synth.sample_rows(n, 384, seed=7).to(cuda)
+    _check_sampled_encode(tq_lib, quant, x, d, b, G, n, rows)
+
+
+def _records_on_device(tq_lib, recs, cuda):
+    return tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+
+
+def test_decode_logits_full_size(tq_lib, cuda):
+    """131072 tokens x 8 KV heads, 32 query heads (GQA 4:1), b = 4: sampled
+    encode parity of the full encode, then every logit over 8 x 131072 seeded
+    records, checked on a sample of tokens."""
+    G, n, d, b, per = 8, 131072, 128, 4, 4
+    x = synth.kv_keys(G, n, d, seed=1, device=cuda)
+    q = synth.kv_queries(G * per, G, d, seed=2, device=cuda, key_seed=1)
+    quant = tq_lib.TurboQuant(d, b, seed=0, groups=G, device=cuda)
+    rows = synth.sample_rows(n, 256, seed=8)
+    _check_sampled_encode(tq_lib, quant, x, d, b, G, n, rows.to(cuda))
+    recs = [synth.random_records(n, b * d // 32, seed=70 + g) for g in range(G)]
+    s = quant.score(_records_on_device(tq_lib, recs, cuda), q)
+    torch.cuda.synchronize()
+    r = rows.numpy()
+    for g in range(G):
+        c, xn, rn = recs[g]
+        qg = q[g].float().cpu().to(torch.float64).numpy()
+        s_ora = O.score(O.Params(d, b, g), c[r], xn[r], rn[r], qg)
+        PT.compare_scores(_np(s[g][:, rows.to(cuda)]), s_ora, np.linalg.norm(qg, axis=1),
+                          xn[r].astype(np.float64))
+
+
+@pytest.mark.parametrize("b", [2, 4])
+def test_embedding_search_full_size(tq_lib, cuda, b):
+    """1e6 x 1536 fp32 unit rows, 1024 queries, top-10: sampled encode parity
+    of the full encode; the top-10 of all 1024 queries over 1e6 seeded records,
+    4 of them checked against the oracle's scores of every record."""
+    n, d, nq, k = 1_000_000, 1536, 1024, 10
+    x = synth.gaussian_rows(n, d, seed=1, device=cuda, unit=True)[None]
+    q = synth.gaussian_rows(nq, d, seed=2, device=cuda, unit=True)[None]
+    quant = tq_lib.TurboQuant(d, b, seed=0, groups=1, device=cuda)
+    rows = synth.sample_rows(n, 128, seed=9).to(cuda)
+    _check_sampled_encode(tq_lib, quant, x, d, b, 1, n, rows)
+    del x
+    recs = [synth.random_records(n, b * d // 32, seed=80)]
+    vals, ids = quant.topk(_records_on_device(tq_lib, recs, cuda), q, k)
+    torch.cuda.synchronize()
+    pick = [0, 1, 511, 1023]
+    c, xn, rn = recs[0]
+    qs = q[0, pick].cpu().to(torch.float64).numpy()
+    s_ora = O.score(O.Params(d, b, 0), c, xn, rn, qs)
+    PT.compare_topk(_np(vals[0, pick]), _np(ids[0, pick]), s_ora, k, np.ones(len(pick)),
+                    float(xn.max()))
+
+
+@pytest.mark.parametrize("b", [1, 2, 3, 4])
+def test_large_d_full_size(tq_lib, cuda, b):
+    """1e6 x 3072 fp32 rows with norms U[0.5, 2]: sampled encode parity; then
+    256 queries scored over 1e6 seeded records, checked on sampled records."""
+    n, d, nq = 1_000_000, 3072, 256
+    x = synth.gaussian_rows(n, d, seed=1, device=cuda)[None]
+    quant = tq_lib.TurboQuant(d, b, seed=0, groups=1, device=cuda)
+    rows = synth.sample_rows(n, 48, seed=10)
+    _check_sampled_encode(tq_lib, quant, x, d, b, 1, n, rows.to(cuda))
+    del x
+    q = synth.gaussian_rows(nq, d, seed=2, device=cuda, norm_range=None)[None]
+    recs = [synth.random_records(n, b * d // 32, seed=90)]
+    s = quant.score(_records_on_device(tq_lib, recs, cuda), q)
+    torch.cuda.synchronize()
+    r = rows.numpy()
+    c, xn, rn = recs[0]
+    qs = q[0].cpu().to(torch.float64).numpy()
+    s_ora = O.score(O.Params(d, b, 0), c[r], xn[r], rn[r], qs)
+    PT.compare_scores(_np(s[0][:, rows.to(cuda)]), s_ora, np.linalg.norm(qs, axis=1),
+                      xn[r].astype(np.float64))

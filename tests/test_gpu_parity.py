@@ -106,6 +106,19 @@ def test_encode_large_dims(quant, oparams, d, b):
         PT.compare_encode(d, b, P.beta, gpu, ora)
 
 
+@pytest.mark.parametrize("d,b,G,n", [(256, 4, 2, 700), (512, 3, 1, 1000), (384, 1, 3, 129)])
+def test_encode_tensor_core_gemm_shapes(quant, oparams, d, b, G, n):
+    """d >= 256: the rotation and QJL products run as split-precision
+    tensor-core GEMMs; bf16 keys (one exact piece) and fp32 rows (three
+    pieces), ragged last tiles, several groups."""
+    if b == 4:
+        x = synth.kv_keys(G, n, d, seed=3)
+    else:
+        x = synth.gaussian_rows(G * n, d, seed=3).reshape(G, n, d)
+    for gpu, ora, P in _encode_both(quant, oparams, x, d, b, groups=G):
+        PT.compare_encode(d, b, P.beta, gpu, ora)
+
+
 def test_encode_edge_rows(quant, oparams):
     d, b = 128, 4
     x = synth.gaussian_rows(40, d, seed=3)
