@@ -38,10 +38,10 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
                 bytes += 2 * align256(3 * dd * 2) + align256((size_t)3 * chunk * d * 2);
             return bytes;
         }
-        case TQ_OP_SCORE:  // status word, transformed queries
-            return 256 + 2 * qbuf;
+        case TQ_OP_SCORE:  // status word, transformed queries (, GEMM operands)
+            return 256 + 2 * qbuf + (score_gemm_supported(d, nq) ? score_gemm_workspace(d, n, nq) : 0);
         case TQ_OP_TOPK:
-            return tq::topk_workspace_bytes(d, b, G, n, nq, k, topk_materialized(G, n, nq));
+            return tq::topk_workspace_bytes(d, b, G, n, nq, k, topk_materialized(d, G, n, nq));
         case TQ_OP_DECODE:
             return 2 * align256((size_t)chunk * d * 4);
         case TQ_OP_EXACT:
@@ -56,11 +56,12 @@ size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool 
     (void)b;
     const size_t qbuf = align256((size_t)G * nq * d * 4);
     if (materialize) {
-        // scores, maxima per 128-key tile, counters, candidate lists
+        // scores, maxima per 128-key tile, counters, candidate lists (, GEMM operands)
         const int64_t ntm = (n + 127) / 128;
         return 256 + 2 * qbuf + align256((size_t)G * nq * n * 4) +
                align256((size_t)G * nq * ntm * 4) + align256((size_t)G * nq * 8) +
-               2 * align256((size_t)G * nq * kTopkCandidates * 4);
+               2 * align256((size_t)G * nq * kTopkCandidates * 4) +
+               (score_gemm_supported(d, nq) ? score_gemm_workspace(d, n, nq) : 0);
     }
     const int64_t ntiles = (n + kTopkTile - 1) / kTopkTile;
     return 256 + 2 * qbuf + align256((size_t)G * nq * ntiles * k * 4) +

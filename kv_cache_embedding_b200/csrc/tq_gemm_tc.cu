@@ -3,7 +3,12 @@
 // rotation, E5 the QJL projection):
 //
 //   C[m][n] = scale(m) * sum_k A[m][k] * B[n][k]     (A [M][K], B [N][K], K-contiguous)
-//   scale(m) = 1 (mode 0), 1/row_scale[m] or 0 if row_scale[m] == 0 (mode 1)
+//   scale(m) = 1 (mode 0), 1/row_scale[m] or 0 if row_scale[m] == 0 (mode 1),
+//              row_scale[m] (mode 2)
+// stored row-major (C[m * ldc + n]) or transposed (C[n * ldc + m], columns
+// n < n_store only), optionally with the maximum of every 128-row tile per
+// column (tmax[n * ldt + m / 128]).  The transposed form with tile maxima is
+// the decoded-key scoring of many queries: rows = keys, columns = queries.
 //
 // Pages: quant_prune_distill #674 (rotate by a random orthogonal matrix; QJL:
 // multiply the residual by a random matrix, keep the sign); RecSysChannel #256
@@ -11,8 +16,10 @@
 //
 // Precision: both operands are split into bf16 pieces, A = a1 + a2 + a3 (one
 // piece when A is bf16 already) and B = b1 + b2 + b3 (each to ~2^-24 of the
-// value); the MMAs sum a1 b1 + a1 b2 + a2 b1 + a1 b3 + a2 b2 + a3 b1 (bf16 x
-// bf16 products are exact in fp32).  The accumulator in tensor memory is
+// value); the MMAs sum the products a_i b_j with i + j < max(pa, pb) (pa, pb
+// pieces of A and B: 3 x 3 -> a1 b1 + a1 b2 + a2 b1 + a1 b3 + a2 b2 + a3 b1;
+// 1 x 3 -> a1 b1 + a1 b2 + a1 b3; 2 x 2 -> a1 b1 + a1 b2 + a2 b1, ~2^-16);
+// bf16 x bf16 products are exact in fp32.  The accumulator in tensor memory is
 // restarted every 128 of K and the chunk sums are added in fp32 registers,
 // so the rounding of an output stays near that of a 128-term fp32 sum for
 // any K, as in the SIMT path.
@@ -46,7 +53,8 @@ constexpr uint32_t kIdesc = idesc_f16(1, kTM, kTN);   // bf16 x bf16 -> f32, K-m
 struct SmemG {
     uint8_t a[kStages][3][kPieceBytes];  // A pieces (1024-aligned, first)
     uint8_t b[kStages][3][kPieceBytes];  // B pieces
-    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], mma_done;
+    float tkey[4][kTN];                  // per epilogue warp: its 32 rows' maximum per column
+    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], mma_done, tmax_bar, tmax_bar2;
     uint32_t tmem_base;
     int abort;
     int zero;
@@ -86,8 +94,9 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-          int M, int N, int K, int pa, float* __restrict__ C, int64_t ldc,
-          const float* __restrict__ row_scale, int scale_mode, int* __restrict__ err) {
+          int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
+          const float* __restrict__ row_scale, int scale_mode, int transposed, int n_store,
+          float* __restrict__ tmax, int64_t ldt, int* __restrict__ err) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     SmemG& sm = *reinterpret_cast<SmemG*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -97,7 +106,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
     const int tiles = tm * tn;
     const int nkb = K / kKB;            // K blocks per tile
     const int nch = nkb / 2;            // 128-wide K chunks per tile
-    const uint32_t stage_tx = (uint32_t)(pa + 3) * kPieceBytes;
+    const uint32_t stage_tx = (uint32_t)(pa + pb) * kPieceBytes;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -109,6 +118,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
             mbar_init(&sm.acc_empty[i], 4);
         }
         mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.tmax_bar, 4);
+        mbar_init(&sm.tmax_bar2, 4);
         sm.abort = 0;
         sm.zero = 0;
         fence_mbar_init();
@@ -142,7 +153,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
                 mbar_arrive_expect_tx(&sm.full[s], stage_tx);
                 for (int p = 0; p < pa; ++p)
                     tma_load_3d(sm.a[s][p], &tmap_a, kb * kKB, m0, p, &sm.full[s]);
-                for (int p = 0; p < 3; ++p)
+                for (int p = 0; p < pb; ++p)
                     tma_load_3d(sm.b[s][p], &tmap_b, kb * kKB, n0, p, &sm.full[s]);
             }
         }
@@ -151,11 +162,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
             mbar_wait(&sm.full[j % kStages], (j / kStages) & 1, &sm.zero, kWaitNs);
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer ----------------
-        // products in order: a1 b1, a1 b2, a2 b1, a1 b3, a2 b2, a3 b1 (pa = 3);
-        // a1 b1, a1 b2, a1 b3 (pa = 1)
-        const int np = (pa == 3) ? 6 : 3;
-        const int pa_of[6] = {0, 0, 1, 0, 1, 2}, pb_of6[6] = {0, 1, 0, 2, 1, 0};
-        const int pb_of3[3] = {0, 1, 2};
+        // products a_i b_j with i + j < max(pa, pb), by increasing i + j
+        int pi_[6], pj_[6], np = 0;
+        const int pmax = pa > pb ? pa : pb;
+        for (int sij = 0; sij < pmax; ++sij)
+            for (int i = 0; i <= sij; ++i)
+                if (i < pa && sij - i < pb) {
+                    pi_[np] = i;
+                    pj_[np] = sij - i;
+                    ++np;
+                }
         uint32_t it = 0, cc = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
@@ -175,9 +191,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
                     }
                     tc_fence_after();
                     for (int q = 0; q < np; ++q) {
-                        const int ia = (pa == 3) ? pa_of[q] : 0;
-                        const int ib = (pa == 3) ? pb_of6[q] : pb_of3[q];
-                        const uint32_t as = smem_u32(sm.a[s][ia]), bs = smem_u32(sm.b[s][ib]);
+                        const uint32_t as = smem_u32(sm.a[s][pi_[q]]), bs = smem_u32(sm.b[s][pj_[q]]);
 #pragma unroll
                         for (int ks = 0; ks < kKB / 16; ++ks)
                             mma_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
@@ -196,7 +210,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
         // ---------------- chunk sums and stores ----------------
         const int q = warp & 3;  // TMEM lane quarter: tile rows 32 q .. 32 q + 31
         const uint32_t lane_addr = tbase + ((uint32_t)(32 * q) << 16);
-        uint32_t cc = 0;
+        uint32_t cc = 0, tb = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const int m0 = (t / tn) * kTM, n0 = (t % tn) * kTN;
@@ -224,17 +238,61 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
             }
             if (!ok) break;
             const int64_t row = (int64_t)m0 + 32 * q + lane;
-            if (row < M) {
-                float sc = 1.f;
-                if (scale_mode == 1) {
-                    const float r = row_scale[row];
-                    sc = (r != 0.f) ? 1.f / r : 0.f;
-                }
-                float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
+            const bool live = row < M;
+            float sc = 1.f;
+            if (live && scale_mode == 1) {
+                const float r = row_scale[row];
+                sc = (r != 0.f) ? 1.f / r : 0.f;
+            } else if (live && scale_mode == 2) {
+                sc = row_scale[row];
+            }
+            if (!transposed) {
+                if (live) {
+                    float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
 #pragma unroll
-                for (int j = 0; j < kTN; j += 4)
-                    dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
-                                             sum[j + 3] * sc);
+                    for (int j = 0; j < kTN; j += 4)
+                        dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
+                                                 sum[j + 3] * sc);
+                }
+            } else {
+                // column j of the tile -> C[(n0 + j) * ldc + row]: a warp writes 32
+                // consecutive rows of each column
+#pragma unroll
+                for (int j = 0; j < kTN; ++j) {
+                    const float v = sum[j] * sc;
+                    if (live && n0 + j < n_store) C[(int64_t)(n0 + j) * ldc + row] = v;
+                    if (tmax) {  // the tile's maximum per column, 4 warps merged in shared memory
+                        float m = live ? v : -INFINITY;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (lane == 0) sm.tkey[q][j] = m;
+                    }
+                }
+                if (tmax) {
+                    // the 4 epilogue warps meet on a bounded barrier, then each
+                    // writes the maxima of 32 columns
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.tmax_bar);
+                    if (!warp_wait(&sm.tmax_bar, tb & 1, abort)) {
+                        ok = give_up(abort, err, 45);
+                        break;
+                    }
+                    ++tb;
+                    const int j = 32 * q + lane;
+                    if (n0 + j < n_store)
+                        tmax[(int64_t)(n0 + j) * ldt + m0 / kTM] =
+                            fmaxf(fmaxf(sm.tkey[0][j], sm.tkey[1][j]),
+                                  fmaxf(sm.tkey[2][j], sm.tkey[3][j]));
+                    // the slots are rewritten only after the next tile's barrier,
+                    // which every warp reaches after this read
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.tmax_bar2);
+                    if (!warp_wait(&sm.tmax_bar2, (tb - 1) & 1, abort)) {
+                        ok = give_up(abort, err, 46);
+                        break;
+                    }
+                }
             }
         }
     }
@@ -309,11 +367,13 @@ int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t
 
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
-                   cudaStream_t s) {
+                   cudaStream_t s, int pb, bool transposed, int n_store, float* tmax,
+                   int64_t ldt) {
     if (M <= 0) return TQ_OK;
-    if (!gemm_tc_supported(N, K) || (pa != 1 && pa != 3) || ldc % 4) return TQ_ERR_ARG;
+    if (!gemm_tc_supported(N, K) || pa < 1 || pa > 3 || pb < 1 || pb > 3) return TQ_ERR_ARG;
+    if (!transposed && ldc % 4) return TQ_ERR_ARG;
     CUtensorMap ma, mb;
-    if (!make_piece_map(&ma, A, pa, M, K) || !make_piece_map(&mb, B, 3, N, K)) return TQ_ERR_CUDA;
+    if (!make_piece_map(&ma, A, pa, M, K) || !make_piece_map(&mb, B, pb, N, K)) return TQ_ERR_CUDA;
     int dev = 0, nsm = 0;
     TQ_TRY_CUDA(cudaGetDevice(&dev));
     TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
@@ -321,8 +381,9 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     const int nctas = (int)(tiles < nsm ? tiles : nsm);
     TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kSmemBytes));
-    k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, C, ldc, row_scale,
-                                                  scale_mode, d_err);
+    k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
+                                                  scale_mode, transposed ? 1 : 0, n_store, tmax,
+                                                  ldt, d_err);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }

@@ -56,9 +56,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // searches run the fused score + running-list kernel instead.
 constexpr int64_t kTopkMaterialize = (int64_t)1 << 24;
 constexpr int kTopkCandidates = 4096;  // gathered candidates per row on that path
-inline bool topk_materialized(int G, int64_t n, int nq) {
-    return (int64_t)G * nq * n <= kTopkMaterialize;
-}
+// (also when the scores come from the decoded-key GEMM, whatever their number)
+bool topk_materialized(int d, int G, int64_t n, int nq);
 
 inline bool valid_db(int d, int b) {
     return d >= kMinD && d <= kMaxD && d % 128 == 0 && b >= 1 && b <= 4;
@@ -87,9 +86,20 @@ bool gemm_tc_supported(int N, int K);
 int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t s);
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
-                   cudaStream_t s);
+                   cudaStream_t s, int pb = 3, bool transposed = false, int n_store = 0,
+                   float* tmax = nullptr, int64_t ldt = 0);
 // The encode path's dense products run on the tensor-core GEMM for d >= 256.
 inline bool encode_gemm_tc(int d) { return d >= 256; }
+// Scoring of many queries at d >= 256 as a GEMM over decoded keys
+// (tq_score_gemm.cu): scores [G][nq][n] (and per-128-key maxima [G][nq][ntm]).
+constexpr int kScoreGemmMinQueries = 64;
+constexpr int64_t kScoreGemmChunk = 32768;  // keys decoded per GEMM
+bool score_gemm_supported(int d, int nq);
+size_t score_gemm_workspace(int d, int64_t n, int nq);
+int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
+               const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,
+               const float* u, float* scores, float* tmax, int64_t ntm, void* op_ws, int* d_err,
+               cudaStream_t s);
 bool score_tc_supported(int d, int b, int G, int64_t n, int nq);
 int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
                     const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,

@@ -46,7 +46,8 @@ extern "C" int tq_topk_noalloc(const tq_codebook_t* cb, const float* d_Pi, const
     if (v) return v == tq::kTopkNothing ? TQ_OK : v;
     const size_t need = tq_workspace_bytes(TQ_OP_TOPK, cb->d, cb->b, G, n, nq, k);
     // The materialised-score path when its scratch fits, else the fused path.
-    bool materialize = tq::topk_materialized(G, n, nq) && need <= (size_t)TQ_NOALLOC_SCRATCH_BYTES;
+    bool materialize =
+        tq::topk_materialized(cb->d, G, n, nq) && need <= (size_t)TQ_NOALLOC_SCRATCH_BYTES;
     if (!materialize && tq::topk_workspace_bytes(cb->d, cb->b, G, n, nq, k, false) >
                             (size_t)TQ_NOALLOC_SCRATCH_BYTES)
         return TQ_ERR_SCRATCH_LIMIT;

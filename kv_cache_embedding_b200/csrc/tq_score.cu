@@ -900,6 +900,11 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     float* u = (float*)((char*)qr + align256((size_t)G * nq * d * 4));
     rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, err, s);
     if (rc) return rc;
+    if (score_gemm_supported(d, nq)) {  // many queries at d >= 256: decoded-key GEMM
+        void* op = (char*)u + align256((size_t)G * nq * d * 4);
+        return score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr, 0,
+                          op, err, s);
+    }
     if (!is_mse(cb) && score_tc_supported(d, b, G, n, nq))
         return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
@@ -948,7 +953,12 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         p += align256((size_t)rows * kCandCapG * 4);
         int* ci = (int*)p;
         int nchunks;
-        if (tc) {  // maxima per 128-key tile
+        if (score_gemm_supported(d, nq)) {  // decoded-key GEMM, maxima per 128-key tile
+            p = (char*)ci + align256((size_t)rows * kCandCapG * 4);
+            TQ_TRY_CUDA(cudaMemsetAsync(cnt, 0, (size_t)rows * 2 * 4, s));
+            rc = score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, ntm, p, err, s);
+            nchunks = (int)ntm;
+        } else if (tc) {  // maxima per 128-key tile
             rc = launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt, err,
                                  s);
             nchunks = (int)ntm;
@@ -1021,7 +1031,7 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
                                  k, d_vals, d_ids);
     if (rc) return rc == kTopkNothing ? TQ_OK : rc;
     return topk_run(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
-                    d_ids, d_ws, ws_bytes, topk_materialized(G, n, nq), (cudaStream_t)stream);
+                    d_ids, d_ws, ws_bytes, topk_materialized(cb->d, G, n, nq), (cudaStream_t)stream);
 }
 
 extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,

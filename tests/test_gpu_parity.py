@@ -270,6 +270,35 @@ def test_exact_topk_many_tiles(tq_lib, cuda):
     PT.compare_topk(_np(vals[0]), _np(ids[0]), ex, k, np.ones(nq), 1.0)
 
 
+@pytest.mark.parametrize("d,b,G,n,nq,mse", [(256, 4, 2, 3000, 70, False), (384, 2, 1, 1025, 130, False),
+                                            (256, 3, 1, 2000, 64, True)])
+def test_score_and_topk_decoded_key_gemm(quant, quant_mse, oparams, tq_lib, cuda, d, b, G, n, nq,
+                                         mse):
+    """d >= 256 with 64+ queries per group: scores as a tensor-core GEMM over
+    decoded keys (transposed store, per-tile maxima for the top-k); ragged key
+    tiles, padded query tiles, several groups, both variants."""
+    k = 10
+    qs = synth.gaussian_rows(G * nq, d, seed=51, norm_range=None).reshape(G, nq, d)
+    W = b * d // 32
+    recs = [synth.random_records(n, W, seed=100 + g) for g in range(G)]
+    codes = tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+    tq = quant_mse(d, b, 0, G) if mse else quant(d, b, 0, G)
+    s_gpu = _np(tq.score(codes, qs.cuda()))
+    vals, ids = tq.topk(codes, qs.cuda(), k)
+    for g in range(G):
+        c, xn, rn = recs[g]
+        if mse:
+            s_ora = O.mse_score(O.MseParams(d, b, g), c, xn, _f64(qs[g]))
+        else:
+            s_ora = O.score(oparams(d, b, g), c, xn, rn, _f64(qs[g]))
+        qn = np.linalg.norm(_f64(qs[g]), axis=1)
+        PT.compare_scores(s_gpu[g], s_ora, qn, xn.astype(np.float64))
+        PT.compare_topk(_np(vals[g]), _np(ids[g]), s_ora, k, qn, float(xn.max()))
+
+
 @pytest.mark.parametrize("b", [1, 3, 4])
 def test_decode(quant, oparams, tq_lib, cuda, b):
     d = 128
