@@ -123,7 +123,10 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     if (need > 0 && (!d_ws || ws_bytes < need)) return TQ_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     // the first 256 bytes of the workspace hold the device status word
-    if (!mse && encode_tc_supported(d, x_dtype, G, n))  // d = 128 bf16 keys: fused tensor-core kernel
+    // d = 128 bf16 keys: fused tensor-core kernel (TMA source and 16-byte code
+    // stores need 16-byte aligned buffers)
+    if (!mse && encode_tc_supported(cb, x_dtype, G, n) && (uintptr_t)d_x % 16 == 0 &&
+        (uintptr_t)d_codes % 16 == 0)
         return launch_encode_tc(cb, d_Pi, d_S, G, n, d_x, d_codes, d_xnorm, d_rnorm,
                                 (int*)d_ws, s);
     TQ_TRY_CUDA(cudaMemsetAsync(d_ws, 0, sizeof(int), s));

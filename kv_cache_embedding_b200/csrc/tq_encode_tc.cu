@@ -8,25 +8,28 @@
 // matrix); seeallochnaya #3476 (round every coordinate on the fixed grid;
 // residual -> random matrix -> sign; "parallelises well on a GPU").
 //
-// Design (transposed orientation: output coordinates are the MMA's M = 128
-// rows, vectors its N = 64 columns):
-//  * The weights live in tensor memory as the MMA's A operand for the whole
-//    kernel: Pi as three bf16 pieces (Pi = p1 + p2 + p3 to ~2^-24) and S as
-//    two fp16 pieces (S = s1 + s2 to ~2^-22).  TMEM columns:
-//      [0,192) Pi pieces | [192,320) S pieces | [320,448) D1 x2 | [448,512) D2
-//  * A tile of 64 bf16 key vectors arrives by TMA (128-byte swizzle) and is
-//    the B operand as is: bf16 x bf16 products are exact, so the rotation
-//    D1 = Pi X^T is fp32-accurate after 3 passes.
-//  * Epilogue warps (thread = output coordinate, kVpw vectors per warp) work
-//    in units scaled by 2^10 (exact: 1/|x|, boundaries and centroids are
-//    pre-multiplied): y' = 2^10 y, bucketize, r' = y' - c'[idx], |r|^2, and r'
-//    as two fp16 pieces written coordinate-major (one 128-byte row per
-//    coordinate, vectors contiguous): the MN-major B operand of D2 = S R^T
-//    (3 passes: s1 h1 + s1 h2 + s2 h1).  Only the sign of D2 is kept.  The
-//    second half of a tile (signs, packing, stores) runs after the first half
-//    of the next tile so the QJL MMA overlaps epilogue work.
-//  * Warp roles: 0 TMA producer, 1 TMEM owner + MMA issuer, 2-3 norms,
-//    4.. epilogue (kEpi warps; kEpi / 4 per TMEM lane quarter).
+// Design (vector-major: a tile is 128 vectors = the MMA's M rows, the 128
+// output coordinates its N columns, so a TMEM lane holds one vector):
+//  * Keys are converted in shared memory from bf16 to fp16 after a power of
+//    two per vector, 2^e, brings |x| into [128, 256): every bf16 value is
+//    then an exact fp16 (8 significant bits of 11), so the rotation needs
+//    only the pieces of Pi: 2^8 Pi = p1 + p2 (fp16, to ~2^-22), 2 passes.
+//    The epilogue warps do this for tile k + 1 (4 threads per key, norm
+//    combined by shuffles) before they process tile k.
+//  * The weights are the MMA's B operand in shared memory (K-major, 128-byte
+//    swizzle): 2^8 Pi as p1, p2 and S as s1, s2 (fp16), 128 KB per group.
+//  * Epilogue thread = (vector, 32-coordinate block): y' = 2^10 y from D1,
+//    bucketize (a table over y'/32 gives the cell below and the one boundary
+//    that can fall inside each 32-wide interval), r' = y' - c'[idx], the block's part of |r'|^2, and r' as two
+//    fp16 pieces written to TMEM as the A operand of D2 = R S^T (3 passes:
+//    h1 s1 + h2 s1 + h1 s2).  Sign bits come back from D2 in the same
+//    thread, so the block's code words are packed in registers and stored
+//    whole: no cross-lane packing or reduction.  The second half of a tile
+//    (signs, packing, stores) runs after the first half of the next tile so
+//    the QJL MMA overlaps epilogue work.
+//  * TMEM columns: [0,256) D1 x2 | [256,384) R pieces | [384,512) D2.
+//  * Warp roles: 0 TMA producer, 1 TMEM owner + MMA issuer, 2-17 norms,
+//    fp16 conversion and epilogue (4 lane quarters x 4 blocks).
 //  * Every wait is bounded (1 s); a warp that gives up sets the abort flag and
 //    the device status word, all roles leave their loops, in-flight TMA loads
 //    and MMAs are drained (again bounded) and TMEM is released.
@@ -45,34 +48,45 @@ namespace {
 using namespace sm100;
 
 constexpr int kD = 128;
-constexpr int kTN = 64;                      // vectors per tile (MMA N)
-constexpr int kXS = 4;                       // key-tile stages
-constexpr int kVpw = 16;                     // vectors per epilogue warp
-constexpr int kNH = kTN / kVpw;              // epilogue warps per TMEM lane quarter
-constexpr int kEpi = 4 * kNH;                // epilogue warps
-constexpr int kThreads = 32 * (4 + kEpi);
-constexpr uint32_t kColPi = 0, kColS = 192, kColD1 = 320, kColD2 = 448, kTmemCols = 512;
-constexpr uint32_t kStageBytes = kTN * kD * 2;   // two 8 KB swizzled regions (k < 64, k >= 64)
-constexpr uint64_t kWaitNs = 1000000000ull;      // 1 s per wait
-constexpr float kRScale = 1024.f;                // r * 2^10 keeps fp16 pieces normal
-constexpr uint32_t kIdescRot = idesc_f16(1, 128, kTN);                // bf16 x bf16 -> f32
-constexpr uint32_t kIdescQjl = idesc_f16(0, 128, kTN) | (1u << 16);   // fp16 x fp16, B MN-major
+constexpr int kTN = 128;                     // vectors per tile (MMA M)
+constexpr int kXS = 2;                       // key-tile stages
+constexpr int kInv = 4;                      // slots of the per-vector scale ring
+constexpr int kEpi = 16;                     // epilogue warps: 4 lane quarters x 4 blocks
+constexpr int kThreads = 32 * (2 + kEpi);
+constexpr int kLut = 128;                    // bucketize table: y'/32 rounded, mod 128
+constexpr float kLutStep = 32.f;
+constexpr uint32_t kColD1 = 0, kColR = 256, kColD2 = 384, kTmemCols = 512;
+constexpr uint32_t kRegion = kTN * 128;      // 128 rows x 128 bytes: k < 64 or k >= 64
+constexpr uint32_t kTileBytes = 2 * kRegion; // one 128 x 128 16-bit operand
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
+constexpr float kRScale = 1024.f;            // r * 2^10 keeps fp16 pieces normal
+constexpr float kPiScale = 256.f;            // 2^8 Pi keeps the second piece normal
+constexpr uint32_t kIdescF16 = idesc_f16(0, 128, 128);  // fp16 x fp16 -> f32, K-major
 
 struct Smem {
-    uint8_t x[kXS][kStageBytes];   // 1024-aligned (first member)
-    uint8_t r[2][2][kStageBytes];  // [tile parity][piece h1, h2]: B operand of the QJL MMA
-    float inv[kXS][kTN];           // 2^10 / |x| per stage
-    float rr[2][4][kTN];           // [tile parity][lane quarter] |r'|^2 partial sums
+    uint8_t x[kXS][kTileBytes];    // keys: bf16 from TMA, then fp16 in place (1024-aligned)
+    uint8_t wpi[2][kTileBytes];    // 2^8 Pi pieces p1, p2
+    uint8_t ws[2][kTileBytes];     // S pieces s1, s2
+    float4 lut[kLut][8];           // (boundary, c'[cell], c'[cell + 1], cell), 8 copies
+    float inv[kInv][kTN];          // 2^10 / (|x| 2^e 2^8) per vector
+    float rr[2][4][kTN];           // [tile parity][block] |r'|^2 partial sums
     float c[8];                    // 2^10 c
     float beta[8];                 // 2^10 beta
-    uint64_t full_x[kXS], empty_x[kXS], norm_full[kXS];
-    uint64_t d1_full[2], d1_empty[2], r_full, d2_full, d2_empty, w_ready, epi_bar, mma_done;
+    uint64_t full_x[kXS], xready[kXS], empty_x[kXS];
+    uint64_t d1_full[2], d1_empty[2], r_full, d2_full, d2_empty, w_ready, mma_done;
     uint32_t tmem_base;
     int abort;
     int zero;
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+// Byte offset of 16-bit element (row, k) in a K-major 128 x 128 operand with
+// the 128-byte swizzle (the layout TMA writes for a {64, 128} box).
+__device__ __forceinline__ uint32_t sw128_offset(int row, int k) {
+    return (uint32_t)(k >> 6) * kRegion + (uint32_t)row * 128u +
+           ((((uint32_t)(k >> 3) & 7u) ^ ((uint32_t)row & 7u)) << 4) + (uint32_t)(k & 7) * 2u;
+}
 
 // Tiles of this CTA: groups are spread over CTAs (cpg CTAs per group when
 // G <= #CTAs, else whole groups round-robin).  f(g, t, first, last) -> bool.
@@ -105,206 +119,95 @@ __device__ __forceinline__ bool give_up(volatile int* abort, int* err, int site)
     return false;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
-    return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-}
-__device__ __forceinline__ uint32_t pack_f16(__half lo, __half hi) {
-    return (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// 32 lanes x 32 bits, 16 consecutive columns: thread t of the warp gets lane
-// (warp's quarter base + t), columns [taddr.col, +16).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-template <int V>
-__device__ __forceinline__ void tmem_ldv(uint32_t taddr, uint32_t (&r)[V]) {
-    if constexpr (V == 16) tmem_ld16(taddr, r);
-    else tmem_ld32(taddr, r);
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-        : "memory");
-}
-
-// Copy the d x d fp32 matrix M (row-major) transposed into shared memory,
-// stage[k][m] = M[m][k], by the epilogue warps (te = 0 .. 32 kEpi - 1): lane
-// = row m within a quarter, so the shared stores of a warp are contiguous;
-// each thread keeps its 8 row loads in flight together.
-__device__ __forceinline__ void stage_transposed(const float* __restrict__ M, float* stage, int te) {
-    const int m = 32 * ((te >> 5) & 3) + (te & 31);
-    const int kg = te >> 7;  // 0..3: which quarter of the 32 float4 of the row
-    float4 v[8];
+// Weights of one group into shared memory as fp16 pieces, by the 512
+// epilogue threads (te): M (d x d fp32, row-major: B operand row n = output
+// coordinate, k = input coordinate) times `scale` = hi + lo.  A thread
+// converts 16-byte chunks (8 k of one row) and keeps its loads in flight.
+__device__ __forceinline__ void weights_to_smem(const float* __restrict__ M, float scale,
+                                                uint8_t* hi, uint8_t* lo, int te) {
+    constexpr int kChunks = kD * kD / 8 / (32 * kEpi);  // 4
+    float4 v[kChunks][2];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        v[j] = __ldg(reinterpret_cast<const float4*>(M + (size_t)m * kD) + 8 * kg + j);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int k = 4 * (8 * kg + j);
-        stage[(k + 0) * kD + m] = v[j].x;
-        stage[(k + 1) * kD + m] = v[j].y;
-        stage[(k + 2) * kD + m] = v[j].z;
-        stage[(k + 3) * kD + m] = v[j].w;
+    for (int u = 0; u < kChunks; ++u) {
+        const int c = te + 32 * kEpi * u;  // row c >> 4, k = 8 (c & 15) ..
+        const float4* src = reinterpret_cast<const float4*>(M + (size_t)(c >> 4) * kD) + 2 * (c & 15);
+        v[u][0] = __ldg(src);
+        v[u][1] = __ldg(src + 1);
     }
-}
-
-// Pieces of row `row` of the staged matrix (stage[k][row]) into TMEM lane
-// `row`: Pi as bf16 pieces 0-2 (bits 0-2 of `mask`), S as fp16 pieces 0-1
-// (bit 3).  Column c of a piece holds k = 2c (low half) and k = 2c + 1 (high
-// half); written 8 columns at a time.
-__device__ void pieces_to_tmem(const float* stage, bool is_pi, int row, int mask,
-                               uint32_t taddr_lane) {
-#pragma unroll 1
-    for (int piece = 0; piece < 3; ++piece) {
-        if (is_pi ? !(mask & (1 << piece)) : (piece == 2 || !(mask & 8))) continue;
-        const uint32_t col0 = is_pi ? kColPi + 64u * piece : kColS + 64u * piece;
-#pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 8) {
-            uint32_t w[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float vx = stage[(2 * (c0 + c)) * kD + row];
-                const float vy = stage[(2 * (c0 + c) + 1) * kD + row];
-                if (is_pi) {  // Pi = p1 + p2 + p3 (bf16)
-                    __nv_bfloat16 a = __float2bfloat16_rn(vx), bb = __float2bfloat16_rn(vy);
-                    float ra = vx - __bfloat162float(a), rb = vy - __bfloat162float(bb);
-                    if (piece >= 1) {
-                        a = __float2bfloat16_rn(ra);
-                        bb = __float2bfloat16_rn(rb);
-                        ra -= __bfloat162float(a);
-                        rb -= __bfloat162float(bb);
-                    }
-                    if (piece == 2) {
-                        a = __float2bfloat16_rn(ra);
-                        bb = __float2bfloat16_rn(rb);
-                    }
-                    w[c] = pack_bf16(a, bb);
-                } else {  // S = s1 + s2 (fp16)
-                    __half a = __float2half_rn(vx), bb = __float2half_rn(vy);
-                    if (piece == 1) {
-                        a = __float2half_rn(vx - __half2float(a));
-                        bb = __float2half_rn(vy - __half2float(bb));
-                    }
-                    w[c] = pack_f16(a, bb);
-                }
-            }
-            tmem_st8(taddr_lane + col0 + (uint32_t)c0, w);
+    for (int u = 0; u < kChunks; ++u) {
+        const int c = te + 32 * kEpi * u;
+        const float e[8] = {v[u][0].x, v[u][0].y, v[u][0].z, v[u][0].w,
+                            v[u][1].x, v[u][1].y, v[u][1].z, v[u][1].w};
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float a = e[2 * p] * scale, b = e[2 * p + 1] * scale;
+            const __half2 h = __floats2half2_rn(a, b);
+            const float2 hf = __half22float2(h);
+            wh[p] = h2_bits(h);
+            wl[p] = h2_bits(__floats2half2_rn(a - hf.x, b - hf.y));
         }
+        const uint32_t off = sw128_offset(c >> 4, 8 * (c & 15));
+        *reinterpret_cast<uint4*>(hi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(lo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
     }
 }
 
-// One halving round of a transposed butterfly: lane keeps half of its n
-// values (selected by `up`), sends the other half to lane ^ m and combines.
-template <int N, class Op, class T>
-__device__ __forceinline__ void halve(T (&v)[N], bool up, int m, Op op) {
+// Code words of one 32-coordinate block (layout of tq.h): the cell fields
+// packed during bucketize and z = [p >= 0] for the QJL projections p.  Every
+// z starts set and a negative p clears its bit (p + 0 turns -0 into +0, so the
+// sign of the sum is exactly p < 0); the words are stored whole at dst.
+template <int B>
+__device__ __forceinline__ void store_block(const uint32_t (&cellw)[4], const uint32_t (&p)[32],
+                                            uint32_t* __restrict__ dst) {
+    constexpr uint32_t kZ = (B == 4) ? 0x88888888u : ((B == 2) ? 0xAAAAAAAAu : 0u);
+    uint32_t w[4] = {cellw[0] | kZ, cellw[1] | kZ, cellw[2] | kZ, cellw[3] | kZ};
+    uint32_t sw = 0xFFFFFFFFu;
 #pragma unroll
-    for (int i = 0; i < N / 2; ++i) {
-        const T lo = v[2 * i], hi = v[2 * i + 1];
-        v[i] = op(up ? hi : lo, __shfl_xor_sync(0xffffffffu, up ? lo : hi, m));
+    for (int j = 0; j < 32; ++j) {
+        const uint32_t neg = __float_as_uint(__uint_as_float(p[j]) + 0.f) >> 31;
+        if (B == 4) w[j >> 3] -= neg << (4 * (j & 7) + 3);
+        if (B == 2) w[j >> 4] -= neg << (2 * (j & 15) + 1);
+        if (B == 1 || B == 3) sw -= neg << j;
     }
+    if (B == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (B == 3) {
+        dst[0] = w[0];
+        dst[1] = w[1];
+        dst[2] = sw;
+    }
+    if (B == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    if (B == 1) dst[0] = sw;
 }
 
-// Sum over the 32 lanes of v[j], for every j < V (V = 16 or 32).  Rounds pair
-// lanes by bits 0.. of the lane index against bits 0.. of j; lane l ends with
-// the sum for j = l % V (lanes l and l + 16 agree when V = 16).
-template <int V>
-__device__ __forceinline__ float transpose_reduce(const float (&v)[V], int lane) {
-    float cur[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) cur[i] = v[i];
-    auto add = [](float a, float b) { return a + b; };
-    halve<V>(cur, lane & 1, 1, add);
-    halve<V / 2>(reinterpret_cast<float(&)[V / 2]>(cur), lane & 2, 2, add);
-    halve<V / 4>(reinterpret_cast<float(&)[V / 4]>(cur), lane & 4, 4, add);
-    halve<V / 8>(reinterpret_cast<float(&)[V / 8]>(cur), lane & 8, 8, add);
-    float t;
-    if constexpr (V == 32) {
-        halve<2>(reinterpret_cast<float(&)[2]>(cur), lane & 16, 16, add);
-        t = cur[0];
+// Number of tiles of this CTA, and its k-th tile, in the order of for_each_tile.
+__device__ __forceinline__ int tile_count(int G, int tpg) {
+    const int cta = blockIdx.x, nctas = gridDim.x;
+    if (G <= nctas) {
+        const int cpg = nctas / G;
+        if (cta >= cpg * G) return 0;
+        const int slot = cta % cpg;
+        return slot < tpg ? (tpg - slot + cpg - 1) / cpg : 0;
+    }
+    return cta < G ? ((G - cta + nctas - 1) / nctas) * tpg : 0;
+}
+
+__device__ __forceinline__ void tile_at(int k, int G, int tpg, int& g, int& t, bool& first) {
+    const int cta = blockIdx.x, nctas = gridDim.x;
+    if (G <= nctas) {
+        const int cpg = nctas / G;
+        g = cta / cpg;
+        t = cta % cpg + k * cpg;
+        first = k == 0;
     } else {
-        t = cur[0] + __shfl_xor_sync(0xffffffffu, cur[0], 16);
-    }
-    return t;
-}
-
-// OR-combine fields of F lanes (F = 8 or 16, already shifted into place) for
-// V vectors: afterwards lane e (= lane % F) holds the finished words of
-// vectors j = e + F*i, i < V/F.
-template <int F, int V>
-__device__ __forceinline__ void transpose_or(const uint32_t (&v)[V], int lane,
-                                             uint32_t (&out)[V / F]) {
-    uint32_t cur[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) cur[i] = v[i];
-    auto orr = [](uint32_t a, uint32_t b) { return a | b; };
-    halve<V>(cur, lane & 1, 1, orr);
-    halve<V / 2>(reinterpret_cast<uint32_t(&)[V / 2]>(cur), lane & 2, 2, orr);
-    halve<V / 4>(reinterpret_cast<uint32_t(&)[V / 4]>(cur), lane & 4, 4, orr);
-    if constexpr (F == 16) halve<V / 8>(reinterpret_cast<uint32_t(&)[V / 8]>(cur), lane & 8, 8, orr);
-#pragma unroll
-    for (int i = 0; i < V / F; ++i) out[i] = cur[i];
-}
-
-// Pack the fields of this lane's coordinate (block q, position `lane`) for
-// the warp's V vectors (rows V*h .. V*h + V - 1 of the tile) and store the
-// finished words of block q straight to the tile's records `dst` (W words per
-// record); rows at or beyond `valid` are not written.
-template <int B, int V>
-__device__ __forceinline__ void pack_store(const uint32_t (&cellw)[V / 8],
-                                           const uint32_t (&pbits)[V], int lane, int q, int h,
-                                           uint32_t* __restrict__ dst, int valid) {
-    constexpr int W = B * kD / 32;
-    uint32_t z[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) z[j] = (__uint_as_float(pbits[j]) >= 0.f) ? 1u : 0u;
-    if (B == 1 || B == 3) {
-        uint32_t mine = 0;
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint32_t w = __ballot_sync(0xffffffffu, z[j] != 0u);
-            if (lane == j) mine = w;
-        }
-        if (lane < V && V * h + lane < valid)
-            dst[(V * h + lane) * W + B * q + (B == 1 ? 0 : 2)] = mine;
-    }
-    if (B == 4) {
-        uint32_t v[V], out[V / 8];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint32_t cell = (cellw[j >> 3] >> (4 * (j & 7))) & 15u;
-            v[j] = (cell | (z[j] << 3)) << (4 * (lane & 7));
-        }
-        transpose_or<8, V>(v, lane, out);
-#pragma unroll
-        for (int i = 0; i < V / 8; ++i) {
-            const int row = V * h + (lane & 7) + 8 * i;
-            if (row < valid) dst[row * W + 4 * q + (lane >> 3)] = out[i];
-        }
-    }
-    if (B == 2 || B == 3) {
-        uint32_t v[V], out[V / 16];
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-            const uint32_t cell = (cellw[j >> 3] >> (4 * (j & 7))) & 15u;
-            const uint32_t f = (B == 2) ? (cell | (z[j] << 1)) : cell;
-            v[j] = f << (2 * (lane & 15));
-        }
-        transpose_or<16, V>(v, lane, out);
-#pragma unroll
-        for (int i = 0; i < V / 16; ++i) {
-            const int row = V * h + (lane & 15) + 16 * i;
-            if (row < valid) dst[row * W + B * q + (lane >> 4)] = out[i];
-        }
+        g = cta + (k / tpg) * nctas;
+        t = k % tpg;
+        first = t == 0;
     }
 }
 
@@ -316,7 +219,6 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             int* __restrict__ err) {
     constexpr int L = (B == 1) ? 1 : (1 << (B - 1));
     constexpr int W = B * kD / 32;
-    constexpr int V = kVpw;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment by pointer arithmetic on the shared array itself, so
     // every access below stays a shared-memory (not generic) access
@@ -328,8 +230,8 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
     if (threadIdx.x == 0) {
         for (int s = 0; s < kXS; ++s) {
             mbar_init(&sm.full_x[s], 1);
-            mbar_init(&sm.empty_x[s], 1 + 2 + kEpi);  // MMA commit + norm warps + epilogue
-            mbar_init(&sm.norm_full[s], 2);
+            mbar_init(&sm.xready[s], kEpi);  // converted by every epilogue warp
+            mbar_init(&sm.empty_x[s], 1);    // MMA commit
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.d1_full[b], 1);
@@ -339,7 +241,6 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
         mbar_init(&sm.d2_full, 1);
         mbar_init(&sm.d2_empty, kEpi);
         mbar_init(&sm.w_ready, kEpi);
-        mbar_init(&sm.epi_bar, kEpi);
         mbar_init(&sm.mma_done, 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // static indices: the codebook stays out of local memory
@@ -359,6 +260,28 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
+    if (B >= 3) {
+        // Bucketize table over i = round(y'/32) + 64 (mod 128): y' in
+        // [(i - 64.5) 32, (i - 63.5) 32] has `below` boundaries under the
+        // interval and at most one inside it (the host checks that the
+        // boundaries are more than 32 apart).  Entry: (that boundary or
+        // +huge, c'[below], c'[below + 1], below).
+        for (int e = threadIdx.x; e < kLut * 8; e += blockDim.x) {
+            const int li = e >> 3;
+            const float lo = ((float)li - 64.5f) * kLutStep, hi = ((float)li - 63.5f) * kLutStep;
+            int below = 0;
+            float bstar = 3.0e38f;
+            for (int k = 0; k + 1 < L; ++k) {
+                const float bk = sm.beta[k];
+                if (bk < lo) ++below;
+                else if (bk <= hi && bstar == 3.0e38f) bstar = bk;
+            }
+            const int above = below + 1 < L ? below + 1 : below;
+            sm.lut[li][e & 7] = make_float4(bstar, sm.c[below], sm.c[above],
+                                            __uint_as_float((uint32_t)below));
+        }
+        __syncthreads();
+    }
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer ----------------
@@ -368,10 +291,10 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             if (i >= (uint32_t)kXS &&
                 !mbar_wait(&sm.empty_x[s], ((i / kXS) - 1) & 1, abort, kWaitNs))
                 return give_up(abort, err, 1);
-            mbar_arrive_expect_tx(&sm.full_x[s], kStageBytes);
+            mbar_arrive_expect_tx(&sm.full_x[s], kTileBytes);
             const int32_t row = (int32_t)((int64_t)g * n + (int64_t)t * kTN);
             tma_load_2d(sm.x[s], &tmap_x, 0, row, &sm.full_x[s]);
-            tma_load_2d(sm.x[s] + kStageBytes / 2, &tmap_x, 64, row, &sm.full_x[s]);
+            tma_load_2d(sm.x[s] + kRegion, &tmap_x, 64, row, &sm.full_x[s]);
             ++i;
             return true;
         });
@@ -386,16 +309,15 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
             if (j >= 1 && !mbar_wait(&sm.d2_empty, (j - 1) & 1, abort, kWaitNs))
                 return give_up(abort, err, 12);
             tc_fence_after();
-            const uint32_t d = tbase + kColD2;
-            const uint32_t rb0 = smem_u32(sm.r[j & 1][0]), rb1 = smem_u32(sm.r[j & 1][1]);
 #pragma unroll
-            for (int combo = 0; combo < 3; ++combo) {  // s1 h1, s1 h2, s2 h1
-                const uint32_t a = tbase + kColS + (combo == 2 ? 64u : 0u);
-                const uint32_t rb = (combo == 1) ? rb1 : rb0;
+            for (int combo = 0; combo < 3; ++combo) {  // h1 s1, h2 s1, h1 s2
+                const uint32_t a = tbase + kColR + (combo == 1 ? 64u : 0u);
+                const uint32_t wb = smem_u32(sm.ws[combo == 2 ? 1 : 0]);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)  // 16 coordinates = 16 rows of 128 B per step
-                    mma_f16_ts(d, a + ks * 8, smem_desc_mnmajor_sw128(rb + ks * 2048),
-                               kIdescQjl, (combo | ks) != 0);
+                for (int ks = 0; ks < 8; ++ks)  // 16 coordinates per step
+                    mma_f16_ts(tbase + kColD2, a + ks * 8,
+                               smem_desc_kmajor_sw128(wb + (ks >> 2) * kRegion + (ks & 3) * 32),
+                               kIdescF16, (combo | ks) != 0);
             }
             tc_commit(&sm.d2_full);
             return true;
@@ -407,21 +329,22 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
                 tc_fence_after();
             }
             const int s = i % kXS, b = i & 1;
-            if (!mbar_wait(&sm.full_x[s], (i / kXS) & 1, abort, kWaitNs))
+            if (!mbar_wait(&sm.xready[s], (i / kXS) & 1, abort, kWaitNs))
                 return give_up(abort, err, 4);
             if (i >= 2 && !mbar_wait(&sm.d1_empty[b], ((i >> 1) - 1) & 1, abort, kWaitNs))
                 return give_up(abort, err, 5);
             tc_fence_after();
-            const uint32_t d = tbase + kColD1 + 64u * b;
             const uint32_t xs = smem_u32(sm.x[s]);
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t wb = smem_u32(sm.wpi[p]);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_f16_ts(d, tbase + kColPi + 64u * p + ks * 8,
-                               smem_desc_kmajor_sw128(xs + (ks >> 2) * (kStageBytes / 2) +
-                                                      (ks & 3) * 32),
-                               kIdescRot, (p | ks) != 0);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ko = (ks >> 2) * kRegion + (ks & 3) * 32;
+                    mma_f16_ss(tbase + kColD1 + 128u * b, smem_desc_kmajor_sw128(xs + ko),
+                               smem_desc_kmajor_sw128(wb + ko), kIdescF16, (p | ks) != 0);
+                }
+            }
             tc_commit(&sm.empty_x[s]);
             tc_commit(&sm.d1_full[b]);
             if (!first && !qjl(i - 1)) return false;
@@ -432,203 +355,225 @@ k_encode_tc(const __grid_constant__ CUtensorMap tmap_x, const float* __restrict_
         // every issued MMA completes before TMEM is released
         tc_commit(&sm.mma_done);
         mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
-    } else if (warp == 2 || warp == 3) {
-        // ---------------- norms (two warps, 32 vectors each) ----------------
-        uint32_t i = 0;
-        const int nr = lane + 32 * (warp - 2);
-        for_each_tile(G, tpg, [&](int g, int t, bool, bool) {
-            const int s = i % kXS;
-            if (!warp_wait(&sm.full_x[s], (i / kXS) & 1, abort)) return give_up(abort, err, 6);
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    } else if (warp >= 2) {
+        // ---------------- norms, fp16 conversion and epilogue ----------------
+        const int ew = warp - 2;                       // 0 .. kEpi - 1
+        const int q = warp & 3, h = ew >> 2;           // lane quarter, 32-coordinate block
+        const int m = q * 32 + lane;                   // vector within the tile
+        const uint32_t lane_addr = tbase + ((uint32_t)(q * 32) << 16);
+        const int te = threadIdx.x - 64;               // 0 .. 32*kEpi - 1
+        const int cr = 8 * ew + (lane & 7), cj = lane >> 3;  // conversion: key row, quarter
+        const float4* lut = &sm.lut[0][lane & 7];
+        const float bt0 = sm.beta[0], c0 = sm.c[0], c1 = sm.c[1];
+        const int ntile = tile_count(G, tpg);
+
+        // Norm of key row cr of tile k (4 threads, 32 bf16 each), its power of
+        // two 2^e, and the row converted in place to fp16 x 2^e.
+        auto convert = [&](int k) -> bool {
+            int g, t;
+            bool first;
+            tile_at(k, G, tpg, g, t, first);
+            const int s = k % kXS;
+            if (!warp_wait(&sm.full_x[s], (k / kXS) & 1, abort)) return give_up(abort, err, 6);
+            uint8_t* rowp = sm.x[s] + cr * 128;
+            uint32_t off[4];
+            uint4 u[4];
 #pragma unroll
-            for (int reg = 0; reg < 2; ++reg) {
-                const uint4* rowp =
-                    reinterpret_cast<const uint4*>(sm.x[s] + reg * (kStageBytes / 2) + nr * 128);
+            for (int kk = 0; kk < 4; ++kk) {
+                const int c = cj + 4 * kk;  // 16-byte chunk: k = 8c .. 8c + 7
+                off[kk] = (uint32_t)(c >> 3) * kRegion + ((((uint32_t)c & 7u) ^ ((uint32_t)cr & 7u)) << 4);
+                u[kk] = *reinterpret_cast<const uint4*>(rowp + off[kk]);
+            }
+            float a2[2] = {0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 v = rowp[c];
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t w4[4] = {u[kk].x, u[kk].y, u[kk].z, u[kk].w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float lo = __uint_as_float(w4[e] << 16);
-                        const float hi = __uint_as_float(w4[e] & 0xffff0000u);
-                        a4[e] = fmaf(lo, lo, a4[e]);
-                        a4[e] = fmaf(hi, hi, a4[e]);
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = __uint_as_float(w4[e] << 16);
+                    const float hi = __uint_as_float(w4[e] & 0xffff0000u);
+                    a2[e & 1] = fmaf(lo, lo, a2[e & 1]);
+                    a2[e & 1] = fmaf(hi, hi, a2[e & 1]);
                 }
             }
-            const float nx = sqrtf((a4[0] + a4[1]) + (a4[2] + a4[3]));
-            sm.inv[s][nr] = (nx > 0.f) ? kRScale / nx : 0.f;
-            const int64_t v = (int64_t)t * kTN + nr;
-            if (v < n) xnorm[(int64_t)g * n + v] = nx;
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&sm.norm_full[s]);
-                mbar_arrive(&sm.empty_x[s]);
+            float sum = a2[0] + a2[1];
+            sum += __shfl_xor_sync(0xffffffffu, sum, 8);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+            float nx = sqrtf(sum);
+            const bool odd = !(sum >= 0x1p-96f && sum <= 0x1p+126f);
+            if (__any_sync(0xffffffffu, odd)) {
+                // squares under- or overflow fp32 (or a zero row): fp64 sums
+                double acc = 0.0;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t w4[4] = {u[kk].x, u[kk].y, u[kk].z, u[kk].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const double lo = (double)__uint_as_float(w4[e] << 16);
+                        const double hi = (double)__uint_as_float(w4[e] & 0xffff0000u);
+                        acc = fma(lo, lo, acc);
+                        acc = fma(hi, hi, acc);
+                    }
+                }
+                acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+                if (odd) nx = (float)sqrt(acc);
             }
-            ++i;
-            return true;
-        });
-    } else if (warp >= 4) {
-        // ---------------- epilogue ----------------
-        const int q = warp & 3, h = (warp - 4) >> 2;  // lane quarter, vector slice
-        const int coord = q * 32 + lane;
-        const uint32_t lane_addr = tbase + ((uint32_t)(q * 32) << 16);
-        // residual row of this coordinate: 128 bytes, 16-byte chunk c (vectors
-        // 8c..8c+7) at position c ^ (coord % 8); this warp writes chunks
-        // (V/8) h .. (V/8) h + V/8 - 1
-        uint32_t roff[V / 8];
+            // 2^e with |x| 2^e in [128, 256) (clamped for extreme norms)
+            const int eb = (int)((__float_as_uint(nx) >> 23) & 0xffu);
+            int ex = (eb == 0) ? 126 : 134 - eb;
+            ex = ex < -120 ? -120 : (ex > 126 ? 126 : ex);
+            const float sc = __uint_as_float((uint32_t)(ex + 127) << 23);
 #pragma unroll
-        for (int ii = 0; ii < V / 8; ++ii)
-            roff[ii] = (uint32_t)coord * 128u +
-                       ((((uint32_t)(V / 8 * h + ii)) ^ (uint32_t)(coord & 7)) << 4);
-        float bt[7];
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t w4[4] = {u[kk].x, u[kk].y, u[kk].z, u[kk].w};
+                uint32_t o[4];
 #pragma unroll
-        for (int k = 0; k < 7; ++k) bt[k] = sm.beta[k];
-        // weight pieces this warp loads into TMEM at each group start
-        const int wmask = (kNH == 4) ? (1 << h) : (h == 0 ? 7 : 8);
-        uint32_t i = 0, eb = 0;
-        const int te = threadIdx.x - 128;  // 0 .. 32*kEpi - 1 over the epilogue warps
-        auto epi_sync = [&]() -> bool {  // all epilogue warps
+                for (int e = 0; e < 4; ++e)
+                    o[e] = h2_bits(__floats2half2_rn(__uint_as_float(w4[e] << 16) * sc,
+                                                     __uint_as_float(w4[e] & 0xffff0000u) * sc));
+                *reinterpret_cast<uint4*>(rowp + off[kk]) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+            if (cj == 0) {
+                sm.inv[k % kInv][cr] = (nx > 0.f) ? (kRScale / kPiScale) / (nx * sc) : 0.f;
+                const int64_t v = (int64_t)t * kTN + cr;
+                if (v < n) xnorm[(int64_t)g * n + v] = nx;
+            }
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.epi_bar);
-            const bool ok = warp_wait(&sm.epi_bar, eb & 1, abort);
-            ++eb;
-            return ok;
+            if (lane == 0) mbar_arrive(&sm.xready[s]);
+            return true;
         };
-        float* stage = reinterpret_cast<float*>(&sm.r[0][0][0]);  // 64 KB, free at group start
+
         // The second half of a tile (sign bits, packing, stores) runs after the
         // first half of the next tile.  State of the pending tile:
         bool pend = false;
         int pg = 0, pt = 0;
         uint32_t pidx = 0;
-        uint32_t pcell[V / 8];
-#pragma unroll
-        for (int u = 0; u < V / 8; ++u) pcell[u] = 0u;
-        auto finish = [&]() -> bool {
+        uint32_t pcell[4] = {0u, 0u, 0u, 0u};
+        auto wait_d2 = [&]() -> bool {  // the QJL MMA of the pending tile is done
             if (!warp_wait(&sm.d2_full, pidx & 1, abort)) return give_up(abort, err, 9);
             tc_fence_after();
-            uint32_t pb[V];
-            tmem_ldv<V>(lane_addr + kColD2 + (uint32_t)(V * h), pb);
+            return true;
+        };
+        auto finish = [&]() {
+            uint32_t p[32];
+            tmem_ld32(lane_addr + kColD2 + 32u * h, p);
             tmem_wait_ld();
-            const int64_t v0 = (int64_t)pt * kTN;
-            const int valid = (int)((n - v0) < kTN ? (n - v0) : kTN);
-            // |r|^2 of the tile is complete: every epilogue warp stored its part
+            // |r'|^2 of the tile is complete: every epilogue warp stored its part
             // before arriving on r_full, which the QJL MMA behind d2_full waited for
-            if (q == 0 && lane < V && V * h + lane < valid) {
+            float rn = 0.f;
+            if (h == 0) {
                 const float (*rrb)[kTN] = sm.rr[pidx & 1];
-                const int vv = V * h + lane;
-                rnorm[(int64_t)pg * n + v0 + vv] =
-                    sqrtf(rrb[0][vv] + rrb[1][vv] + rrb[2][vv] + rrb[3][vv]) * (1.f / kRScale);
+                rn = sqrtf((rrb[0][m] + rrb[1][m]) + (rrb[2][m] + rrb[3][m])) * (1.f / kRScale);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.d2_empty);
-            pack_store<B, V>(pcell, pb, lane, q, h, codes + ((int64_t)pg * n + v0) * W, valid);
+            const int64_t v = (int64_t)pt * kTN + m;
+            if (v < n) {
+                const int64_t rec = (int64_t)pg * n + v;
+                if (h == 0) rnorm[rec] = rn;
+                store_block<B>(pcell, p, codes + rec * W + B * h);
+            }
             pend = false;
-            return true;
         };
-        bool running = true;
-        for_each_tile(G, tpg, [&](int g, int t, bool first, bool) {
+        bool running = ntile == 0 || convert(0);
+        for (int k = 0; running && k < ntile; ++k) {
+            int g, t;
+            bool first;
+            tile_at(k, G, tpg, g, t, first);
+            if (k + 1 < ntile && !convert(k + 1)) {
+                running = false;
+                break;
+            }
             if (first) {
-                // every MMA of the previous group must be done before its weights go
-                if (pend && !finish()) return running = false;
-                // Pi, then S, staged transposed through shared memory
-                for (int mat = 0; mat < 2; ++mat) {
-                    if (!epi_sync()) return running = give_up(abort, err, 13);
-                    stage_transposed((mat == 0 ? Pi : S) + (size_t)g * kD * kD, stage, te);
-                    if (!epi_sync()) return running = give_up(abort, err, 14);
-                    pieces_to_tmem(stage, mat == 0, coord, wmask, lane_addr);
+                // every MMA of the previous group is done once its last QJL MMA is
+                if (pend) {
+                    if (!wait_d2()) {
+                        running = false;
+                        break;
+                    }
+                    finish();
                 }
-                if (!epi_sync()) return running = give_up(abort, err, 15);
-                tmem_wait_st();
-                tc_fence_before();
+                weights_to_smem(Pi + (size_t)g * kD * kD, kPiScale, sm.wpi[0], sm.wpi[1], te);
+                weights_to_smem(S + (size_t)g * kD * kD, 1.f, sm.ws[0], sm.ws[1], te);
+                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.w_ready);
             }
-            const int s = i % kXS, b = i & 1;
-            if (!warp_wait(&sm.d1_full[b], (i >> 1) & 1, abort))
-                return running = give_up(abort, err, 7);
+            const int b = k & 1, s = k % kXS;
+            if (!warp_wait(&sm.d1_full[b], (k >> 1) & 1, abort)) {
+                running = give_up(abort, err, 7);
+                break;
+            }
             tc_fence_after();
-            uint32_t acc[V];
-            tmem_ldv<V>(lane_addr + kColD1 + 64u * b + (uint32_t)(V * h), acc);
+            uint32_t acc[32];
+            tmem_ld32(lane_addr + kColD1 + 128u * b + 32u * h, acc);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.d1_empty[b]);
-            if (!warp_wait(&sm.norm_full[s], (i / kXS) & 1, abort))
-                return running = give_up(abort, err, 8);
-            float inv[V];
-#pragma unroll
-            for (int j = 0; j < V; j += 4) {
-                const float4 t4 = *reinterpret_cast<const float4*>(&sm.inv[s][V * h + j]);
-                inv[j] = t4.x;
-                inv[j + 1] = t4.y;
-                inv[j + 2] = t4.z;
-                inv[j + 3] = t4.w;
+            // the scale of tile k was written before every warp arrived on xready
+            if (!warp_wait(&sm.xready[s], (k / kXS) & 1, abort)) {
+                running = give_up(abort, err, 8);
+                break;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty_x[s]);
+            const float inv = sm.inv[k % kInv][m];
 
-            uint32_t ccur[V / 8];
+            uint32_t cellw[4] = {0u, 0u, 0u, 0u};
+            float rr = 0.f;
+            uint32_t hp1[16], hp2[16];
 #pragma unroll
-            for (int u = 0; u < V / 8; ++u) ccur[u] = 0u;
-            float rr[V];
-            uint32_t hp1[V / 2], hp2[V / 2];
-#pragma unroll
-            for (int j = 0; j < V; j += 2) {
+            for (int j = 0; j < 32; j += 2) {
                 float sr[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float y = __uint_as_float(acc[j + e]) * inv[j + e];  // 2^10 y
-                    uint32_t cc = 0;
+                    const float y = __uint_as_float(acc[j + e]) * inv;  // 2^10 y
                     float r = y;
-                    if (B == 4) {  // three compares down the boundary tree
-                        const bool p2 = y >= bt[3];
-                        const bool p1 = y >= (p2 ? bt[5] : bt[1]);
-                        const bool p0 = y >= (p2 ? (p1 ? bt[6] : bt[4]) : (p1 ? bt[2] : bt[0]));
-                        cc = (p2 ? 4u : 0u) + (p1 ? 2u : 0u) + (p0 ? 1u : 0u);
-                    } else if (B > 1) {
-#pragma unroll
-                        for (int k = 0; k + 1 < L; ++k) cc += (y >= bt[k]) ? 1u : 0u;
+                    if (B >= 3) {
+                        const float tf = fmaf(y, 1.f / kLutStep, 12582912.f + 64.f);
+                        const float4 en = lut[(__float_as_uint(tf) & (kLut - 1)) * 8];
+                        const bool up = y >= en.x;
+                        r = y - (up ? en.z : en.y);
+                        const uint32_t cc = __float_as_uint(en.w) + (up ? 1u : 0u);
+                        if (B == 4) cellw[(j + e) >> 3] += cc << (4 * ((j + e) & 7));
+                        else cellw[(j + e) >> 4] += cc << (2 * ((j + e) & 15));
+                    } else if (B == 2) {
+                        const bool up = y >= bt0;
+                        r = y - (up ? c1 : c0);
+                        if (up) cellw[(j + e) >> 4] += 1u << (2 * ((j + e) & 15));
                     }
-                    if (B > 1) r = y - sm.c[cc];
-                    ccur[(j + e) >> 3] += cc << (4 * ((j + e) & 7));
-                    rr[j + e] = r * r;
+                    rr = fmaf(r, r, rr);
                     sr[e] = r;
                 }
                 const __half2 h1 = __floats2half2_rn(sr[0], sr[1]);
                 const float2 f1 = __half22float2(h1);
-                const __half2 h2 = __floats2half2_rn(sr[0] - f1.x, sr[1] - f1.y);
-                hp1[j >> 1] = *reinterpret_cast<const uint32_t*>(&h1);
-                hp2[j >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+                hp1[j >> 1] = h2_bits(h1);
+                hp2[j >> 1] = h2_bits(__floats2half2_rn(sr[0] - f1.x, sr[1] - f1.y));
             }
-            uint8_t* r0 = sm.r[b][0];
-            uint8_t* r1 = sm.r[b][1];
-#pragma unroll
-            for (int ii = 0; ii < V / 8; ++ii) {
-                *reinterpret_cast<uint4*>(r0 + roff[ii]) =
-                    make_uint4(hp1[4 * ii], hp1[4 * ii + 1], hp1[4 * ii + 2], hp1[4 * ii + 3]);
-                *reinterpret_cast<uint4*>(r1 + roff[ii]) =
-                    make_uint4(hp2[4 * ii], hp2[4 * ii + 1], hp2[4 * ii + 2], hp2[4 * ii + 3]);
+            // the QJL MMA of the pending tile still reads the R columns
+            if (pend && !wait_d2()) {
+                running = false;
+                break;
             }
-            const float tot = transpose_reduce<V>(rr, lane);
-            if (lane < V) sm.rr[b][q][V * h + lane] = tot;
-            fence_proxy_async_smem();
+            tmem_st16(lane_addr + kColR + 16u * h, hp1);
+            tmem_st16(lane_addr + kColR + 64u + 16u * h, hp2);
+            sm.rr[b][h][m] = rr;
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.r_full);
 
-            if (pend && !finish()) return running = false;
+            if (pend) finish();
             pend = true;
             pg = g;
             pt = t;
-            pidx = i;
+            pidx = (uint32_t)k;
 #pragma unroll
-            for (int u = 0; u < V / 8; ++u) pcell[u] = ccur[u];
-            ++i;
-            return true;
-        });
-        if (running && pend) finish();
+            for (int u = 0; u < 4; ++u) pcell[u] = cellw[u];
+        }
+        if (running && pend && wait_d2()) finish();
     }
 
     tc_fence_before();
@@ -670,9 +615,12 @@ int launch_b(const CUtensorMap& map, const float* Pi, const float* S, const KCod
 
 }  // namespace
 
-bool encode_tc_supported(int d, int x_dtype, int G, int64_t n) {
-    return d == kD && x_dtype == TQ_BF16 && (int64_t)G * n < ((int64_t)1 << 31) &&
-           encode_tiled_fn() != nullptr;
+bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n) {
+    if (cb->d != kD || x_dtype != TQ_BF16 || (int64_t)G * n >= ((int64_t)1 << 31)) return false;
+    // the bucketize table holds at most one boundary per 32 / 2^10 of y
+    for (int k = 0; k + 2 < cb->levels; ++k)
+        if (!(cb->boundaries[k + 1] - cb->boundaries[k] > kLutStep / kRScale)) return false;
+    return encode_tiled_fn() != nullptr;
 }
 
 int launch_encode_tc(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,

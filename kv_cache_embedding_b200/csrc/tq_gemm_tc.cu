@@ -81,17 +81,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, one CTA.
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
           int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
@@ -194,7 +183,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
                         const uint32_t as = smem_u32(sm.a[s][pi_[q]]), bs = smem_u32(sm.b[s][pj_[q]]);
 #pragma unroll
                         for (int ks = 0; ks < kKB / 16; ++ks)
-                            mma_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
+                            mma_f16_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
                                    smem_desc_kmajor_sw128(bs + ks * 32), kIdesc,
                                    (h | q | ks) != 0);
                     }

@@ -78,7 +78,7 @@ namespace tq {
 int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const float* B,
                  bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
                  cudaStream_t s);
-bool encode_tc_supported(int d, int x_dtype, int G, int64_t n);
+bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n);
 // Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from bf16
 // pieces of A ([pa][M][K], pa = 1 or 3) and B ([3][N][K]); d_err as the
 // encode kernels' status word.

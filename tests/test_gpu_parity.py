@@ -379,6 +379,27 @@ def test_encode_tc_bf16_shapes(quant, oparams, tq_lib, G, n, b):
         PT.compare_encode(128, b, P.beta, gpu, ora, bound_flags=(n * 128 >= 10 ** 5))
 
 
+@pytest.mark.parametrize("b", [1, 4])
+def test_encode_tc_bf16_edge_rows(quant, oparams, tq_lib, b):
+    """Edge rows through the tensor-core kernel, which rescales every key by a
+    power of two before its fp16 conversion: zero, tiny (1e-30) and huge
+    (1e30) rows, an axis-aligned row and a row with one x1000 outlier."""
+    d = 128
+    x = synth.gaussian_rows(300, d, seed=4)
+    x[5] = 0.0
+    x[6] = 1e-30
+    x[7] = 1e30 / math.sqrt(d)
+    x[8, :] = 0.0
+    x[8, 17] = 2.0
+    x[9, 3] *= 1000.0
+    xb = x.to(torch.bfloat16)
+    for gpu, ora, P in _encode_both(quant, oparams, xb[None], d, b):
+        PT.compare_encode(d, b, P.beta, gpu, ora, bound_flags=False)
+    B = tq_lib.binding
+    assert B.tq_device_status(quant(d, b).ws.buf.data_ptr(),
+                              torch.cuda.current_stream().cuda_stream) == 0
+
+
 def test_encode_tc_matches_portable_path(quant, tq_lib):
     """The tensor-core kernel (bf16 input) and the SIMT path (the same values
     given as fp32) produce the same records up to boundary flips."""
