@@ -197,6 +197,31 @@ def test_score_groups_and_query_passes(quant, oparams, tq_lib, cuda, G, n, nq, b
         PT.compare_scores(s_gpu[g], s_ora, np.linalg.norm(_f64(qs[g]), axis=1), xn.astype(np.float64))
 
 
+@pytest.mark.parametrize("G,n,nq,d", [(3, 2051, 1, 128), (2, 4097, 3, 128), (1, 1027, 4, 128),
+                                      (2, 3000, 4, 256), (1, 1024, 2, 128)])
+def test_score_few_queries_shapes(quant, oparams, tq_lib, cuda, G, n, nq, d):
+    """b = 4 with at most 4 queries per group (the SIMT scoring kernel): 1, 3
+    and 4 queries, key counts that are not multiples of the 256 keys of a
+    block, d = 256, several groups; scores and top-10."""
+    b = 4
+    W = b * d // 32
+    qs = synth.gaussian_rows(G * nq, d, seed=70, norm_range=None).reshape(G, nq, d)
+    recs = [synth.random_records(n, W, seed=80 + g) for g in range(G)]
+    codes = tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+    tq = quant(d, b, 0, G)
+    s_gpu = _np(tq.score(codes, qs.cuda()))
+    vals, ids = tq.topk(codes, qs.cuda(), 10)
+    for g in range(G):
+        c, xn, rn = recs[g]
+        s_ora = O.score(oparams(d, b, g), c, xn, rn, _f64(qs[g]))
+        qn = np.linalg.norm(_f64(qs[g]), axis=1)
+        PT.compare_scores(s_gpu[g], s_ora, qn, xn.astype(np.float64))
+        PT.compare_topk(_np(vals[g]), _np(ids[g]), s_ora, 10, qn, float(xn.max()))
+
+
 @pytest.mark.parametrize("n,k,nq", [(4096, 10, 17), (2500, 1, 3), (2500, 32, 3), (33, 32, 2)])
 def test_topk(quant, oparams, tq_lib, cuda, n, k, nq):
     d, b = 128, 4
