@@ -47,6 +47,7 @@ def lib():
         L.tqo_mse_encode.argtypes = [i32, i32, P, P, P, i64, P, P, P, P, P, P]
         L.tqo_mse_score.argtypes = [i32, i32, P, i64, P, P, i64, P, P]
         L.tqo_mse_decode.argtypes = [i32, i32, P, P, i64, P, P, P]
+        L.tqo_softmax_weighted_sum.argtypes = [i64, i64, i32, P, P, P]
         _lib = L
     return _lib
 
@@ -280,3 +281,26 @@ def mse_decode(params, codes, xnorm):
     _check(lib().tqo_mse_decode(d, b, _p(params.c), _p(params.Pi), n, _p(codes),
                                 _p(_f32(xnorm)), _p(out)), "mse_decode")
     return out
+
+
+# ---------------------------------------------------------------- decode attention
+def softmax_weighted_sum(logits, values):
+    """out[t] = sum_j softmax(logits[t])_j values[j] in fp64: [nq, d]."""
+    logits = np.ascontiguousarray(_f64(logits)).reshape(-1, np.shape(values)[0])
+    values = np.ascontiguousarray(_f64(values))
+    nq, n = logits.shape
+    d = values.shape[1]
+    out = np.empty((nq, d), np.float64)
+    _check(lib().tqo_softmax_weighted_sum(nq, n, d, _p(logits), _p(values), _p(out)),
+           "softmax_weighted_sum")
+    return out
+
+
+def attention_decode(kparams, kcodes, kxnorm, krnorm, vparams, vcodes, vxnorm, q, scale):
+    """Decode attention over quantized keys and values: the logits are scale
+    times the inner-product estimates of the key records, the values are the
+    MSE-only dequantized rows; returns [nq, d]."""
+    logits = score(kparams, kcodes, kxnorm, krnorm, q) * float(scale)
+    values = mse_decode(vparams, vcodes, vxnorm)
+    return softmax_weighted_sum(logits, values)
+

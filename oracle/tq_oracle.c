@@ -712,3 +712,36 @@ int tqo_mse_decode(int d, int b, const float *c, const float *Pi, int64_t n,
     }
     return 0;
 }
+
+
+/* ---------------------------------------------------------------------------
+ * Decode attention over quantized keys and values (a reading: the pages stop
+ * at the attention logits of quant_prune_distill #674 and the comuna.ru
+ * summary; softmax and the value sum are the standard attention that those
+ * logits feed).  For every query row t:
+ *   l_j = scale * s_tj            (s: the estimated inner products)
+ *   p_j = exp(l_j - max_j l_j) / sum_j exp(l_j - max_j l_j)
+ *   out_t = sum_j p_j v_j         (v: the dequantized value rows)
+ * logits [nq][n], values [n][d], out [nq][d]; n >= 1.
+ * ------------------------------------------------------------------------- */
+int tqo_softmax_weighted_sum(int64_t nq, int64_t n, int d, const double *logits,
+                             const double *values, double *out)
+{
+    if (nq < 0 || n < 1 || d < 1) return -1;
+    for (int64_t t = 0; t < nq; t++) {
+        const double *l = logits + (size_t)t * n;
+        double mx = l[0], sum = 0.0;
+        for (int64_t j = 1; j < n; j++)
+            if (l[j] > mx) mx = l[j];
+        double *o = out + (size_t)t * d;
+        for (int i = 0; i < d; i++) o[i] = 0.0;
+        for (int64_t j = 0; j < n; j++) {
+            const double w = exp(l[j] - mx);
+            sum += w;
+            for (int i = 0; i < d; i++) o[i] += w * values[(size_t)j * d + i];
+        }
+        for (int i = 0; i < d; i++) o[i] /= sum;
+    }
+    return 0;
+}
+

@@ -78,6 +78,10 @@ int tqo_mse_score(int d, int b, const float *c, int64_t n, const uint32_t *codes
 int tqo_mse_decode(int d, int b, const float *c, const float *Pi, int64_t n,
                    const uint32_t *codes, const float *xnorm, double *out);
 
+/* Decode attention: out_t = sum_j softmax_j(logits_t) values_j (fp64). */
+int tqo_softmax_weighted_sum(int64_t nq, int64_t n, int d, const double *logits,
+                             const double *values, double *out);
+
 #ifdef __cplusplus
 }
 #endif
