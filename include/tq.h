@@ -81,6 +81,7 @@ extern "C" {
 #define TQ_OP_TOPK    3
 #define TQ_OP_DECODE  4
 #define TQ_OP_EXACT   5
+#define TQ_OP_ATTENTION 6
 
 /* codebook variants */
 #define TQ_VARIANT_PROD 0  /* inner-product quantizer: (b-1)-bit Lloyd-Max index
@@ -217,6 +218,31 @@ TQ_API int tq_logits_fp32(int d, int G, int64_t n, const float *d_keys, int nq,
 TQ_API int tq_exact_topk(int d, int G, int64_t n, const float *d_x, int nq,
                   const void *d_q, int q_dtype, int k, float *d_vals,
                   int64_t *d_ids, void *d_ws, size_t ws_bytes, void *stream);
+
+/* Decode attention over quantized keys and values (d = 128).  The pages stop
+ * at the attention logits (comuna.ru "Google speeds up LLMs 8x": logits from
+ * 4-bit keys; quant_prune_distill #674: the inner-product estimate and its
+ * dequantization); this entry point takes the plain reading that those
+ * logits feed standard softmax attention.  For every group g and query row t:
+ *   l_j   = scale * s_tj      (s: the tq_score estimate of key record j)
+ *   out_t = sum_j softmax_j(l) vhat_j,
+ *   vhat_j = |v_j| Pi_v,g^T c_v[cell_j]   (the MSE-only dequantization).
+ * Keys: inner-product records of cb_k (TQ_VARIANT_PROD) with d_Pi_k, d_S_k;
+ * values: MSE-only records of cb_v (TQ_VARIANT_MSE) with d_Pi_v; both
+ * [G][n] records (layout above) with their norms.  d_q: [G][nq][d] (q_dtype);
+ * scale: finite (1/sqrt(d) for the usual attention); d_out: [G][nq][d] fp32.
+ * d_ws: >= tq_workspace_bytes(TQ_OP_ATTENTION, 128, b, G, n, nq, 0).
+ * n >= 1 and nq >= 1, else TQ_ERR_ARG; a variant other than PROD for cb_k or
+ * MSE for cb_v is TQ_ERR_ARG; d != 128 is TQ_ERR_UNSUPPORTED.  Support path,
+ * not part of the timed step. */
+TQ_API int tq_attention_decode(const tq_codebook_t *cb_k, const float *d_Pi_k,
+                               const float *d_S_k, const tq_codebook_t *cb_v,
+                               const float *d_Pi_v, int G, int64_t n,
+                               const uint32_t *d_kcodes, const float *d_kxnorm,
+                               const float *d_krnorm, const uint32_t *d_vcodes,
+                               const float *d_vxnorm, int nq, const void *d_q, int q_dtype,
+                               float scale, float *d_out, void *d_ws, size_t ws_bytes,
+                               void *stream);
 
 /* Top-k without a caller workspace, for callers that cannot allocate device
  * memory.  The pages have no counterpart of this entry point; it exists for

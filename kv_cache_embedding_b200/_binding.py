@@ -26,12 +26,13 @@ TQ_BF16 = 1
 TQ_VARIANT_PROD = 0
 TQ_VARIANT_MSE = 1
 
-TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT = range(6)
+(TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT,
+ TQ_OP_ATTENTION) = range(7)
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_build_codebook_mse",
            "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
-           "tq_device_status", "tq_selftest_wait_timeout")
+           "tq_device_status", "tq_selftest_wait_timeout", "tq_attention_decode")
 
 
 class tq_codebook_t(C.Structure):
@@ -88,6 +89,9 @@ def _load():
     L.tq_logits_fp32.argtypes = [i32, i32, i64, P, i32, P, i32, P, P]
     L.tq_exact_topk.restype = i32
     L.tq_exact_topk.argtypes = [i32, i32, i64, P, i32, P, i32, i32, P, P, P, sz, P]
+    L.tq_attention_decode.restype = i32
+    L.tq_attention_decode.argtypes = [cbp, P, P, cbp, P, i32, i64, P, P, P, P, P, i32, P, i32,
+                                      C.c_float, P, P, sz, P]
     return L
 
 
@@ -168,3 +172,13 @@ def tq_logits_fp32(d, G, n, d_keys, nq, d_q, q_dtype, d_out, stream):
 def tq_exact_topk(d, G, n, d_x, nq, d_q, q_dtype, k, d_vals, d_ids, d_ws, ws_bytes, stream):
     return _ok("tq_exact_topk", lib.tq_exact_topk(d, G, n, d_x, nq, d_q, q_dtype, k, d_vals,
                                                   d_ids, d_ws, ws_bytes, stream))
+
+
+def tq_attention_decode(cb_k, d_Pi_k, d_S_k, cb_v, d_Pi_v, G, n, d_kcodes, d_kxnorm, d_krnorm,
+                        d_vcodes, d_vxnorm, nq, d_q, q_dtype, scale, d_out, d_ws, ws_bytes,
+                        stream):
+    return _ok("tq_attention_decode",
+               lib.tq_attention_decode(C.byref(cb_k), d_Pi_k, d_S_k, C.byref(cb_v), d_Pi_v, G, n,
+                                       d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, nq, d_q,
+                                       q_dtype, scale, d_out, d_ws, ws_bytes, stream))
+

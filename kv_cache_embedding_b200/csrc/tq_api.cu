@@ -46,6 +46,9 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
             return 2 * align256((size_t)chunk * d * 4);
         case TQ_OP_EXACT:
             return align256((size_t)nq * ((chunk + 3) & ~int64_t(3)) * 4) + parts;
+        case TQ_OP_ATTENTION:  // d = 128 only; status word, queries, split partials
+            if (d != 128 || n < 1 || nq < 1) return (size_t)-1;
+            return attn_workspace_bytes(G, n, nq);
         default:
             return (size_t)-1;
     }

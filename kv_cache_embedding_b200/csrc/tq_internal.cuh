@@ -78,6 +78,14 @@ namespace tq {
 int launch_sgemm(int M, int N, int K, const void* A, int a_dtype, int lda, const float* B,
                  bool b_nk, int ldb, float* C, int ldc, const float* row_scale, int scale_mode,
                  cudaStream_t s);
+// qr = Q Pi^T and u = qr S^T (S may be null: u = 0) for every group's nq
+// query rows (fp32 or bf16); clears the device status word *err.
+int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const void* d_q,
+               int q_dtype, float* qr, float* u, int* err, cudaStream_t s);
+// Argument checks shared by the scoring entry points.
+int check_common(const tq_codebook_t* cb, int G, int64_t n, int nq, int q_dtype);
+// Decode attention (tq_attention.cu): workspace of tq_attention_decode.
+size_t attn_workspace_bytes(int G, int64_t n, int nq);
 bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n);
 // Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from bf16
 // pieces of A ([pa][M][K], pa = 1 or 3) and B ([3][N][K]); d_err as the

@@ -139,6 +139,26 @@ class TurboQuant:
                   _ptr(out[0]), _ptr(out[1]), wp, wn, _stream())
         return out
 
+    def attention_decode(self, kcodes, values, vcodes, q, scale=None, out=None):
+        """Softmax attention of the queries q [G, nq, d] over the keys encoded
+        by this (inner-product) quantizer and the values encoded by `values`
+        (an MSE-only TurboQuant of the same d and groups): [G, nq, d] fp32.
+        scale defaults to 1/sqrt(d)."""
+        q = self._grouped(q)
+        nq = q.shape[1]
+        n = kcodes.n
+        if scale is None:
+            scale = self.d ** -0.5
+        if out is None:
+            out = torch.empty(self.G, nq, self.d, dtype=torch.float32, device=self.device)
+        wp, wn = self.ws.get(B.tq_workspace_bytes(B.TQ_OP_ATTENTION, self.d, self.b, self.G, n,
+                                                  nq, 0))
+        B.tq_attention_decode(self.cb, _ptr(self.Pi), _ptr(self.S), values.cb, _ptr(values.Pi),
+                              self.G, n, _ptr(kcodes.codes), _ptr(kcodes.xnorm),
+                              _ptr(kcodes.rnorm), _ptr(vcodes.codes), _ptr(vcodes.xnorm), nq,
+                              _ptr(q), _dtype_code(q), float(scale), _ptr(out), wp, wn, _stream())
+        return out
+
     def decode(self, codes, out=None):
         n = codes.n
         if out is None:

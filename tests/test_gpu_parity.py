@@ -537,3 +537,60 @@ def test_mse_decode(quant_mse, tq_lib, cuda, b):
     got = _np(quant_mse(d, b).decode(_to_codes(tq_lib, c, xn, rn, cuda))[0]).astype(np.float64)
     err = np.linalg.norm(got - ref, axis=1) / np.linalg.norm(ref, axis=1)
     assert err.max() <= 1e-4, err.max()
+
+
+# ---------------------------------------------------------------- decode attention
+def _records_on(tq_lib, cuda, recs):
+    return tq_lib.Codes(
+        torch.stack([torch.from_numpy(r[0].view(np.int32)) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[1]) for r in recs]).to(cuda),
+        torch.stack([torch.from_numpy(r[2]) for r in recs]).to(cuda))
+
+
+def _attention_case(quant, quant_mse, oparams, tq_lib, cuda, G, n, nq, b_k, b_v, seed,
+                    groups_checked=None):
+    d = 128
+    krecs = [synth.random_records(n, b_k * d // 32, seed=seed + g) for g in range(G)]
+    vrecs = [synth.random_records(n, b_v * d // 32, seed=seed + 100 + g) for g in range(G)]
+    if nq % 4 == 0 and G * nq >= G:
+        qs = synth.kv_queries(G * nq, G, d, seed=seed + 200)
+    else:
+        qs = synth.gaussian_rows(G * nq, d, seed=seed + 200, norm_range=None).reshape(G, nq, d)
+    tk, tv = quant(d, b_k, 0, G), quant_mse(d, b_v, 1, G)
+    out = _np(tk.attention_decode(_records_on(tq_lib, cuda, krecs), tv,
+                                  _records_on(tq_lib, cuda, vrecs), qs.cuda()))
+    scale = 1.0 / math.sqrt(d)
+    for g in (groups_checked if groups_checked is not None else range(G)):
+        kc, kxn, krn = krecs[g]
+        vc, vxn, _ = vrecs[g]
+        Pk, Pv = oparams(d, b_k, g), O.MseParams(d, b_v, 1 + g)
+        ora = O.attention_decode(Pk, kc, kxn, krn, Pv, vc, vxn, _f64(qs[g]), scale)
+        vmax = np.abs(O.mse_decode(Pv, vc, vxn)).max()
+        err = np.abs(out[g] - ora).max()
+        assert err <= 1e-4 * vmax, (g, err, vmax)
+
+
+@pytest.mark.parametrize("G,n,nq,b_k,b_v", [(2, 3001, 4, 4, 4), (1, 5000, 1, 3, 2),
+                                            (3, 257, 8, 2, 3), (1, 1, 4, 4, 4),
+                                            (2, 70_000, 4, 4, 4), (1, 600, 2, 1, 1)])
+def test_attention_decode(quant, quant_mse, oparams, tq_lib, cuda, G, n, nq, b_k, b_v):
+    """Softmax attention over key and value records against the oracle: GQA
+    groups of 4 queries, one query, two query passes, a single key, splits
+    of many tiles with a ragged last tile, every key and value bit width.
+    Bound: |out - oracle| <= 1e-4 max |vhat| (the logits agree to ~1e-6
+    relative, the fp32 sums over <= 4096 keys per split to ~1e-6)."""
+    _attention_case(quant, quant_mse, oparams, tq_lib, cuda, G, n, nq, b_k, b_v, seed=300)
+
+
+def test_attention_decode_errors(quant, quant_mse, tq_lib, cuda):
+    tk, tv = quant(128, 4), quant_mse(128, 4)
+    empty = tq_lib.Codes(torch.zeros(1, 0, 16, dtype=torch.int32, device=cuda),
+                         torch.zeros(1, 0, device=cuda), torch.zeros(1, 0, device=cuda))
+    q = torch.randn(1, 4, 128, device=cuda)
+    with pytest.raises(tq_lib.binding.TQError):
+        tk.attention_decode(empty, tv, empty, q)
+    one = tq_lib.Codes(torch.zeros(1, 1, 16, dtype=torch.int32, device=cuda),
+                       torch.ones(1, 1, device=cuda), torch.zeros(1, 1, device=cuda))
+    with pytest.raises(tq_lib.binding.TQError):  # keys must be inner-product records
+        tv.attention_decode(one, tv, one, q)
+
