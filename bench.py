@@ -538,7 +538,38 @@ def run_ours(args, cfg, rank, world, dist):
                        "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / topk_ms * 1e3, 1)}
     if args.config == "decode" and rank == 0:
         out["fp32_baseline"] = fp32_baseline(cfg, x, q, flush, args)
+        out["attention"] = attention_decode_time(cfg, x, q, flush, args)
     return out
+
+
+def attention_decode_time(cfg, x, q, flush, args):
+    """Decode attention over the same keys (b-bit inner-product records) and
+    seeded values (4-bit MSE-only records): one tq_attention_decode call per
+    timed iteration, L2 flushed in between.  Not part of the step."""
+    import kv_cache_embedding_b200 as K
+    import synth
+    G, n, d = cfg["G"], cfg["n"], cfg["d"]
+    tk = K.TurboQuant(d, cfg["b"], seed=0, groups=G, device=x.device)
+    tv = K.TurboQuant(d, 4, seed=1, groups=G, device=x.device, variant="mse")
+    kc = tk.encode(x)
+    vc = tv.encode(synth.kv_keys(G, n, d, seed=5, device=x.device))
+    out = tk.attention_decode(kc, tv, vc, q)
+    for _ in range(3):
+        tk.attention_decode(kc, tv, vc, q, out=out)
+    ts = []
+    for _ in range(max(3, min(args.steps, 50))):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        tk.attention_decode(kc, tv, vc, q, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    ms = sum(ts) / len(ts)
+    byts = (kc.codes.numel() * 4 + kc.xnorm.numel() * 8 + vc.codes.numel() * 4 +
+            vc.xnorm.numel() * 4 + q.numel() * q.element_size() + out.numel() * 4)
+    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1),
+            "values": "4-bit MSE-only records (seeded keys-like rows)", "scale": "1/sqrt(d)"}
 
 
 def fp32_baseline(cfg, x, q, flush, args):

@@ -75,6 +75,30 @@ def test_decode_logits_full_size(tq_lib, cuda):
                           xn[r].astype(np.float64))
 
 
+def test_decode_attention_full_size(tq_lib, cuda):
+    """Decode attention at 131072 tokens x 8 KV heads, 32 query heads (GQA
+    4:1), 4-bit keys and 4-bit MSE-only values (seeded records): the launch
+    the bench times; the first and last KV heads checked whole against the
+    oracle with the bound of the small cases."""
+    G, n, d, per = 8, 131072, 128, 4
+    q = synth.kv_queries(G * per, G, d, seed=2, device=cuda, key_seed=1)
+    krecs = [synth.random_records(n, 16, seed=500 + g) for g in range(G)]
+    vrecs = [synth.random_records(n, 16, seed=600 + g) for g in range(G)]
+    tk = tq_lib.TurboQuant(d, 4, seed=0, groups=G, device=cuda)
+    tv = tq_lib.TurboQuant(d, 4, seed=1, groups=G, device=cuda, variant="mse")
+    out = _np(tk.attention_decode(_records_on_device(tq_lib, krecs, cuda), tv,
+                                  _records_on_device(tq_lib, vrecs, cuda), q))
+    for g in (0, G - 1):
+        kc, kxn, krn = krecs[g]
+        vc, vxn, _ = vrecs[g]
+        Pv = O.MseParams(d, 4, 1 + g)
+        qg = q[g].float().cpu().to(torch.float64).numpy()
+        ora = O.attention_decode(O.Params(d, 4, g), kc, kxn, krn, Pv, vc, vxn, qg,
+                                 1.0 / np.sqrt(d))
+        vmax = np.abs(O.mse_decode(Pv, vc, vxn)).max()
+        assert np.abs(out[g] - ora).max() <= 1e-4 * vmax
+
+
 @pytest.mark.parametrize("b", [2, 4])
 def test_embedding_search_full_size(tq_lib, cuda, b):
     """1e6 x 1536 fp32 unit rows, 1024 queries, top-10: sampled encode parity
