@@ -25,7 +25,8 @@
 // any K, as in the SIMT path.
 //
 // Tiles: 128 rows (MMA M) x 128 columns (MMA N), K in blocks of 64 staged by
-// TMA with the 128-byte swizzle (two stages).  Warp 0 issues the TMA loads,
+// TMA with the 128-byte swizzle, in as many stages as 12 pieces of 16 KB hold
+// (2 for 3 + 3 pieces, 3 for 2 + 2, 4 for 1 + 2 ...).  Warp 0 issues the TMA loads,
 // warp 1 owns tensor memory and issues the MMAs, warps 2-5 (one per TMEM lane
 // quarter) add up the chunk sums and store the tile.  Every wait is bounded
 // (1 s); a warp that gives up sets the abort flag and the status word.
@@ -44,17 +45,19 @@ using namespace sm100;
 
 constexpr int kTM = 128, kTN = 128, kKB = 64;        // tile rows, columns, K block
 constexpr int kPieceBytes = kTM * kKB * 2;            // one bf16 piece of a tile (16 KB)
-constexpr int kStages = 2;
+constexpr int kPool = 12;                             // 16 KB operand pieces in shared memory
+constexpr int kMaxStages = 6;
 constexpr int kThreads = 32 * 6;
 constexpr uint32_t kTmemCols = 2 * kTN;               // two chunk accumulators
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t kIdesc = idesc_f16(1, kTM, kTN);   // bf16 x bf16 -> f32, K-major A and B
 
 struct SmemG {
-    uint8_t a[kStages][3][kPieceBytes];  // A pieces (1024-aligned, first)
-    uint8_t b[kStages][3][kPieceBytes];  // B pieces
+    // stage s holds pieces [s (pa + pb), (s + 1)(pa + pb)): A's pa, then B's pb
+    // (1024-aligned, first); as many stages as the pool holds, up to 6
+    uint8_t pool[kPool][kPieceBytes];
     float tkey[4][kTN];                  // per epilogue warp: its 32 rows' maximum per column
-    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], mma_done, tmax_bar, tmax_bar2;
+    uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done, tmax_bar, tmax_bar2;
     uint32_t tmem_base;
     int abort;
     int zero;
@@ -96,9 +99,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
     const int nkb = K / kKB;            // K blocks per tile
     const int nch = nkb / 2;            // 128-wide K chunks per tile
     const uint32_t stage_tx = (uint32_t)(pa + pb) * kPieceBytes;
+    const int ns = min(kMaxStages, kPool / (pa + pb));  // pipeline stages
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kMaxStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -133,22 +137,23 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             const int m0 = (t / tn) * kTM, n0 = (t % tn) * kTN;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kStages;
-                if (it >= (uint32_t)kStages &&
-                    !mbar_wait(&sm.empty[s], ((it / kStages) - 1) & 1, abort, kWaitNs)) {
+                const int s = (int)(it % (uint32_t)ns);
+                if (it >= (uint32_t)ns &&
+                    !mbar_wait(&sm.empty[s], ((it / ns) - 1) & 1, abort, kWaitNs)) {
                     ok = give_up(abort, err, 41);
                     break;
                 }
                 mbar_arrive_expect_tx(&sm.full[s], stage_tx);
+                uint8_t* st = sm.pool[s * (pa + pb)];
                 for (int p = 0; p < pa; ++p)
-                    tma_load_3d(sm.a[s][p], &tmap_a, kb * kKB, m0, p, &sm.full[s]);
+                    tma_load_3d(st + p * kPieceBytes, &tmap_a, kb * kKB, m0, p, &sm.full[s]);
                 for (int p = 0; p < pb; ++p)
-                    tma_load_3d(sm.b[s][p], &tmap_b, kb * kKB, n0, p, &sm.full[s]);
+                    tma_load_3d(st + (pa + p) * kPieceBytes, &tmap_b, kb * kKB, n0, p, &sm.full[s]);
             }
         }
         // no TMA write may still be in flight when the CTA exits
-        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0); j < it; ++j)
-            mbar_wait(&sm.full[j % kStages], (j / kStages) & 1, &sm.zero, kWaitNs);
+        for (uint32_t j = (it > (uint32_t)ns ? it - ns : 0); j < it; ++j)
+            mbar_wait(&sm.full[j % ns], (j / ns) & 1, &sm.zero, kWaitNs);
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer ----------------
         // products a_i b_j with i + j < max(pa, pb), by increasing i + j
@@ -173,14 +178,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
                 tc_fence_after();
                 const uint32_t d = tbase + ab * kTN;
                 for (int h = 0; h < 2; ++h, ++it) {
-                    const int s = it % kStages;
-                    if (!mbar_wait(&sm.full[s], (it / kStages) & 1, abort, kWaitNs)) {
+                    const int s = (int)(it % (uint32_t)ns);
+                    if (!mbar_wait(&sm.full[s], (it / ns) & 1, abort, kWaitNs)) {
                         ok = give_up(abort, err, 43);
                         break;
                     }
                     tc_fence_after();
                     for (int q = 0; q < np; ++q) {
-                        const uint32_t as = smem_u32(sm.a[s][pi_[q]]), bs = smem_u32(sm.b[s][pj_[q]]);
+                        const uint32_t as = smem_u32(sm.pool[s * (pa + pb) + pi_[q]]),
+                                       bs = smem_u32(sm.pool[s * (pa + pb) + pa + pj_[q]]);
 #pragma unroll
                         for (int ks = 0; ks < kKB / 16; ++ks)
                             mma_f16_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
