@@ -48,7 +48,8 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
             return align256((size_t)nq * ((chunk + 3) & ~int64_t(3)) * 4) + parts;
         case TQ_OP_ATTENTION:  // d = 128 only; status word, queries, split partials
             if (d != 128 || n < 1 || nq < 1) return (size_t)-1;
-            return attn_workspace_bytes(G, n, nq);
+            if (b < 1 || b > 4) return (size_t)-1;
+            return attn_workspace_bytes(b, G, n, nq);
         default:
             return (size_t)-1;
     }

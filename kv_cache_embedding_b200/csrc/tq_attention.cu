@@ -11,13 +11,16 @@
 // value sum are the standard attention those logits feed (the pages do not
 // describe this step).
 //
-// Design: split-K over the keys of a group (flash-decoding).  A block takes
-// `split` keys in tiles of 256 (one key per thread for the logits, the same
-// estimator code as tq_score), keeps a running maximum and sum per query, and
+// Design: the logits come from tq_score itself (its scoring kernels for the
+// group's query count) into the workspace; then split-K over the keys of a
+// group (flash-decoding).  A block takes `split` keys in tiles of 256, keeps a
+// running maximum and sum per query, and
 // accumulates sum_j p_j |v_j| c_v[cell_j] in the rotated value domain: thread
-// (coordinate k, half h) walks the tile's value records staged in shared
-// memory.  Because Pi_v^T is linear it is applied once per query, after the
-// splits are merged (k_attn_combine), instead of once per value.
+// (coordinate pair, quarter of the tile) walks the tile's value records staged
+// in shared memory and updates both coordinates with packed fp32x2 FMAs (at
+// b_v = 4 one byte-indexed table load gives both centroids).  Because Pi_v^T
+// is linear it is applied once per query, after the splits are merged
+// (k_attn_combine), instead of once per value.
 #include <cmath>
 
 #include "tq_internal.cuh"
@@ -26,7 +29,7 @@
 namespace tq {
 namespace {
 
-using namespace sc;
+using sc::ffma2;
 
 constexpr int kAD = 128;         // head dimension
 constexpr int kAT = 256;         // keys per tile = threads per block
@@ -42,26 +45,22 @@ __device__ __forceinline__ uint32_t value_cell(const uint32_t* blk, int j) {
     return (blk[0] >> j) & 1u;
 }
 
-template <int B, int BV, int NQ>
-__global__ __launch_bounds__(kAT) void k_attn_partial(
-    const uint32_t* __restrict__ kcodes, const float* __restrict__ kxn,
-    const float* __restrict__ krn, const uint32_t* __restrict__ vcodes,
-    const float* __restrict__ vxn, int64_t n, int nq, const float* __restrict__ qr,
-    const float* __restrict__ u, KCodebook kcb, KCodebook vcb, float scale, int split,
+template <int BV, int NQ>
+__global__ __launch_bounds__(kAT, 8) void k_attn_partial(
+    const float* __restrict__ logits, const uint32_t* __restrict__ vcodes,
+    const float* __restrict__ vxn, int64_t n, int nq, KCodebook vcb, float scale, int split,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_acc) {
-    constexpr int WK = B * kAD / 32, WV = BV * kAD / 32;
-    __shared__ __align__(16) float2 s_qu[NQ * kAD];
-    __shared__ float2 s_tab[16];
+    constexpr int WV = BV * kAD / 32;
     __shared__ float s_vc[16];
+    __shared__ float2 s_vpair[256];  // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble])
     __shared__ uint32_t s_vcodes[kAT * WV];
     __shared__ __align__(16) float s_w[kAT][NQ];
     __shared__ float s_red[kAT / 32][NQ];
-    __shared__ float s_half[NQ][kAD];
+    __shared__ float2 s_part[3][NQ][kAD / 2];
     const int g = blockIdx.y, sp = blockIdx.x, nsplit = gridDim.x;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
     const int t = threadIdx.x, lane = t % 32, warp = t / 32;
-    load_score_smem<B, NQ>(kcb, qr, u, (int64_t)g * nq + q0, qn, kAD, s_qu, s_tab);
     if (t < 16) {
         float c = 0.f;
         switch (t) {  // static indices keep the codebook in parameter space
@@ -73,35 +72,31 @@ __global__ __launch_bounds__(kAT) void k_attn_partial(
         s_vc[t] = c;
     }
     __syncthreads();
+    if (BV == 4) s_vpair[t] = make_float2(s_vc[t & 15], s_vc[t >> 4]);
 
     const int64_t r_beg = (int64_t)sp * split;
     const int64_t r_end = min(n, r_beg + split);
-    const float k0 = kSqrtHalfPi / (float)kAD;
-    const int kc = t % kAD, h = t / kAD;  // value phase: coordinate, half of the tile
-    const int vblk = kc / 32, vj = kc % 32;
-    float M[NQ], L[NQ], accv[NQ];
+    // value phase: coordinates 2 cp, 2 cp + 1 over quarter hq of every tile
+    const int cp = t % (kAD / 2), hq = t / (kAD / 2);
+    const int vblk = (2 * cp) / 32, vj = (2 * cp) % 32;
+    float M[NQ], L[NQ];
+    float2 accv[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
         M[q] = -INFINITY;
         L[q] = 0.f;
-        accv[q] = 0.f;
+        accv[q] = make_float2(0.f, 0.f);
     }
     for (int64_t r = r_beg; r < r_end; r += kAT) {
         const int cnt = (int)min((int64_t)kAT, r_end - r);
         const int64_t j = r + t;
         const bool ok = t < cnt;
         const int64_t gj = (int64_t)g * n + (ok ? j : r);
-        // logits of this thread's key
-        float2 acc[1][NQ];
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) acc[0][q] = make_float2(0.f, 0.f);
-        const uint32_t* rec[1] = {kcodes + gj * WK};
-        score_keys<B, NQ, 1, true>(rec, kAD, s_qu, s_tab, acc);
+        // scaled logits of this thread's key
         float l[NQ];
-        const float xn = kxn[gj], kap = k0 * krn[gj];
 #pragma unroll
         for (int q = 0; q < NQ; ++q)
-            l[q] = ok ? scale * (xn * (acc[0][q].x + kap * acc[0][q].y)) : -INFINITY;
+            l[q] = (ok && q < qn) ? scale * logits[((int64_t)g * nq + q0 + q) * n + j] : -INFINITY;
         // the tile's value records, staged whole (coalesced)
         const uint32_t* vsrc = vcodes + ((int64_t)g * n + r) * WV;
         for (int e = t; e < cnt * WV; e += kAT) s_vcodes[e] = vsrc[e];
@@ -135,21 +130,31 @@ __global__ __launch_bounds__(kAT) void k_attn_partial(
             for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
             if (lane == 0) s_red[warp][q] = ps;
         }
-        // value sums of this thread's coordinate over its half of the tile
+        // value sums of this thread's coordinate pair over its quarter of the tile
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) accv[q] *= alpha[q];
-        const int jj1 = min(cnt, kAT / 2 * (h + 1));
-        for (int jj = kAT / 2 * h; jj < jj1; ++jj) {
-            const float c = s_vc[value_cell<BV>(s_vcodes + jj * WV + vblk * BV, vj)];
+        for (int q = 0; q < NQ; ++q) {
+            accv[q].x *= alpha[q];
+            accv[q].y *= alpha[q];
+        }
+        const int jj1 = min(cnt, kAT / 4 * (hq + 1));
+        for (int jj = kAT / 4 * hq; jj < jj1; ++jj) {
+            const uint32_t* blk = s_vcodes + jj * WV + vblk * BV;
+            float2 c2;
+            if (BV == 4) {
+                c2 = s_vpair[__byte_perm(blk[vj >> 3], 0u, 0x4440u | ((vj >> 1) & 3))];
+            } else {
+                c2 = make_float2(s_vc[value_cell<BV>(blk, vj)], s_vc[value_cell<BV>(blk, vj + 1)]);
+            }
             if (NQ == 4) {
                 const float4 w4 = *reinterpret_cast<const float4*>(&s_w[jj][0]);
-                accv[0] = fmaf(w4.x, c, accv[0]);
-                accv[1] = fmaf(w4.y, c, accv[1]);
-                accv[2] = fmaf(w4.z, c, accv[2]);
-                accv[3] = fmaf(w4.w, c, accv[3]);
+                accv[0] = ffma2(make_float2(w4.x, w4.x), c2, accv[0]);
+                accv[1 % NQ] = ffma2(make_float2(w4.y, w4.y), c2, accv[1 % NQ]);
+                accv[2 % NQ] = ffma2(make_float2(w4.z, w4.z), c2, accv[2 % NQ]);
+                accv[3 % NQ] = ffma2(make_float2(w4.w, w4.w), c2, accv[3 % NQ]);
             } else {
 #pragma unroll
-                for (int q = 0; q < NQ; ++q) accv[q] = fmaf(s_w[jj][q], c, accv[q]);
+                for (int q = 0; q < NQ; ++q)
+                    accv[q] = ffma2(make_float2(s_w[jj][q], s_w[jj][q]), c2, accv[q]);
             }
         }
         __syncthreads();  // s_red holds the tile sums; s_vcodes / s_w may be reused
@@ -162,19 +167,22 @@ __global__ __launch_bounds__(kAT) void k_attn_partial(
         }
         __syncthreads();  // s_red is rewritten by the next tile
     }
-    // merge the two halves of every coordinate and write the split's partials
-    if (h == 1) {
+    // merge the four quarters of every coordinate pair and write the split's partials
+    if (hq > 0) {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) s_half[q][kc] = accv[q];
+        for (int q = 0; q < NQ; ++q) s_part[hq - 1][q][cp] = accv[q];
     }
     __syncthreads();
-    if (h == 0) {
+    if (hq == 0) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
             if (q >= qn) continue;
             const int64_t row = (int64_t)g * nq + q0 + q;
-            part_acc[(row * nsplit + sp) * kAD + kc] = accv[q] + s_half[q][kc];
-            if (kc == 0) {
+            const float2 a1 = s_part[0][q][cp], a2 = s_part[1][q][cp], a3 = s_part[2][q][cp];
+            const float2 sum = make_float2((accv[q].x + a1.x) + (a2.x + a3.x),
+                                           (accv[q].y + a1.y) + (a2.y + a3.y));
+            *reinterpret_cast<float2*>(&part_acc[(row * nsplit + sp) * kAD + 2 * cp]) = sum;
+            if (cp == 0) {
                 part_m[row * nsplit + sp] = M[q];
                 part_l[row * nsplit + sp] = L[q];
             }
@@ -211,61 +219,47 @@ __global__ __launch_bounds__(kAD) void k_attn_combine(const float* __restrict__ 
     out[row * kAD + k] = o;
 }
 
-template <int B, int BV, int NQ>
-int launch_partial(dim3 grid, const uint32_t* kc, const float* kx, const float* kr,
-                   const uint32_t* vc, const float* vx, int64_t n, int nq, const float* qr,
-                   const float* u, const KCodebook& kcb, const KCodebook& vcb, float scale,
-                   int split, float* pm, float* pl, float* pa, cudaStream_t s) {
-    k_attn_partial<B, BV, NQ><<<grid, kAT, 0, s>>>(kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb,
-                                                   scale, split, pm, pl, pa);
+template <int BV, int NQ>
+int launch_partial(dim3 grid, const float* logits, const uint32_t* vc, const float* vx, int64_t n,
+                   int nq, const KCodebook& vcb, float scale, int split, float* pm, float* pl,
+                   float* pa, cudaStream_t s) {
+    k_attn_partial<BV, NQ><<<grid, kAT, 0, s>>>(logits, vc, vx, n, nq, vcb, scale, split, pm, pl,
+                                               pa);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
 
-template <int B, int BV>
-int launch_partial_nq(dim3 grid, int NQ, const uint32_t* kc, const float* kx, const float* kr,
-                      const uint32_t* vc, const float* vx, int64_t n, int nq, const float* qr,
-                      const float* u, const KCodebook& kcb, const KCodebook& vcb, float scale,
-                      int split, float* pm, float* pl, float* pa, cudaStream_t s) {
-    if (NQ == 1)
-        return launch_partial<B, BV, 1>(grid, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale,
-                                        split, pm, pl, pa, s);
-    return launch_partial<B, BV, 4>(grid, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale,
-                                    split, pm, pl, pa, s);
-}
-
-template <int B>
-int launch_partial_bv(int bv, dim3 grid, int NQ, const uint32_t* kc, const float* kx,
-                      const float* kr, const uint32_t* vc, const float* vx, int64_t n, int nq,
-                      const float* qr, const float* u, const KCodebook& kcb, const KCodebook& vcb,
-                      float scale, int split, float* pm, float* pl, float* pa, cudaStream_t s) {
-    switch (bv) {
-        case 1: return launch_partial_nq<B, 1>(grid, NQ, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale, split, pm, pl, pa, s);
-        case 2: return launch_partial_nq<B, 2>(grid, NQ, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale, split, pm, pl, pa, s);
-        case 3: return launch_partial_nq<B, 3>(grid, NQ, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale, split, pm, pl, pa, s);
-        default: return launch_partial_nq<B, 4>(grid, NQ, kc, kx, kr, vc, vx, n, nq, qr, u, kcb, vcb, scale, split, pm, pl, pa, s);
-    }
+template <int BV>
+int launch_partial_nq(dim3 grid, int NQ, const float* logits, const uint32_t* vc, const float* vx,
+                      int64_t n, int nq, const KCodebook& vcb, float scale, int split, float* pm,
+                      float* pl, float* pa, cudaStream_t s) {
+    if (NQ == 1) return launch_partial<BV, 1>(grid, logits, vc, vx, n, nq, vcb, scale, split, pm, pl, pa, s);
+    return launch_partial<BV, 4>(grid, logits, vc, vx, n, nq, vcb, scale, split, pm, pl, pa, s);
 }
 
 }  // namespace
 
 // Queries per pass and keys per split of the decode-attention kernels: enough
-// blocks for two per SM over all groups and passes, splits of whole tiles.
+// blocks for eight per SM over all groups and passes (the tile loop waits on
+// its loads; other blocks hide that), splits of whole tiles.
 int attn_queries_per_pass(int nq) { return nq <= 1 ? 1 : 4; }
 
 int64_t attn_split(int64_t n, int G, int nq) {
     const int64_t passes = (nq + attn_queries_per_pass(nq) - 1) / attn_queries_per_pass(nq);
-    const int64_t want = 2 * 148;
+    const int64_t want = 8 * 148;
     int64_t per = (n * G * passes + want - 1) / want;
     per = (per + kAT - 1) / kAT * kAT;
     return per < kAT ? kAT : (per > kAttnSplitMax ? kAttnSplitMax : per);
 }
 
-size_t attn_workspace_bytes(int G, int64_t n, int nq) {
+// [tq_score's workspace (its status word first) | logits [G][nq][n] |
+//  split maxima | split sums | split value sums [G][nq][nsplit][d]]
+size_t attn_workspace_bytes(int b, int G, int64_t n, int nq) {
     const int64_t split = attn_split(n, G, nq);
     const int64_t nsplit = (n + split - 1) / split;
     const size_t rows = (size_t)G * nq;
-    return 256 + 2 * align256(rows * kAD * 4) + 2 * align256(rows * nsplit * 4) +
+    return align256(tq_workspace_bytes(TQ_OP_SCORE, kAD, b, G, n, nq, 0)) +
+           align256(rows * (size_t)n * 4) + 2 * align256(rows * nsplit * 4) +
            align256(rows * nsplit * kAD * 4);
 }
 
@@ -290,28 +284,29 @@ extern "C" int tq_attention_decode(const tq_codebook_t* cb_k, const float* d_Pi_
     if (!d_Pi_k || !d_S_k || !d_Pi_v || !d_kcodes || !d_kxnorm || !d_krnorm || !d_vcodes ||
         !d_vxnorm || !d_q || !d_out || !std::isfinite(scale))
         return TQ_ERR_ARG;
-    const size_t need = attn_workspace_bytes(G, n, nq);
+    const size_t need = attn_workspace_bytes(cb_k->b, G, n, nq);
     if (!d_ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t split = attn_split(n, G, nq);
     const int64_t nsplit = (n + split - 1) / split;
     const size_t rows = (size_t)G * nq;
-    int* err = (int*)d_ws;
-    float* qr = (float*)((char*)d_ws + 256);
-    float* u = (float*)((char*)qr + align256(rows * kAD * 4));
-    float* pm = (float*)((char*)u + align256(rows * kAD * 4));
+    const size_t score_ws = align256(tq_workspace_bytes(TQ_OP_SCORE, kAD, cb_k->b, G, n, nq, 0));
+    float* logits = (float*)((char*)d_ws + score_ws);
+    float* pm = (float*)((char*)logits + align256(rows * (size_t)n * 4));
     float* pl = (float*)((char*)pm + align256(rows * nsplit * 4));
     float* pa = (float*)((char*)pl + align256(rows * nsplit * 4));
-    int rc = query_prep(d_Pi_k, d_S_k, G, kAD, nq, d_q, q_dtype, qr, u, err, s);
+    // the estimated inner products, by the scoring path tq_score takes for nq
+    int rc = tq_score(cb_k, d_Pi_k, d_S_k, G, n, d_kcodes, d_kxnorm, d_krnorm, nq, d_q, q_dtype,
+                      logits, d_ws, score_ws, stream);
     if (rc) return rc;
     const int NQ = attn_queries_per_pass(nq);
     const dim3 grid((unsigned)nsplit, (unsigned)G, (unsigned)((nq + NQ - 1) / NQ));
-    const KCodebook kcb = make_kcodebook(cb_k), vcb = make_kcodebook(cb_v);
-    switch (cb_k->b) {
-        case 1: rc = launch_partial_bv<1>(cb_v->b, grid, NQ, d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, n, nq, qr, u, kcb, vcb, scale, (int)split, pm, pl, pa, s); break;
-        case 2: rc = launch_partial_bv<2>(cb_v->b, grid, NQ, d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, n, nq, qr, u, kcb, vcb, scale, (int)split, pm, pl, pa, s); break;
-        case 3: rc = launch_partial_bv<3>(cb_v->b, grid, NQ, d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, n, nq, qr, u, kcb, vcb, scale, (int)split, pm, pl, pa, s); break;
-        default: rc = launch_partial_bv<4>(cb_v->b, grid, NQ, d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, n, nq, qr, u, kcb, vcb, scale, (int)split, pm, pl, pa, s); break;
+    const KCodebook vcb = make_kcodebook(cb_v);
+    switch (cb_v->b) {
+        case 1: rc = launch_partial_nq<1>(grid, NQ, logits, d_vcodes, d_vxnorm, n, nq, vcb, scale, (int)split, pm, pl, pa, s); break;
+        case 2: rc = launch_partial_nq<2>(grid, NQ, logits, d_vcodes, d_vxnorm, n, nq, vcb, scale, (int)split, pm, pl, pa, s); break;
+        case 3: rc = launch_partial_nq<3>(grid, NQ, logits, d_vcodes, d_vxnorm, n, nq, vcb, scale, (int)split, pm, pl, pa, s); break;
+        default: rc = launch_partial_nq<4>(grid, NQ, logits, d_vcodes, d_vxnorm, n, nq, vcb, scale, (int)split, pm, pl, pa, s); break;
     }
     if (rc) return rc;
     k_attn_combine<<<dim3((unsigned)nq, (unsigned)G), kAD, 0, s>>>(pm, pl, pa, (int)nsplit, nq,

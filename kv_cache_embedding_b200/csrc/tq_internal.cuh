@@ -85,7 +85,7 @@ int query_prep(const float* d_Pi, const float* d_S, int G, int d, int nq, const 
 // Argument checks shared by the scoring entry points.
 int check_common(const tq_codebook_t* cb, int G, int64_t n, int nq, int q_dtype);
 // Decode attention (tq_attention.cu): workspace of tq_attention_decode.
-size_t attn_workspace_bytes(int G, int64_t n, int nq);
+size_t attn_workspace_bytes(int b, int G, int64_t n, int nq);
 bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n);
 // Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from bf16
 // pieces of A ([pa][M][K], pa = 1 or 3) and B ([3][N][K]); d_err as the
