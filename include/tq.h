@@ -219,6 +219,17 @@ TQ_API int tq_exact_topk(int d, int G, int64_t n, const float *d_x, int nq,
                   const void *d_q, int q_dtype, int k, float *d_vals,
                   int64_t *d_ids, void *d_ws, size_t ws_bytes, void *stream);
 
+/* Merge of top-k lists computed on shards of one database (SURVEY-style
+ * search sharding: each shard's tq_topk, ids made global by the caller, then
+ * one merge; the pages' vector search is one top-k over all records).
+ * d_vals / d_ids: [nlists][rows][k] (the layout of an all-gather of every
+ * shard's [rows][k] lists); missing entries carry id INT64_MAX.  Output:
+ * [rows][k], values non-increasing, ties by smaller id (the tq_topk order).
+ * 1 <= k <= 32 and nlists >= 1, else TQ_ERR_ARG.  No workspace. */
+TQ_API int tq_topk_merge(int64_t rows, int nlists, int k, const float *d_vals,
+                         const int64_t *d_ids, float *d_out_vals, int64_t *d_out_ids,
+                         void *stream);
+
 /* Decode attention over quantized keys and values (d = 128).  The pages stop
  * at the attention logits (comuna.ru "Google speeds up LLMs 8x": logits from
  * 4-bit keys; quant_prune_distill #674: the inner-product estimate and its

@@ -32,7 +32,8 @@ TQ_VARIANT_MSE = 1
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_build_codebook_mse",
            "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
-           "tq_device_status", "tq_selftest_wait_timeout", "tq_attention_decode")
+           "tq_device_status", "tq_selftest_wait_timeout", "tq_attention_decode",
+           "tq_topk_merge")
 
 
 class tq_codebook_t(C.Structure):
@@ -89,6 +90,8 @@ def _load():
     L.tq_logits_fp32.argtypes = [i32, i32, i64, P, i32, P, i32, P, P]
     L.tq_exact_topk.restype = i32
     L.tq_exact_topk.argtypes = [i32, i32, i64, P, i32, P, i32, i32, P, P, P, sz, P]
+    L.tq_topk_merge.restype = i32
+    L.tq_topk_merge.argtypes = [i64, i32, i32, P, P, P, P, P]
     L.tq_attention_decode.restype = i32
     L.tq_attention_decode.argtypes = [cbp, P, P, cbp, P, i32, i64, P, P, P, P, P, i32, P, i32,
                                       C.c_float, P, P, sz, P]
@@ -181,4 +184,9 @@ def tq_attention_decode(cb_k, d_Pi_k, d_S_k, cb_v, d_Pi_v, G, n, d_kcodes, d_kxn
                lib.tq_attention_decode(C.byref(cb_k), d_Pi_k, d_S_k, C.byref(cb_v), d_Pi_v, G, n,
                                        d_kcodes, d_kxnorm, d_krnorm, d_vcodes, d_vxnorm, nq, d_q,
                                        q_dtype, scale, d_out, d_ws, ws_bytes, stream))
+
+
+def tq_topk_merge(rows, nlists, k, d_vals, d_ids, d_out_vals, d_out_ids, stream):
+    return _ok("tq_topk_merge", lib.tq_topk_merge(rows, nlists, k, d_vals, d_ids, d_out_vals,
+                                                  d_out_ids, stream))
 

@@ -395,21 +395,25 @@ __global__ __launch_bounds__(256) void k_rows_topk_tile(const float* __restrict_
     }
 }
 
-// Merge [rows][nparts][K] partial lists (missing entries: id INT64_MAX) into
-// the final K per row.  One warp per row (4 rows per 128-thread block): the
-// entries stream through a running best-K list, 16 per lane loaded ahead.
+// Merge partial lists of K entries (missing entries: id INT64_MAX) into the
+// final K per row; list p of row r starts at r * row_stride + p * list_stride
+// ([rows][nparts][K]: K * nparts, K; [nparts][rows][K]: K, rows * K).  One warp
+// per row (4 rows per 128-thread block): the entries stream through a running
+// best-K list, 16 per lane loaded ahead.
 __global__ __launch_bounds__(128) void k_topk_merge(const float* __restrict__ part_vals,
                                                     const int64_t* __restrict__ part_ids,
                                                     int64_t rows, int nparts, int K,
                                                     float* __restrict__ vals,
-                                                    int64_t* __restrict__ ids) {
+                                                    int64_t* __restrict__ ids,
+                                                    int64_t row_stride, int64_t list_stride) {
     constexpr int C = 16;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int64_t row = (int64_t)blockIdx.x * 4 + warp;
     if (row >= rows) return;
-    const float* pv = part_vals + row * nparts * K;
-    const int64_t* pi = part_ids + row * nparts * K;
+    const float* pv = part_vals + row * row_stride;
+    const int64_t* pi = part_ids + row * row_stride;
     const int64_t count = (int64_t)nparts * K;
+    const bool packed = list_stride == K;
     WarpList<int64_t> L;
     L.init();
     for (int64_t base = 0; base < count; base += 32 * C) {
@@ -418,8 +422,9 @@ __global__ __launch_bounds__(128) void k_topk_merge(const float* __restrict__ pa
 #pragma unroll
         for (int j = 0; j < C; ++j) {
             const int64_t e = base + 32 * j + lane;
-            v[j] = e < count ? pv[e] : -INFINITY;
-            id[j] = e < count ? pi[e] : INT64_MAX;
+            const int64_t a = packed ? e : (e / K) * list_stride + e % K;
+            v[j] = e < count ? pv[a] : -INFINITY;
+            id[j] = e < count ? pi[a] : INT64_MAX;
         }
 #pragma unroll
         for (int j = 0; j < C; ++j) L.offer(id[j] != INT64_MAX, v[j], id[j], K, lane);
@@ -854,7 +859,8 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         default: rc = launch_topk_b<4>(d_codes, d_xnorm, d_rnorm, n, d, G, nq, qr, u, kc, k, pv, pi, &tg, s); break;
     }
     if (rc) return rc;
-    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, tg.nblk, k, d_vals, d_ids);
+    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, tg.nblk, k, d_vals, d_ids,
+                                                             (int64_t)tg.nblk * k, k);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -1018,7 +1024,24 @@ extern "C" int tq_exact_topk(int d, int G, int64_t n, const float* d_x, int nq, 
         }
     }
     const int64_t rows = (int64_t)G * nq;
-    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, ntiles, k, d_vals, d_ids);
+    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, ntiles, k, d_vals, d_ids,
+                                                             (int64_t)ntiles * k, k);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
+
+// Merge of top-k lists computed on shards of a database (on one GPU or on
+// several, gathered): every list already holds global ids.
+extern "C" int tq_topk_merge(int64_t rows, int nlists, int k, const float* d_vals,
+                             const int64_t* d_ids, float* d_out_vals, int64_t* d_out_ids,
+                             void* stream) {
+    if (rows < 0 || nlists < 1 || k < 1 || k > kMaxK) return TQ_ERR_ARG;
+    if (rows == 0) return TQ_OK;
+    if (!d_vals || !d_ids || !d_out_vals || !d_out_ids) return TQ_ERR_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(d_vals, d_ids, rows, nlists, k,
+                                                             d_out_vals, d_out_ids, k, rows * k);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+

@@ -594,3 +594,37 @@ def test_attention_decode_errors(quant, quant_mse, tq_lib, cuda):
     with pytest.raises(tq_lib.binding.TQError):  # keys must be inner-product records
         tv.attention_decode(one, tv, one, q)
 
+
+# ---------------------------------------------------------------- sharded search merge
+@pytest.mark.parametrize("nshards,k", [(3, 10), (5, 32), (1, 4)])
+def test_topk_merge_of_shards(quant, oparams, tq_lib, cuda, nshards, k):
+    """tq_topk on uneven shards of one record set, ids made global, merged by
+    tq_topk_merge: equal to tq_topk over the whole set (same scores, same
+    order) and to the oracle; duplicates straddle a shard cut (tie order)."""
+    from kv_cache_embedding_b200 import sharded
+    d, b, n, G, nq = 128, 4, 20_011, 2, 4
+    recs = [list(synth.random_records(n, b * d // 32, seed=700 + g)) for g in range(G)]
+    cut = sharded.shard_bounds(n, nshards, 0)[1]
+    for r in recs:
+        r[0][cut - 5:cut + 5], r[1][cut - 5:cut + 5], r[2][cut - 5:cut + 5] = r[0][3], r[1][3], r[2][3]
+    qs = synth.gaussian_rows(G * nq, d, seed=710, norm_range=None).reshape(G, nq, d)
+    tq = quant(d, b, 0, G)
+    whole = _records_on(tq_lib, cuda, recs)
+    wv, wi = tq.topk(whole, qs.cuda(), k)
+    lv, li = [], []
+    for sh in range(nshards):
+        a, e = sharded.shard_bounds(n, nshards, sh)
+        part = tq_lib.Codes(whole.codes[:, a:e].contiguous(), whole.xnorm[:, a:e].contiguous(),
+                            whole.rnorm[:, a:e].contiguous())
+        v, i = tq.topk(part, qs.cuda(), k)
+        lv.append(v.reshape(-1, k))
+        li.append((i + a).reshape(-1, k))
+    mv, mi = sharded.merge_lists(torch.stack(lv), torch.stack(li), k)
+    torch.cuda.synchronize()
+    assert torch.equal(mi.reshape(wi.shape), wi) and torch.equal(mv.reshape(wv.shape), wv)
+    for g in range(G):
+        c, xn, rn = recs[g]
+        s_ora = O.score(oparams(d, b, g), c, xn, rn, _f64(qs[g]))
+        PT.compare_topk(_np(mv.reshape(wv.shape)[g]), _np(mi.reshape(wi.shape)[g]), s_ora, k,
+                        np.linalg.norm(_f64(qs[g]), axis=1), float(xn.max()))
+
