@@ -48,6 +48,7 @@ constexpr int kPieceBytes = kTM * kKB * 2;            // one bf16 piece of a til
 constexpr int kPool = 12;                             // 16 KB operand pieces in shared memory
 constexpr int kMaxStages = 6;
 constexpr int kThreads = 32 * 6;
+constexpr int kThreadsDecode = 32 * 8;                // + 2 warps decoding A from records
 constexpr uint32_t kTmemCols = 2 * kTN;               // two chunk accumulators
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr uint32_t kIdesc = idesc_f16(1, kTM, kTN);   // bf16 x bf16 -> f32, K-major A and B
@@ -57,6 +58,9 @@ struct SmemG {
     // (1024-aligned, first); as many stages as the pool holds, up to 6
     uint8_t pool[kPool][kPieceBytes];
     float tkey[4][kTN];                  // per epilogue warp: its 32 rows' maximum per column
+    uint32_t dtab[16];                   // decoded-A mode: packed bf16 pieces of c[cell]
+    uint2 dpair[256][8];                 // b = 4: code byte -> (hi pair, lo pair) words, 8 copies
+    uint32_t dsign[256];                 // b = 4: code byte -> sign flips of the pair (z = 0)
     uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done, tmax_bar, tmax_bar2;
     uint32_t tmem_base;
     int abort;
@@ -84,11 +88,159 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Decoded-A mode: rows rl and rl + 32 of tile m0, K block kb (64 of the
+// K = 2d columns: the centroid half, then the sign half), written as the
+// bf16 pieces hi / lo in the 128-byte-swizzled K-major layout of a TMA box.
+// The code words of rows rl and rl + 32 of tile m0 for K block kb (2 blocks
+// of 32 coordinates = 2B words each) and those rows' |r|.
+template <int B>
+__device__ __forceinline__ void load_rows(const KeyDecode& kd, int64_t M, int m0, int kb, int rl,
+                                          uint32_t (&w)[2][2 * B], float (&rn)[2]) {
+    const int W = kd.d / 32 * B;
+    const int c0 = kb * kKB >= kd.d ? kb * kKB - kd.d : kb * kKB;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int64_t row = (int64_t)m0 + rl + 32 * half;
+        const int64_t src = row < M ? row : 0;  // rows past M decode row 0 (not stored)
+        const uint32_t* rec = kd.codes + src * W + (c0 / 32) * B;
+#pragma unroll
+        for (int i = 0; i < 2 * B; ++i) w[half][i] = __ldg(rec + i);
+        rn[half] = __ldg(kd.rnorm + src);
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void decode_rows(const KeyDecode& kd, const uint32_t* dtab,
+                                            const uint2* dpair, const uint32_t* dsign, int kb,
+                                            int rl, const uint32_t (&wr)[2][2 * B],
+                                            const float (&rn)[2], uint8_t* hi, uint8_t* lo) {
+    const bool sgn = kb * kKB >= kd.d;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int r = rl + 32 * half;
+        const uint32_t* w = wr[half];
+        uint32_t kp = 0u;  // bf16 hi | lo << 16 of kappa
+        if (sgn && !kd.mse) {
+            const float kap = kd.kscale * rn[half];
+            const __nv_bfloat16 h = __float2bfloat16_rn(kap);
+            const __nv_bfloat16 l = __float2bfloat16_rn(kap - __bfloat162float(h));
+            kp = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(l) << 16);
+        }
+        if (B == 4) {  // one code byte = one coordinate pair: table lookups
+            const uint32_t khi = (kp & 0xffffu) * 0x10001u, klo = (kp >> 16) * 0x10001u;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {  // chunk u: word u of the two blocks
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t f = __byte_perm(w[u], 0u, 0x4440u | e);
+                    if (!sgn) {
+                        const uint2 pr = dpair[f * 8 + (rl & 7)];
+                        hw[e] = pr.x;
+                        lw[e] = pr.y;
+                    } else if (kd.mse) {
+                        hw[e] = 0u;
+                        lw[e] = 0u;
+                    } else {
+                        const uint32_t fl = dsign[f];
+                        hw[e] = khi ^ fl;
+                        lw[e] = klo ^ fl;
+                    }
+                }
+                const uint32_t off = (uint32_t)r * 128u + ((((uint32_t)u) ^ ((uint32_t)r & 7u)) << 4);
+                *reinterpret_cast<uint4*>(hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            continue;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {  // 16-byte chunks of 8 coordinates
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t v[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int j = 8 * u + 2 * e + h2, blk = j >> 5, jj = j & 31;
+                    uint32_t idx, z;
+                    if (B == 4) {
+                        const uint32_t f = (w[blk * 4 + (jj >> 3)] >> (4 * (jj & 7))) & 15u;
+                        idx = f & 7u;
+                        z = f >> 3;
+                    } else if (B == 3) {
+                        idx = (w[blk * 3 + (jj >> 4)] >> (2 * (jj & 15))) & 3u;
+                        z = (w[blk * 3 + 2] >> jj) & 1u;
+                    } else if (B == 2) {
+                        const uint32_t f = (w[blk * 2 + (jj >> 4)] >> (2 * (jj & 15))) & 3u;
+                        idx = f & 1u;
+                        z = f >> 1;
+                    } else {
+                        idx = 0u;
+                        z = (w[blk] >> jj) & 1u;
+                    }
+                    if (!sgn) {
+                        v[h2] = dtab[kd.mse ? (idx | (z << (B - 1))) : idx];
+                    } else {
+                        v[h2] = kd.mse ? 0u : (z ? kp : (kp ^ 0x80008000u));
+                    }
+                }
+                hw[e] = __byte_perm(v[0], v[1], 0x5410);  // the two hi halves
+                lw[e] = __byte_perm(v[0], v[1], 0x7632);  // the two lo halves
+            }
+            const uint32_t off = (uint32_t)r * 128u + ((((uint32_t)u) ^ ((uint32_t)r & 7u)) << 4);
+            *reinterpret_cast<uint4*>(hi + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(lo + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+    }
+}
+
+// Decoded-A producer (one of the two decode warps): every (tile, K block) in
+// the order of the other roles, the next block's words loaded while the
+// current one is decoded.  Returns false when a wait gave up.
+template <int B>
+__device__ bool decode_loop(const KeyDecode& kd, SmemG& sm, int64_t M, int tiles, int tn, int nkb,
+                            int ns, int pa, int pb, int rl, volatile int* abort, int* err) {
+    const int lane = threadIdx.x % 32;
+    int t = blockIdx.x, kb = 0;
+    if (t >= tiles) return true;
+    uint32_t wc[2][2 * B], wn[2][2 * B];
+    float rc[2], rnx[2];
+    load_rows<B>(kd, M, (t / tn) * kTM, kb, rl, wc, rc);
+    for (uint32_t it = 0;; ++it) {
+        // the next (tile, K block)
+        int t2 = t, kb2 = kb + 1;
+        if (kb2 == nkb) {
+            kb2 = 0;
+            t2 += gridDim.x;
+        }
+        const bool more = t2 < tiles;
+        if (more) load_rows<B>(kd, M, (t2 / tn) * kTM, kb2, rl, wn, rnx);
+        const int s = (int)(it % (uint32_t)ns);
+        if (it >= (uint32_t)ns && !warp_wait(&sm.empty[s], ((it / ns) - 1) & 1, abort))
+            return give_up(abort, err, 47);
+        decode_rows<B>(kd, sm.dtab, &sm.dpair[0][0], sm.dsign, kb, rl, wc, rc,
+                       sm.pool[s * (pa + pb)], sm.pool[s * (pa + pb) + 1]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.full[s]);
+        if (!more) return true;
+        t = t2;
+        kb = kb2;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            rc[h] = rnx[h];
+#pragma unroll
+            for (int i = 0; i < 2 * B; ++i) wc[h][i] = wn[h][i];
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreadsDecode, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
           int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
           const float* __restrict__ row_scale, int scale_mode, int transposed, int n_store,
-          float* __restrict__ tmax, int64_t ldt, int* __restrict__ err) {
+          float* __restrict__ tmax, int64_t ldt, int* __restrict__ err, KeyDecode kd,
+          int decode) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     SmemG& sm = *reinterpret_cast<SmemG*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -98,12 +250,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
     const int tiles = tm * tn;
     const int nkb = K / kKB;            // K blocks per tile
     const int nch = nkb / 2;            // 128-wide K chunks per tile
-    const uint32_t stage_tx = (uint32_t)(pa + pb) * kPieceBytes;
+    const uint32_t stage_tx = (uint32_t)(decode ? pb : pa + pb) * kPieceBytes;
     const int ns = min(kMaxStages, kPool / (pa + pb));  // pipeline stages
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMaxStages; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], decode ? 3 : 1);  // TMA (+ the 2 decode warps)
             mbar_init(&sm.empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -117,6 +269,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
         sm.zero = 0;
         fence_mbar_init();
     }
+    if (decode && threadIdx.x < 16) {
+        uint32_t v = 0u;
+        switch (threadIdx.x) {  // static indices keep the table in parameter space
+#define TQ_DT(F) case F: v = kd.tab[F]; break;
+            TQ_DT(0) TQ_DT(1) TQ_DT(2) TQ_DT(3) TQ_DT(4) TQ_DT(5) TQ_DT(6) TQ_DT(7)
+            TQ_DT(8) TQ_DT(9) TQ_DT(10) TQ_DT(11) TQ_DT(12) TQ_DT(13) TQ_DT(14) TQ_DT(15)
+#undef TQ_DT
+        }
+        sm.dtab[threadIdx.x] = v;
+    }
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, kTmemCols);
         tmem_relinquish();
@@ -129,6 +291,17 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
+    if (decode && kd.b == 4) {  // pair tables from the centroid pieces
+        for (int e = threadIdx.x; e < 256 * 8; e += blockDim.x) {
+            const uint32_t f = (uint32_t)e >> 3;
+            const uint32_t a = sm.dtab[kd.mse ? (f & 15u) : (f & 7u)];
+            const uint32_t b = sm.dtab[kd.mse ? (f >> 4) : ((f >> 4) & 7u)];
+            sm.dpair[f][e & 7] = make_uint2(__byte_perm(a, b, 0x5410), __byte_perm(a, b, 0x7632));
+        }
+        for (int f = threadIdx.x; f < 256; f += blockDim.x)
+            sm.dsign[f] = ((f & 0x08) ? 0u : 0x8000u) | ((f & 0x80) ? 0u : 0x80000000u);
+        __syncthreads();
+    }
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer ----------------
@@ -145,8 +318,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
                 }
                 mbar_arrive_expect_tx(&sm.full[s], stage_tx);
                 uint8_t* st = sm.pool[s * (pa + pb)];
-                for (int p = 0; p < pa; ++p)
-                    tma_load_3d(st + p * kPieceBytes, &tmap_a, kb * kKB, m0, p, &sm.full[s]);
+                if (!decode)
+                    for (int p = 0; p < pa; ++p)
+                        tma_load_3d(st + p * kPieceBytes, &tmap_a, kb * kKB, m0, p, &sm.full[s]);
                 for (int p = 0; p < pb; ++p)
                     tma_load_3d(st + (pa + p) * kPieceBytes, &tmap_b, kb * kKB, n0, p, &sm.full[s]);
             }
@@ -201,6 +375,15 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
         // every issued MMA completes before tensor memory is released
         tc_commit(&sm.mma_done);
         mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
+    } else if (warp >= 6) {
+        // ---------------- A from code records (decoded-A mode) ----------------
+        const int rl = 64 * (warp - 6) + lane;  // rows rl, rl + 32 of every tile
+        switch (kd.b) {
+            case 1: decode_loop<1>(kd, sm, M, tiles, tn, nkb, ns, pa, pb, rl, abort, err); break;
+            case 2: decode_loop<2>(kd, sm, M, tiles, tn, nkb, ns, pa, pb, rl, abort, err); break;
+            case 3: decode_loop<3>(kd, sm, M, tiles, tn, nkb, ns, pa, pb, rl, abort, err); break;
+            default: decode_loop<4>(kd, sm, M, tiles, tn, nkb, ns, pa, pb, rl, abort, err); break;
+        }
     } else if (warp >= 2) {
         // ---------------- chunk sums and stores ----------------
         const int q = warp & 3;  // TMEM lane quarter: tile rows 32 q .. 32 q + 31
@@ -378,7 +561,29 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
                                      (int)kSmemBytes));
     k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
                                                   scale_mode, transposed ? 1 : 0, n_store, tmax,
-                                                  ldt, d_err);
+                                                  ldt, d_err, KeyDecode{}, 0);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
+int launch_gemm_tc_decoded(int M, int N, const KeyDecode& kd, const __nv_bfloat16* B, float* C,
+                           int64_t ldc, const float* row_scale, int* d_err, cudaStream_t s,
+                           int n_store, float* tmax, int64_t ldt) {
+    if (M <= 0) return TQ_OK;
+    const int K = 2 * kd.d;
+    if (!gemm_tc_supported(N, K) || kd.b < 1 || kd.b > 4) return TQ_ERR_ARG;
+    CUtensorMap mb;
+    if (!make_piece_map(&mb, B, 2, N, K)) return TQ_ERR_CUDA;
+    int dev = 0, nsm = 0;
+    TQ_TRY_CUDA(cudaGetDevice(&dev));
+    TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    const int64_t tiles = (int64_t)((M + kTM - 1) / kTM) * (N / kTN);
+    const int nctas = (int)(tiles < nsm ? tiles : nsm);
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes));
+    // the A map is unused in this mode: the B map stands in for the parameter
+    k_gemm_tc<<<nctas, kThreadsDecode, kSmemBytes, s>>>(mb, mb, M, N, K, 2, 2, C, ldc, row_scale,
+                                                        2, 1, n_store, tmax, ldt, d_err, kd, 1);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }

@@ -96,12 +96,26 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb = 3, bool transposed = false, int n_store = 0,
                    float* tmax = nullptr, int64_t ldt = 0);
+// A operand decoded from code records inside the GEMM (scoring of many
+// queries): row m of A = (c[idx] | kappa_m (2z - 1)) over K = 2d as bf16
+// pieces hi, lo (kappa_m = kscale |r_m|; the MSE-only variant has c[cell] and
+// zeros); tab[cell] = bf16 hi | bf16 lo << 16 of the centroid.
+struct KeyDecode {
+    const uint32_t* codes;  // [M][d/32 * b] records
+    const float* rnorm;     // [M]
+    int d, b, mse;
+    float kscale;           // sqrt(pi/2) / d
+    uint32_t tab[16];
+};
+// C^T tile store with per-128-row maxima, A decoded from records (pa = pb = 2).
+int launch_gemm_tc_decoded(int M, int N, const KeyDecode& kd, const __nv_bfloat16* B, float* C,
+                           int64_t ldc, const float* row_scale, int* d_err, cudaStream_t s,
+                           int n_store, float* tmax, int64_t ldt);
 // The encode path's dense products run on the tensor-core GEMM for d >= 256.
 inline bool encode_gemm_tc(int d) { return d >= 256; }
 // Scoring of many queries at d >= 256 as a GEMM over decoded keys
 // (tq_score_gemm.cu): scores [G][nq][n] (and per-128-key maxima [G][nq][ntm]).
 constexpr int kScoreGemmMinQueries = 64;
-constexpr int64_t kScoreGemmChunk = 32768;  // keys decoded per GEMM
 bool score_gemm_supported(int d, int nq);
 size_t score_gemm_workspace(int d, int64_t n, int nq);
 int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,

@@ -9,10 +9,14 @@
 // part plus the 1-bit QJL correction); comuna.ru "Google speeds up LLMs 8x"
 // (vector search over the quantized database).
 //
-// A and B are written as two bf16 pieces each (x = hi + lo to ~2^-16 of |x|)
-// and the GEMM sums hi hi + hi lo + lo hi, an error well inside the score
-// tolerance.  Scores go out transposed ([query][key], coalesced over keys)
-// with the maximum of every 128-key tile per query for the top-k threshold.
+// A and B are two bf16 pieces each (x = hi + lo to ~2^-16 of |x|) and the GEMM
+// sums hi hi + hi lo + lo hi, an error well inside the score tolerance.  Up
+// to 256 queries the keys' pieces are decoded from the records inside the
+// GEMM (two warps write them into each shared-memory stage), so only the
+// records cross HBM; with more queries they are decoded once per chunk of
+// 32768 keys into the workspace.  The queries' pieces come by TMA.  Scores go out transposed
+// ([query][key], coalesced over keys) with the maximum of every 128-key tile
+// per query for the top-k threshold.
 #include <cuda_bf16.h>
 
 #include "tq_internal.cuh"
@@ -21,6 +25,7 @@ namespace tq {
 namespace {
 
 constexpr float kSqrtHalfPi = 1.2533141373155002512f;
+constexpr int64_t kMaxRows = (int64_t)1 << 30;  // a multiple of 128
 
 __device__ __forceinline__ void split2(float v, __nv_bfloat16& hi, __nv_bfloat16& lo) {
     hi = __float2bfloat16_rn(v);
@@ -123,10 +128,20 @@ bool topk_materialized(int d, int G, int64_t n, int nq) {
     return (int64_t)G * nq * n <= kTopkMaterialize || score_gemm_supported(d, nq);
 }
 
+// Up to 256 queries the keys are decoded inside the GEMM (two query tiles per
+// key tile); beyond that re-decoding every key tile for each query tile costs
+// more than writing the decoded keys once per chunk and reading them back.
+constexpr int kDecodeInGemmMaxQueries = 256;
+constexpr int64_t kScoreGemmChunk = 32768;  // keys decoded per GEMM (materialised form)
+
 size_t score_gemm_workspace(int d, int64_t n, int nq) {
-    const int64_t chunk = n < kScoreGemmChunk ? n : kScoreGemmChunk;
     const int64_t nq_pad = (nq + 127) / 128 * 128;
-    return align256((size_t)2 * nq_pad * 2 * d * 2) + align256((size_t)2 * chunk * 2 * d * 2);
+    size_t bytes = align256((size_t)2 * nq_pad * 2 * d * 2);
+    if (nq_pad > kDecodeInGemmMaxQueries) {
+        const int64_t chunk = n < kScoreGemmChunk ? n : kScoreGemmChunk;
+        bytes += align256((size_t)2 * chunk * 2 * d * 2);
+    }
+    return bytes;
 }
 
 int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
@@ -135,32 +150,59 @@ int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_code
                cudaStream_t s) {
     const int d = cb->d, b = cb->b;
     const int W = words_per_vector(d, b);
-    const KCodebook kc = make_kcodebook(cb);
     const int nq_pad = (nq + 127) / 128 * 128;
-    const int64_t chunk = n < kScoreGemmChunk ? n : kScoreGemmChunk;
     __nv_bfloat16* Bq = (__nv_bfloat16*)op_ws;
-    __nv_bfloat16* Ak = (__nv_bfloat16*)((char*)op_ws + align256((size_t)2 * nq_pad * 2 * d * 2));
+    KeyDecode kd{};
+    kd.d = d;
+    kd.b = b;
+    kd.mse = is_mse(cb) ? 1 : 0;
+    kd.kscale = kSqrtHalfPi / (float)d;
+    for (int c = 0; c < 16; ++c) {  // bf16 pieces of every centroid
+        const float v = c < cb->levels ? cb->centroids[c] : 0.f;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+        kd.tab[c] = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(l) << 16);
+    }
     for (int g = 0; g < G; ++g) {
         const int64_t qn = (int64_t)nq_pad * 2 * d;
         k_query_operand<<<(unsigned)((qn + 255) / 256), 256, 0, s>>>(
             qr + (int64_t)g * nq * d, u + (int64_t)g * nq * d, nq, nq_pad, d, Bq);
         TQ_CHECK_LAUNCH();
-        for (int64_t r0 = 0; r0 < n; r0 += chunk) {
-            const int64_t rows = (n - r0) < chunk ? (n - r0) : chunk;
-            const int64_t off = (int64_t)g * n + r0;
-            const int64_t items = rows * (d / 32);
-            const unsigned blocks = (unsigned)((items + 255) / 256);
-            switch (b) {
-                case 1: k_key_operand<1><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
-                case 2: k_key_operand<2><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
-                case 3: k_key_operand<3><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
-                default: k_key_operand<4><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
+        if (nq_pad > kDecodeInGemmMaxQueries) {  // decoded keys through HBM, chunk by chunk
+            __nv_bfloat16* Ak =
+                (__nv_bfloat16*)((char*)op_ws + align256((size_t)2 * nq_pad * 2 * d * 2));
+            const KCodebook kc = make_kcodebook(cb);
+            const int64_t chunk = n < kScoreGemmChunk ? n : kScoreGemmChunk;
+            for (int64_t r0 = 0; r0 < n; r0 += chunk) {
+                const int64_t rows = (n - r0) < chunk ? (n - r0) : chunk;
+                const int64_t off = (int64_t)g * n + r0;
+                const unsigned blocks = (unsigned)((rows * (d / 32) + 255) / 256);
+                switch (b) {
+                    case 1: k_key_operand<1><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
+                    case 2: k_key_operand<2><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
+                    case 3: k_key_operand<3><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
+                    default: k_key_operand<4><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
+                }
+                TQ_CHECK_LAUNCH();
+                float* tm = tmax ? tmax + (int64_t)g * nq * ntm + r0 / 128 : nullptr;
+                const int rc = launch_gemm_tc((int)rows, nq_pad, 2 * d, Ak, 2, Bq,
+                                              scores + (int64_t)g * nq * n + r0, n, d_xnorm + off,
+                                              2, d_err, s, 2, true, nq, tm, ntm);
+                if (rc) return rc;
             }
-            TQ_CHECK_LAUNCH();
+            continue;
+        }
+        // key ranges of at most 2^30 (the GEMM's row count is an int); in
+        // practice one launch per group
+        for (int64_t r0 = 0; r0 < n; r0 += kMaxRows) {
+            const int64_t rows = (n - r0) < kMaxRows ? (n - r0) : kMaxRows;
+            const int64_t off = (int64_t)g * n + r0;
+            kd.codes = d_codes + off * W;
+            kd.rnorm = d_rnorm + off;
             float* tm = tmax ? tmax + (int64_t)g * nq * ntm + r0 / 128 : nullptr;
-            const int rc = launch_gemm_tc((int)rows, nq_pad, 2 * d, Ak, 2, Bq,
-                                          scores + (int64_t)g * nq * n + r0, n, d_xnorm + off, 2,
-                                          d_err, s, 2, true, nq, tm, ntm);
+            const int rc = launch_gemm_tc_decoded((int)rows, nq_pad, kd, Bq,
+                                                  scores + (int64_t)g * nq * n + r0, n,
+                                                  d_xnorm + off, d_err, s, nq, tm, ntm);
             if (rc) return rc;
         }
     }
