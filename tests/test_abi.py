@@ -69,6 +69,11 @@ def test_workspace_sizes(tq_lib):
     t = B.tq_workspace_bytes(B.TQ_OP_TOPK, 128, 4, 1, 10 ** 6, 1024, 10)
     assert t >= 1024 * ((10 ** 6 + 1023) // 1024) * 10 * 12
     assert B.tq_workspace_bytes(99, 128, 4, 1, 1, 1, 1) == big
+    # decode attention: d = 128 only, n >= 1; holds the logits [G][nq][n]
+    a = B.tq_workspace_bytes(B.TQ_OP_ATTENTION, 128, 4, 8, 131072, 4, 0)
+    assert a >= 8 * 4 * 131072 * 4 + s
+    assert B.tq_workspace_bytes(B.TQ_OP_ATTENTION, 256, 4, 1, 100, 4, 0) == big
+    assert B.tq_workspace_bytes(B.TQ_OP_ATTENTION, 128, 4, 1, 0, 4, 0) == big
 
 
 def test_bad_arguments_rejected_without_device_work(tq_lib):
@@ -98,6 +103,29 @@ def test_bad_arguments_rejected_without_device_work(tq_lib):
     assert lib.tq_decode(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 1, 1, 8, None) == B.TQ_ERR_WORKSPACE
     assert lib.tq_logits_fp32(96, 1, 10, 1, 1, 1, 0, 1, None) == B.TQ_ERR_UNSUPPORTED
     assert lib.tq_exact_topk(128, 1, 10, 1, 1, 1, 0, 20, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    # merge of shard lists
+    assert lib.tq_topk_merge(4, 2, 0, 1, 1, 1, 1, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk_merge(4, 2, 33, 1, 1, 1, 1, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk_merge(4, 0, 10, 1, 1, 1, 1, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk_merge(4, 2, 10, None, 1, 1, 1, None) == B.TQ_ERR_ARG
+    assert lib.tq_topk_merge(0, 2, 10, None, None, None, None, None) == B.TQ_OK
+    # decode attention: keys PROD, values MSE, d = 128, n >= 1, finite scale
+    kcb, vcb = B.tq_codebook_t(), B.tq_codebook_t()
+    kcb.d, kcb.b, kcb.groups, kcb.levels, kcb.variant = 128, 4, 1, 8, B.TQ_VARIANT_PROD
+    vcb.d, vcb.b, vcb.groups, vcb.levels, vcb.variant = 128, 4, 1, 16, B.TQ_VARIANT_MSE
+
+    def attn(k=kcb, v=vcb, G=1, n=10, nq=4, scale=0.1, ws=1 << 30):
+        return lib.tq_attention_decode(C.byref(k), 1, 1, C.byref(v), 1, G, n, 1, 1, 1, 1, 1, nq,
+                                       1, 0, scale, 1, 1, ws, None)
+    assert attn(n=0) == B.TQ_ERR_ARG
+    assert attn(nq=0) == B.TQ_ERR_ARG
+    assert attn(k=vcb) == B.TQ_ERR_ARG
+    assert attn(v=kcb) == B.TQ_ERR_ARG
+    assert attn(G=2) == B.TQ_ERR_MISMATCH
+    assert attn(scale=float("nan")) == B.TQ_ERR_ARG
+    assert attn(ws=64) == B.TQ_ERR_WORKSPACE
+    kcb.d = 96
+    assert attn() == B.TQ_ERR_UNSUPPORTED
 
 
 def test_binding_raises_on_error(tq_lib):
