@@ -219,9 +219,9 @@ TQ_API int tq_exact_topk(int d, int G, int64_t n, const float *d_x, int nq,
                   const void *d_q, int q_dtype, int k, float *d_vals,
                   int64_t *d_ids, void *d_ws, size_t ws_bytes, void *stream);
 
-/* Merge of top-k lists computed on shards of one database (SURVEY-style
- * search sharding: each shard's tq_topk, ids made global by the caller, then
- * one merge; the pages' vector search is one top-k over all records).
+/* Merge of top-k lists computed on shards of one database (each shard's
+ * tq_topk, ids made global by the caller, then one merge; the pages' vector
+ * search is one top-k over all records, and sharding does not change it).
  * d_vals / d_ids: [nlists][rows][k] (the layout of an all-gather of every
  * shard's [rows][k] lists); missing entries carry id INT64_MAX.  Output:
  * [rows][k], values non-increasing, ties by smaller id (the tq_topk order).

@@ -29,7 +29,7 @@
  *           independently on the fixed grid;
  *         - step 2): residual multiplied by a random matrix, keep the sign.
  *
- * Readings where the pages are silent (all listed in the design doc):
+ * Readings where the pages are silent (the plainest reading each time):
  *   R1  random numbers: SplitMix64 (Steele, Lea, Flood, OOPSLA 2014) in
  *       counter form, keyed by (seed, stream); Box-Muller for Gaussians.
  *   R2  Pi = Q * diag(sign R_jj) from the Householder QR of a Gaussian
