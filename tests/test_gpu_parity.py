@@ -296,12 +296,15 @@ def test_exact_topk_many_tiles(tq_lib, cuda):
 
 
 @pytest.mark.parametrize("d,b,G,n,nq,mse", [(256, 4, 2, 3000, 70, False), (384, 2, 1, 1025, 130, False),
-                                            (256, 3, 1, 2000, 64, True)])
+                                            (256, 3, 1, 2000, 64, True), (256, 4, 1, 1500, 100, True),
+                                            (512, 1, 1, 700, 64, False), (256, 4, 2, 1000, 300, False)])
 def test_score_and_topk_decoded_key_gemm(quant, quant_mse, oparams, tq_lib, cuda, d, b, G, n, nq,
                                          mse):
     """d >= 256 with 64+ queries per group: scores as a tensor-core GEMM over
     decoded keys (transposed store, per-tile maxima for the top-k); ragged key
-    tiles, padded query tiles, several groups, both variants."""
+    tiles, padded query tiles, several groups, both variants, every bit width
+    of the in-GEMM decode (b = 4 through its byte tables), and 300 queries
+    (decoded keys through the workspace)."""
     k = 10
     qs = synth.gaussian_rows(G * nq, d, seed=51, norm_range=None).reshape(G, nq, d)
     W = b * d // 32
