@@ -82,6 +82,7 @@ extern "C" {
 #define TQ_OP_DECODE  4
 #define TQ_OP_EXACT   5
 #define TQ_OP_ATTENTION 6
+#define TQ_OP_SCORE_TOPK 7
 
 /* codebook variants */
 #define TQ_VARIANT_PROD 0  /* inner-product quantizer: (b-1)-bit Lloyd-Max index
@@ -196,6 +197,18 @@ TQ_API int tq_topk(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
             const float *d_rnorm, int nq, const void *d_q, int q_dtype, int k,
             float *d_vals, int64_t *d_ids, void *d_ws, size_t ws_bytes,
             void *stream);
+
+/* S0-S2 in one call: the estimates of tq_score into d_scores and, from the
+ * same scoring pass, the top-k of tq_topk into d_vals / d_ids (the queries
+ * are transformed and scored once instead of once per call).  Arguments,
+ * shapes, results and errors are those of tq_score and tq_topk; d_scores is
+ * required.  d_ws: >= tq_workspace_bytes(TQ_OP_SCORE_TOPK, d, b, G, n, nq, k)
+ * (no room for the scores: they live in d_scores). */
+TQ_API int tq_score_topk(const tq_codebook_t *cb, const float *d_Pi, const float *d_S, int G,
+                         int64_t n, const uint32_t *d_codes, const float *d_xnorm,
+                         const float *d_rnorm, int nq, const void *d_q, int q_dtype, int k,
+                         float *d_scores, float *d_vals, int64_t *d_ids, void *d_ws,
+                         size_t ws_bytes, void *stream);
 
 /* Dequantization (quant_prune_distill #674: "inverse rotation and
  * renormalisation"):  xhat = |x| Pi_g^T (c[idx] + |r| sqrt(pi/2)/d S_g^T (2z-1)).

@@ -27,13 +27,13 @@ TQ_VARIANT_PROD = 0
 TQ_VARIANT_MSE = 1
 
 (TQ_OP_BUILD, TQ_OP_ENCODE, TQ_OP_SCORE, TQ_OP_TOPK, TQ_OP_DECODE, TQ_OP_EXACT,
- TQ_OP_ATTENTION) = range(7)
+ TQ_OP_ATTENTION, TQ_OP_SCORE_TOPK) = range(8)
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_build_codebook_mse",
            "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
            "tq_device_status", "tq_selftest_wait_timeout", "tq_attention_decode",
-           "tq_topk_merge")
+           "tq_topk_merge", "tq_score_topk")
 
 
 class tq_codebook_t(C.Structure):
@@ -90,6 +90,8 @@ def _load():
     L.tq_logits_fp32.argtypes = [i32, i32, i64, P, i32, P, i32, P, P]
     L.tq_exact_topk.restype = i32
     L.tq_exact_topk.argtypes = [i32, i32, i64, P, i32, P, i32, i32, P, P, P, sz, P]
+    L.tq_score_topk.restype = i32
+    L.tq_score_topk.argtypes = [cbp, P, P, i32, i64, P, P, P, i32, P, i32, i32, P, P, P, P, sz, P]
     L.tq_topk_merge.restype = i32
     L.tq_topk_merge.argtypes = [i64, i32, i32, P, P, P, P, P]
     L.tq_attention_decode.restype = i32
@@ -189,4 +191,11 @@ def tq_attention_decode(cb_k, d_Pi_k, d_S_k, cb_v, d_Pi_v, G, n, d_kcodes, d_kxn
 def tq_topk_merge(rows, nlists, k, d_vals, d_ids, d_out_vals, d_out_ids, stream):
     return _ok("tq_topk_merge", lib.tq_topk_merge(rows, nlists, k, d_vals, d_ids, d_out_vals,
                                                   d_out_ids, stream))
+
+
+def tq_score_topk(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_scores,
+                  d_vals, d_ids, d_ws, ws_bytes, stream):
+    return _ok("tq_score_topk",
+               lib.tq_score_topk(C.byref(cb), d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q,
+                                 q_dtype, k, d_scores, d_vals, d_ids, d_ws, ws_bytes, stream))
 

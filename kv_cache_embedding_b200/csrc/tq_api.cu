@@ -42,6 +42,8 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
             return 256 + 2 * qbuf + (score_gemm_supported(d, nq) ? score_gemm_workspace(d, n, nq) : 0);
         case TQ_OP_TOPK:
             return tq::topk_workspace_bytes(d, b, G, n, nq, k, topk_materialized(d, G, n, nq));
+        case TQ_OP_SCORE_TOPK:  // as TQ_OP_TOPK's materialised form, scores in the caller's output
+            return tq::topk_workspace_bytes(d, b, G, n, nq, k, true, false);
         case TQ_OP_DECODE:
             return 2 * align256((size_t)chunk * d * 4);
         case TQ_OP_EXACT:
@@ -56,13 +58,14 @@ extern "C" size_t tq_workspace_bytes(int op, int d, int b, int G, int64_t n, int
 }
 
 namespace tq {
-size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize) {
+size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize,
+                            bool scores_in_ws) {
     (void)b;
     const size_t qbuf = align256((size_t)G * nq * d * 4);
     if (materialize) {
         // scores, maxima per 128-key tile, counters, candidate lists (, GEMM operands)
         const int64_t ntm = (n + 127) / 128;
-        return 256 + 2 * qbuf + align256((size_t)G * nq * n * 4) +
+        return 256 + 2 * qbuf + (scores_in_ws ? align256((size_t)G * nq * n * 4) : 0) +
                align256((size_t)G * nq * ntm * 4) + align256((size_t)G * nq * 8) +
                2 * align256((size_t)G * nq * kTopkCandidates * 4) +
                (score_gemm_supported(d, nq) ? score_gemm_workspace(d, n, nq) : 0);

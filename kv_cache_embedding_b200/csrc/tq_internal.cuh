@@ -132,8 +132,11 @@ int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d
 int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
              const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
              const void* d_q, int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
-             size_t ws_bytes, bool materialize, cudaStream_t s);
-size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize);
+             size_t ws_bytes, bool materialize, cudaStream_t s, float* scores_out = nullptr);
+// scores_in_ws: the materialised path keeps the score matrix in the workspace
+// (false when the caller's score output holds it, as in tq_score_topk)
+size_t topk_workspace_bytes(int d, int b, int G, int64_t n, int nq, int k, bool materialize,
+                            bool scores_in_ws = true);
 // tq_topk's argument checks: TQ_OK to run, kTopkNothing when there is nothing
 // to compute (a successful no-op), else the error status.
 constexpr int kTopkNothing = 1;

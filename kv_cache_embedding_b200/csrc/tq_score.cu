@@ -780,9 +780,11 @@ namespace tq {
 int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
              const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
              const void* d_q, int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
-             size_t ws_bytes, bool materialize, cudaStream_t s) {
+             size_t ws_bytes, bool materialize, cudaStream_t s, float* scores_out) {
     const int d = cb->d, b = cb->b;
-    if (!d_ws || ws_bytes < topk_workspace_bytes(d, b, G, n, nq, k, materialize))
+    if (scores_out) materialize = true;
+    if (!d_ws ||
+        ws_bytes < topk_workspace_bytes(d, b, G, n, nq, k, materialize, scores_out == nullptr))
         return TQ_ERR_WORKSPACE;
     int rc;
     const int ntiles = (int)((n + kTopkTile - 1) / kTopkTile);
@@ -802,8 +804,11 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         // the per-row selection
         const bool tc = !is_mse(cb) && score_tc_supported(d, b, G, n, nq);
         const int64_t ntm = (n + 127) / 128;
-        float* sc = (float*)p;
-        p += align256((size_t)rows * n * 4);
+        float* sc = scores_out;  // the caller's score output, else the workspace
+        if (!sc) {
+            sc = (float*)p;
+            p += align256((size_t)rows * n * 4);
+        }
         float* cm = (float*)p;
         p += align256((size_t)rows * ntm * 4);
         int* cnt = (int*)p;  // [2][rows]: candidate counts, finished blocks
@@ -892,6 +897,19 @@ extern "C" int tq_topk(const tq_codebook_t* cb, const float* d_Pi, const float* 
     if (rc) return rc == kTopkNothing ? TQ_OK : rc;
     return topk_run(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
                     d_ids, d_ws, ws_bytes, topk_materialized(cb->d, G, n, nq), (cudaStream_t)stream);
+}
+
+extern "C" int tq_score_topk(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,
+                             int64_t n, const uint32_t* d_codes, const float* d_xnorm,
+                             const float* d_rnorm, int nq, const void* d_q, int q_dtype, int k,
+                             float* d_scores, float* d_vals, int64_t* d_ids, void* d_ws,
+                             size_t ws_bytes, void* stream) {
+    const int rc = topk_validate(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype,
+                                 k, d_vals, d_ids);
+    if (rc) return rc == kTopkNothing ? TQ_OK : rc;
+    if (!d_scores) return TQ_ERR_ARG;
+    return topk_run(cb, d_Pi, d_S, G, n, d_codes, d_xnorm, d_rnorm, nq, d_q, q_dtype, k, d_vals,
+                    d_ids, d_ws, ws_bytes, true, (cudaStream_t)stream, d_scores);
 }
 
 extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G,

@@ -159,6 +159,24 @@ class TurboQuant:
                               _ptr(q), _dtype_code(q), float(scale), _ptr(out), wp, wn, _stream())
         return out
 
+    def score_topk(self, codes, q, k, scores_out=None, topk_out=None):
+        """score() and topk() from one scoring pass: (scores [G, nq, n],
+        (vals, ids) [G, nq, k])."""
+        q = self._grouped(q)
+        nq = q.shape[1]
+        n = codes.n
+        if scores_out is None:
+            scores_out = torch.empty(self.G, nq, n, dtype=torch.float32, device=self.device)
+        if topk_out is None:
+            topk_out = (torch.empty(self.G, nq, k, dtype=torch.float32, device=self.device),
+                        torch.empty(self.G, nq, k, dtype=torch.int64, device=self.device))
+        wp, wn = self.ws.get(B.tq_workspace_bytes(B.TQ_OP_SCORE_TOPK, self.d, self.b, self.G, n,
+                                                  nq, k))
+        B.tq_score_topk(self.cb, _ptr(self.Pi), _ptr(self.S), self.G, n, _ptr(codes.codes),
+                        _ptr(codes.xnorm), _ptr(codes.rnorm), nq, _ptr(q), _dtype_code(q), k,
+                        _ptr(scores_out), _ptr(topk_out[0]), _ptr(topk_out[1]), wp, wn, _stream())
+        return scores_out, topk_out
+
     def decode(self, codes, out=None):
         n = codes.n
         if out is None:

@@ -69,6 +69,10 @@ def test_workspace_sizes(tq_lib):
     t = B.tq_workspace_bytes(B.TQ_OP_TOPK, 128, 4, 1, 10 ** 6, 1024, 10)
     assert t >= 1024 * ((10 ** 6 + 1023) // 1024) * 10 * 12
     assert B.tq_workspace_bytes(99, 128, 4, 1, 1, 1, 1) == big
+    # scores + top-k: the top-k workspace without room for the scores
+    st = B.tq_workspace_bytes(B.TQ_OP_SCORE_TOPK, 128, 4, 8, 32768, 4, 10)
+    tt = B.tq_workspace_bytes(B.TQ_OP_TOPK, 128, 4, 8, 32768, 4, 10)
+    assert 0 < st and st + 8 * 4 * 32768 * 4 <= tt
     # decode attention: d = 128 only, n >= 1; holds the logits [G][nq][n]
     a = B.tq_workspace_bytes(B.TQ_OP_ATTENTION, 128, 4, 8, 131072, 4, 0)
     assert a >= 8 * 4 * 131072 * 4 + s
@@ -103,6 +107,11 @@ def test_bad_arguments_rejected_without_device_work(tq_lib):
     assert lib.tq_decode(C.byref(cb), 1, 1, 1, 10, 1, 1, 1, 1, 1, 8, None) == B.TQ_ERR_WORKSPACE
     assert lib.tq_logits_fp32(96, 1, 10, 1, 1, 1, 0, 1, None) == B.TQ_ERR_UNSUPPORTED
     assert lib.tq_exact_topk(128, 1, 10, 1, 1, 1, 0, 20, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    # scores + top-k in one call: the score output is required
+    assert lib.tq_score_topk(C.byref(cb), 1, 1, 1, 100, 1, 1, 1, 4, 1, 0, 10, None, 1, 1, 1,
+                             1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_score_topk(C.byref(cb), 1, 1, 1, 100, 1, 1, 1, 4, 1, 0, 33, 1, 1, 1, 1,
+                             1 << 30, None) == B.TQ_ERR_ARG
     # merge of shard lists
     assert lib.tq_topk_merge(4, 2, 0, 1, 1, 1, 1, None) == B.TQ_ERR_ARG
     assert lib.tq_topk_merge(4, 2, 33, 1, 1, 1, 1, None) == B.TQ_ERR_ARG

@@ -631,3 +631,31 @@ def test_topk_merge_of_shards(quant, oparams, tq_lib, cuda, nshards, k):
         PT.compare_topk(_np(mv.reshape(wv.shape)[g]), _np(mi.reshape(wi.shape)[g]), s_ora, k,
                         np.linalg.norm(_f64(qs[g]), axis=1), float(xn.max()))
 
+
+# ---------------------------------------------------------------- scores and top-k in one call
+@pytest.mark.parametrize("d,b,G,n,nq", [(128, 4, 2, 5000, 4), (128, 4, 1, 3001, 16),
+                                        (256, 4, 1, 2000, 70), (128, 2, 1, 2_200_000, 8),
+                                        (128, 3, 3, 777, 1)])
+def test_score_topk_equals_separate_calls(quant, oparams, tq_lib, cuda, d, b, G, n, nq):
+    """tq_score_topk writes exactly tq_score's estimates and tq_topk's lists
+    (SIMT, tensor-core and decoded-key GEMM scoring; beyond 2^24 scores, where
+    tq_topk takes its fused path); the oracle checks one group."""
+    k = 10
+    W = b * d // 32
+    recs = [synth.random_records(n, W, seed=800 + g) for g in range(G)]
+    qs = synth.gaussian_rows(G * nq, d, seed=810, norm_range=None).reshape(G, nq, d)
+    tq = quant(d, b, 0, G)
+    codes = _records_on(tq_lib, cuda, recs)
+    s1 = tq.score(codes, qs.cuda())
+    v1, i1 = tq.topk(codes, qs.cuda(), k)
+    s2, (v2, i2) = tq.score_topk(codes, qs.cuda(), k)
+    torch.cuda.synchronize()
+    assert torch.equal(s1, s2)
+    assert torch.equal(i1, i2) and torch.equal(v1, v2)
+    if n <= 100_000:
+        c, xn, rn = recs[0]
+        s_ora = O.score(oparams(d, b, 0), c, xn, rn, _f64(qs[0]))
+        qn = np.linalg.norm(_f64(qs[0]), axis=1)
+        PT.compare_scores(_np(s2[0]), s_ora, qn, xn.astype(np.float64))
+        PT.compare_topk(_np(v2[0]), _np(i2[0]), s_ora, k, qn, float(xn.max()))
+
