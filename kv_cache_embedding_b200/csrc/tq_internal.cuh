@@ -122,6 +122,16 @@ int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_code
                const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,
                const float* u, float* scores, float* tmax, int64_t ntm, void* op_ws, int* d_err,
                cudaStream_t s);
+// Scoring of up to 16 queries per pass at d = 128 as exact int8 tensor-core
+// products (tq_score_i8.cu); inner-product records with b = 2..4 whose code
+// array is 16-byte aligned.  Same outputs as launch_score_tc.  With k0 and
+// n_stride (>= 0) it scores keys k0 .. k0 + n of arrays holding n_stride keys
+// per group, into scores [G][nq][n] (and maxima [G][nq][ceil(n / 128)]).
+bool score_i8_supported(const tq_codebook_t* cb, int G, int64_t n, int nq, const void* d_codes);
+int launch_score_i8(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
+                    const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,
+                    const float* u, float* d_scores, float* tmax, int* zero_cnt, int* d_err,
+                    cudaStream_t s, int64_t n_stride = -1, int64_t k0 = 0);
 bool score_tc_supported(int d, int b, int G, int64_t n, int nq);
 int launch_score_tc(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_codes,
                     const float* d_xnorm, const float* d_rnorm, int nq, const float* qr,

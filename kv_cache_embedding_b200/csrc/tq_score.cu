@@ -293,7 +293,7 @@ __global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict
                                                       int nchunks, int K, int* cand_cnt, int* done,
                                                       float* cand_v, int* cand_i,
                                                       float* __restrict__ vals,
-                                                      int64_t* __restrict__ ids) {
+                                                      int64_t* __restrict__ ids, int64_t id0) {
     __shared__ int s_last;
     const int64_t row = blockIdx.y;
     const int P = gridDim.x;
@@ -372,7 +372,7 @@ __global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict
     if (lane < K) {
         const bool have = L.id != id_none<int>();
         vals[row * K + lane] = have ? L.v : -INFINITY;
-        ids[row * K + lane] = have ? (int64_t)L.id : INT64_MAX;
+        ids[row * K + lane] = have ? id0 + (int64_t)L.id : INT64_MAX;
     }
 }
 
@@ -764,6 +764,9 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
         return score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr, 0,
                           op, err, s);
     }
+    if (score_i8_supported(cb, G, n, nq, d_codes))
+        return launch_score_i8(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
+                               nullptr, err, s);
     if (!is_mse(cb) && score_tc_supported(d, b, G, n, nq))
         return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
@@ -822,6 +825,10 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
             TQ_TRY_CUDA(cudaMemsetAsync(cnt, 0, (size_t)rows * 2 * 4, s));
             rc = score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, ntm, p, err, s);
             nchunks = (int)ntm;
+        } else if (score_i8_supported(cb, G, n, nq, d_codes)) {  // maxima per 128-key tile
+            rc = launch_score_i8(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt, err,
+                                 s);
+            nchunks = (int)ntm;
         } else if (tc) {  // maxima per 128-key tile
             rc = launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt, err,
                                  s);
@@ -848,9 +855,68 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         P = P > pmax ? pmax : P;
         dim3 grid((unsigned)P, (unsigned)rows);
         k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, n, nchunks, k, cnt, cnt + rows, cv, ci, d_vals,
-                                            d_ids);
+                                            d_ids, 0);
         TQ_CHECK_LAUNCH();
         return TQ_OK;
+    }
+    if (score_i8_supported(cb, G, n, nq, d_codes)) {
+        // too many scores to hold at once: the same integer tensor-core scores
+        // (so the lists equal tq_score_topk's) over chunks of keys sized to the
+        // workspace, each chunk's top-k, then the merge of the chunks' lists
+        const size_t avail = ws_bytes - (size_t)(p - (char*)d_ws);
+        int64_t nc = 0, nch = 0;
+        for (int64_t m = 1;; ++m) {
+            const int64_t c = ((n + m - 1) / m + 127) / 128 * 128;
+            const int64_t h = (n + c - 1) / c;
+            const size_t need = align256((size_t)rows * c * 4) + align256((size_t)rows * (c / 128) * 4) +
+                                align256((size_t)rows * 2 * 4) + 2 * align256((size_t)rows * kCandCapG * 4) +
+                                align256((size_t)h * rows * k * 4) + align256((size_t)h * rows * k * 8);
+            if (need <= avail) {
+                nc = c;
+                nch = h;
+                break;
+            }
+            if (c <= 128) break;
+        }
+        if (nc > 0) {
+            float* sc = (float*)p;
+            p += align256((size_t)rows * nc * 4);
+            float* cm = (float*)p;
+            p += align256((size_t)rows * (nc / 128) * 4);
+            int* cnt = (int*)p;
+            p += align256((size_t)rows * 2 * 4);
+            float* cv = (float*)p;
+            p += align256((size_t)rows * kCandCapG * 4);
+            int* ci = (int*)p;
+            p += align256((size_t)rows * kCandCapG * 4);
+            float* pv = (float*)p;
+            p += align256((size_t)nch * rows * k * 4);
+            int64_t* pi = (int64_t*)p;
+            int nsm = 0, dev = 0;
+            TQ_TRY_CUDA(cudaGetDevice(&dev));
+            TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+            for (int64_t h = 0; h < nch; ++h) {
+                const int64_t k0 = h * nc;
+                const int64_t len = (n - k0) < nc ? (n - k0) : nc;
+                rc = launch_score_i8(cb, G, len, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt,
+                                     err, s, n, k0);
+                if (rc) return rc;
+                int64_t P = (len + 256 * 16 - 1) / (256 * 16);
+                const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
+                const int64_t pmax = (len + 255) / 256;
+                P = P < pmin ? pmin : P;
+                P = P > pmax ? pmax : P;
+                dim3 grid((unsigned)P, (unsigned)rows);
+                k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, len, (int)((len + 127) / 128), k, cnt,
+                                                    cnt + rows, cv, ci, pv + h * rows * k,
+                                                    pi + h * rows * k, k0);
+                TQ_CHECK_LAUNCH();
+            }
+            k_topk_merge<<<(unsigned)((rows + 3) / 4), 128, 0, s>>>(pv, pi, rows, (int)nch, k, d_vals,
+                                                                     d_ids, k, rows * k);
+            TQ_CHECK_LAUNCH();
+            return TQ_OK;
+        }
     }
     // fused: per-range best-K lists [G][nq][nblk][K], then the merge
     float* pv = (float*)p;
