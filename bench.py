@@ -1,20 +1,29 @@
 """Benchmark of the TurboQuant hot path on B200: encode -> score -> top-k.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config kv|decode|tiny|search|larged]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
 One step = one pass of the whole path over one batch of synthetic input:
 tq_encode of every vector, then the estimates of the queries against all
-codes and their top-10 (one tq_score_topk call when a config has both, which
-transforms and scores the queries once; else tq_score or tq_topk alone).
-Default workload ("kv"): KV-cache keys
-bf16 [8 KV heads, 32768 tokens, 128], b = 4, with 4 decode query heads per KV
-head (GQA 4:1, 32 query heads).  Inputs sit in HBM before the timed region;
-L2 (126 MB) is flushed by writing a 256 MB buffer between timed steps.
+codes and their top-10 (one tq_score_topk call when a workload has both,
+which transforms and scores the queries once; else tq_topk alone).
 
-Multi-GPU (torchrun, one rank per GPU): weak scaling -- every rank encodes and
-scores its own independent batch (the vectors are independent problems, so
-there is no data-path collective); the time is the max over ranks.
+Without --config every workload runs in one process -- tiny, kv, decode,
+search, larged -- and ONE JSON line is printed.  Its headline (value,
+ms_per_step, roofline, cpu_baseline, e2e) is large-d (10^6 x 3072 fp32 rows,
+b = 4, 256 queries), the largest single-GPU workload; the others sit in its
+"configs" object, each with its own timing, roofline and cpu_baseline.  The
+headline times exactly --steps steps; every other workload repeats its step
+until its timed region lasts at least a second (so the clock sampler sees it).
+Inputs sit in HBM before a timed region; L2 (126 MB) is flushed by writing a
+256 MB buffer between timed steps.
+
+Multi-GPU: --gpus N > 1 starts N ranks itself (torchrun, one rank per GPU,
+NCCL) unless it already runs under torchrun.  Every workload but search is
+weak-scaled (each rank encodes and scores its own seeded batch; the vectors
+are independent problems, so no data-path collective).  The search is
+strong-scaled: one database of 10^6 rows sharded across the ranks, each
+rank's top-10 made global and merged after one all-gather
+(kv_cache_embedding_b200.sharded).  Times are the max over ranks.
 
 --impl reference times the plain CPU oracle on the host cores on a bounded
 sample of the same workload (rank 0 only).
@@ -23,6 +32,7 @@ import argparse
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -36,6 +46,8 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 METRIC = "tq_encode Mvec/s and tq_score scores/s over packed codes; HBM GB/s vs B200 peak"
+HEADLINE = "larged"
+ALL = ("tiny", "kv", "decode", "search", "larged")
 
 CONFIGS = {
     # name: G groups, n vectors/group, d, b, input kind, queries per group, k
@@ -50,21 +62,21 @@ CONFIGS = {
                    desc="decode attention logits, Llama-3.1-8B-shaped: 32 q heads / 8 KV heads, "
                         "head_dim 128, context 131072, bf16, b=4"),
     "tiny": dict(G=1, n=4096, d=128, b=4, x="rows", nq=64, q="gauss", k=10, score=True, topk=True,
-                 desc="tiny: 4096 x 128 fp32 rows (norms U[0.5,2]), 64 queries, b=4"),
+                 desc="4096 x 128 fp32 rows (norms U[0.5,2]), 64 queries, b=4"),
     "search": dict(G=1, n=1_000_000, d=1536, b=4, x="unit", nq=1024, q="unit", k=10, score=False,
-                   topk=True, desc="embedding search: 1e6 x 1536 fp32 unit rows, 1024 queries, "
+                   topk=True, desc="embedding search 1e6 x 1536 fp32 unit rows, 1024 queries, "
                                    "b=4, top-10"),
     "larged": dict(G=1, n=1_000_000, d=3072, b=4, x="rows", nq=256, q="gauss", k=10, score=True,
-                   topk=True, desc="large-d: 1e6 x 3072 fp32 rows (norms U[0.5,2]), 256 queries, "
+                   topk=True, desc="1e6 x 3072 fp32 rows (norms U[0.5,2]), 256 queries, "
                                    "b=4"),
 }
 
 FFMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FP32 CUDA-core peak at max SM clock
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# the dominant kernel, from one ncu capture of `python bench.py --steps 2
-# --warmup 3 --no-cpu-baseline --no-count` (summary under profiles/).  It is
-# reported only while the kernel's sources still hash to what was captured.
+# a workload's dominant kernel, from one ncu capture (summaries under
+# profiles/).  It is reported only while the kernel's sources still hash to
+# what was captured.
 NCU_TRAFFIC = {
     ("kv", "k_encode_tc"): {
         "sources": ["kv_cache_embedding_b200/csrc/tq_encode_tc.cu"],
@@ -97,7 +109,10 @@ def peaks():
 
 
 # ---------------------------------------------------------------- inputs
-def make_inputs(cfg, device, seed_offset=0, max_rows=None):
+def make_inputs(cfg, device, seed_offset=0, max_rows=None, rows=None):
+    """(x [G, n, d], q [G, nq, d]) of a workload.  rows = (start, stop) keeps
+    that slice of every group's rows (one shard of a database that is the same
+    whatever the number of shards)."""
     import synth
     G, n, d, nq = cfg["G"], cfg["n"], cfg["d"], cfg["nq"]
     if max_rows is not None and n > max_rows:
@@ -109,6 +124,8 @@ def make_inputs(cfg, device, seed_offset=0, max_rows=None):
         x = synth.gaussian_rows(G * n, d, seed=s, device=device, unit=True).reshape(G, n, d)
     else:
         x = synth.gaussian_rows(G * n, d, seed=s, device=device).reshape(G, n, d)
+    if rows is not None:
+        x = x[:, rows[0]:rows[1]].clone()
     if cfg["q"] == "kv":
         q = synth.kv_queries(G * nq, G, d, seed=s + 1, device=device, key_seed=s)
     elif cfg["q"] == "unit":
@@ -246,17 +263,32 @@ def job_throughput(units_per_rank, world, steps, total_ms):
     return units_per_rank * world * steps / (total_ms / 1e3) / 1e6
 
 
+def launch_ranks(args):
+    """Re-run this script as `--gpus` ranks under torchrun (rendezvous on
+    127.0.0.1); returns torchrun's exit status."""
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+           "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 # ---------------------------------------------------------------- our arm
 class Step:
-    """One pass of the hot path with preallocated outputs and workspaces."""
+    """One pass of the hot path with preallocated outputs and workspaces.
+    With `shard` = (n_total, group) the top-k runs over a database sharded
+    across ranks (local top-k, global ids, all-gather, merge)."""
 
-    def __init__(self, tq, cfg, x, q):
+    def __init__(self, tq, cfg, x, q, shard=None):
         import kv_cache_embedding_b200 as K
         self.K = K
         self.cfg = cfg
         self.tq = tq
         self.x, self.q = x, q
-        G, n, d, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["nq"], cfg["k"]
+        self.shard = shard
+        G, n, d, nq, k = cfg["G"], x.shape[1], cfg["d"], cfg["nq"], cfg["k"]
         dev = x.device
         self.codes = K.Codes(torch.empty(G, n, tq.words, dtype=torch.int32, device=dev),
                              torch.empty(G, n, dtype=torch.float32, device=dev),
@@ -272,7 +304,6 @@ class Step:
                    B.tq_workspace_bytes(B.TQ_OP_TOPK, d, cfg["b"], G, n, nq, k),
                    B.tq_workspace_bytes(B.TQ_OP_SCORE_TOPK, d, cfg["b"], G, n, nq, k))
         tq.ws.get(need)
-        self.ev = None
 
     def outputs(self):
         """Every result tensor of a step (what an end-to-end caller reads back)."""
@@ -305,7 +336,13 @@ class Step:
         if events:
             events[2].record()
         if self.topk is not None:
-            tq.topk(self.codes, self.q, self.cfg["k"], out=self.topk)
+            if self.shard is not None:
+                v, i = self.K.sharded.sharded_topk(tq, self.codes, self.q, self.cfg["k"],
+                                                   self.shard[0], self.shard[1])
+                self.topk[0].copy_(v)
+                self.topk[1].copy_(i)
+            else:
+                tq.topk(self.codes, self.q, self.cfg["k"], out=self.topk)
         if events:
             events[3].record()
 
@@ -326,103 +363,87 @@ def count_launches(step):
         return None, [f"profiler unavailable: {e}"]
 
 
-def alg_bytes_flops(cfg):
-    G, n, d, b, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
+def alg_bytes_flops(cfg, n=None):
+    G, d, b, nq, k = cfg["G"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
+    n = cfg["n"] if n is None else n
     esz = 2 if cfg["x"] == "kv" else 4
     rec = b * d // 8 + 8
     enc_bytes = G * n * (d * esz + rec)
     # two d x d products per vector (rotation, QJL projection); one for MSE-only
     enc_flops = (2.0 if cfg.get("variant", "prod") == "mse" else 4.0) * d * d * G * n
-    score_bytes = G * n * rec + G * nq * n * 4
+    score_bytes = G * n * rec + (G * nq * n * 4 if cfg["score"] else 0)
     score_flops = 4.0 * d * G * n * nq
-    topk_bytes = G * n * rec + G * nq * k * 12
     return dict(enc_bytes=enc_bytes, enc_flops=enc_flops, score_bytes=score_bytes,
-                score_flops=score_flops, topk_bytes=topk_bytes, rec=rec)
+                score_flops=score_flops, rec=rec, in_bytes=d * esz)
 
 
-def run_ours(args, cfg, rank, world, dist):
-    import kv_cache_embedding_b200 as K
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    x, q = make_inputs(cfg, dev, seed_offset=rank)
-    tq = K.TurboQuant(cfg["d"], cfg["b"], seed=0, groups=cfg["G"], device=dev,
-                      variant=cfg.get("variant", "prod"))
-    step = Step(tq, cfg, x, q)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    torch.cuda.synchronize()
+def encode_roofline(name, cfg, ab, enc_ms, pk, clocks):
+    """Roofline of the encode call, the dominant kernel of every workload's
+    step: achieved algorithmic FLOP/s (4 d^2 per vector, 2 d^2 for the
+    MSE-only variant) against the peak of the unit it runs on.  The 16-bit
+    tensor peak is the measured bf16 one (fp16 runs at the same rate): the
+    burst figure, or the sustained one when the timed region ran under the
+    power cap, divided by the mean number of 16-bit passes per product."""
+    ach = ab["enc_flops"] / (enc_ms / 1e3) / 1e12
+    mse = cfg.get("variant", "prod") == "mse"
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    bf16 = pk["bf16_sus"] if capped else pk["bf16"]
+    which = "sustained" if capped else "burst"
+    hbm = {"hbm_gbs": round(ab["enc_bytes"] / enc_ms / 1e6, 1),
+           "hbm_frac": round(ab["enc_bytes"] / enc_ms / 1e6 / pk["hbm"], 4),
+           "alg_bytes": ab["enc_bytes"]}
+    if cfg["d"] == 128 and cfg["x"] == "kv" and not mse:
+        peak = bf16 / 2.5
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "traffic": ncu_traffic(name, "k_encode_tc"),
+                "kernel": "k_encode_tc (tq_encode: rotation (2 fp16 passes) + QJL (3) on "
+                          "tcgen05, fused epilogue)",
+                "peak_source": f"measured bf16 {which} (MEASURED_PEAKS.json) / 2.5 passes "
+                               f"(fp16 = bf16 rate)" if pk["src"] == "measured" else
+                               f"fallback bf16 {which} / 2.5 passes",
+                "frac_of_3xtf32_fp32_equivalent": round(ach / (bf16 * 0.5 / 3.0), 4), **hbm}
+    # tensor-core GEMMs on fp16 pieces: the rotation takes 3 passes for fp32
+    # rows (2 x 2 pieces) and 2 for bf16 rows (one exact piece), the QJL 3
+    p_rot = 2 if cfg["x"] == "kv" else 3
+    passes = [p_rot] if mse else [p_rot, 3]
+    peak = bf16 * len(passes) / sum(passes)
+    return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+            "kernel": "k_gemm_tc (tq_encode: rotation and QJL as tcgen05 GEMMs on fp16 pieces) "
+                      "+ k_rownorm_split16 + k_quantize16 + k_pack",
+            "peak_source": (f"measured bf16 {which} (MEASURED_PEAKS.json)" if pk["src"] == "measured"
+                            else f"fallback bf16 {which}") +
+                           f" / {sum(passes) / len(passes):g} passes (mean over the products)",
+            **hbm}
 
-    nlaunch, kernel_names = count_launches(step) if not args.no_count else (None, [])
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    # The step as one CUDA graph (the same public calls, captured once): its
-    # replays are the timed steps.  Per-call times come from a second timed
-    # pass of plain stream launches.
-    graph = None
-    if not args.no_graph:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                step.run()
-            torch.cuda.synchronize()
-            for _ in range(args.warmup):
-                graph.replay()
-            torch.cuda.synchronize()
-        except Exception as e:  # capture unsupported: plain launches
-            print(f"graph capture failed ({e}); timing plain launches", file=sys.stderr)
-            graph = None
-            torch.cuda.synchronize()
-    sampler = ClockSampler(dev)
-    sampler.start()
-    sampler.wait_first()
-    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0 = time.time()
-    for i in range(args.steps):
+
+def time_steps(run, flush, steps):
+    """Device time (ms) of `steps` calls of run(), L2 flushed before each;
+    one event pair per call on the current stream."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
         flush.zero_()
-        if graph is not None:
-            gev[i][0].record()
-            graph.replay()
-            gev[i][1].record()
-        else:
-            step.run(evs[i])
+        a.record()
+        run()
+        b.record()
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    t1 = time.time()
-    if graph is not None:  # per-call breakdown, plain launches
-        for i in range(args.steps):
-            flush.zero_()
-            step.run(evs[i])
-        torch.cuda.synchronize()
-    time.sleep(0.3)
-    sampler.stop()
-    enc = [e[0].elapsed_time(e[1]) for e in evs]
-    sco = [e[1].elapsed_time(e[2]) for e in evs]
-    tpk = [e[2].elapsed_time(e[3]) for e in evs]
-    if graph is not None:
-        tot_ms = sum(e[0].elapsed_time(e[1]) for e in gev)
-    else:
-        tot_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
-    tot_ms, se, ss, st = rank_max(dist, [tot_ms, sum(enc), sum(sco), sum(tpk)], dev)
-    K_ = args.steps
-    ms_step = tot_ms / K_
-    units = cfg["G"] * cfg["n"] * world
-    value = job_throughput(cfg["G"] * cfg["n"], world, K_, tot_ms)
+    return [a.elapsed_time(b) for a, b in ev]
 
-    # e2e: every step copies its inputs from pinned host memory to the device,
-    # runs the same three public calls and copies every result back to pinned
-    # host memory.  Two buffer sets and one stream per copy direction let the
-    # copies of neighbouring steps overlap the compute (and each other).
+
+def e2e_time(tq, cfg, x, q, steps, dist, dev, shard):
+    """End-to-end step through the public API with host buffers: every step
+    copies its inputs from pinned host memory, runs the same calls and copies
+    every result back to pinned host memory.  Two buffer sets and one stream
+    per copy direction let the copies of neighbouring steps overlap the
+    compute.  Returns (ms per step, h2d bytes, d2h bytes)."""
     xh = x.cpu().pin_memory()
     qh = q.cpu().pin_memory()
     bufs = []
     for _ in range(2):
         xd, qd = torch.empty_like(x), torch.empty_like(q)
-        stp = Step(tq, cfg, xd, qd)
+        stp = Step(tq, cfg, xd, qd, shard)
         host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in stp.outputs()]
         bufs.append((xd, qd, stp, host))
     s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
@@ -430,7 +451,7 @@ def run_ours(args, cfg, rank, world, dist):
     ev_c = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_run(m):
+    def run(m):
         start = torch.cuda.Event()
         start.record()
         for s_ in (s_in, s_c, s_out):
@@ -459,80 +480,121 @@ def run_ours(args, cfg, rank, world, dist):
         for s_ in (s_in, s_c, s_out):
             cur.wait_stream(s_)
 
-    e2e_run(max(2, min(args.warmup, 3)))
+    run(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(2, min(args.steps, 20))
     if dist:
         dist.barrier()
     e0.record()
-    e2e_run(e2e_steps)
+    run(steps)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = rank_max(dist, [e0.elapsed_time(e1) / e2e_steps], dev)[0]
+    ms = rank_max(dist, [e0.elapsed_time(e1) / steps], dev)[0]
     h2d = xh.numel() * xh.element_size() + qh.numel() * qh.element_size()
     d2h = sum(t.numel() * t.element_size() for t in bufs[0][3])
+    return ms, h2d, d2h
 
-    ab = alg_bytes_flops(cfg)
-    pk = peaks()
-    enc_ms = se / K_
-    score_ms = ss / K_ if cfg["score"] else None
-    topk_ms = st / K_ if cfg["topk"] else None
-    # dominant kernel: the encode call.  For d = 128 bf16 keys it is one fused
-    # tcgen05 kernel: the rotation takes 2 fp16 passes (exact fp16 keys times
-    # two pieces of Pi), the QJL product 3, so its peak is the measured 16-bit
-    # peak / 2.5 (the mean pass count over the two equal-sized products).
-    ach = ab["enc_flops"] / (enc_ms / 1e3) / 1e12
-    mse = cfg.get("variant", "prod") == "mse"
-    tc = cfg["d"] == 128 and cfg["x"] == "kv" and not mse
-    if cfg["d"] >= 256:
-        # split-precision tcgen05 GEMMs: the rotation takes 3 16-bit passes for
-        # bf16 inputs (one exact piece) and 6 for fp32 inputs, the QJL product 6
-        p_rot = 3 if cfg["x"] == "kv" else 6
-        passes = [p_rot] if mse else [p_rot, 6]
-        peak = pk["bf16"] * len(passes) / sum(passes)
-        roofline = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
-                    "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
-                    "alg_bytes": ab["enc_bytes"],
-                    "kernel": "k_gemm_tc (tq_encode: rotation and QJL as split-bf16 tcgen05 "
-                              "GEMMs) + k_quantize + k_pack",
-                    "peak_source": f"measured bf16 burst (MEASURED_PEAKS.json) / "
-                                   f"{sum(passes) / len(passes):g} passes (mean over the products)",
-                    "hbm_gbs": round(ab["enc_bytes"] / enc_ms / 1e6, 1),
-                    "hbm_frac": round(ab["enc_bytes"] / enc_ms / 1e6 / pk["hbm"], 4)}
-    elif tc:
-        peak = pk["bf16"] / 2.5
-        roofline = {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
-                    "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                    "traffic": ncu_traffic(args.config, "k_encode_tc"),
-                    "alg_bytes": ab["enc_bytes"],
-                    "kernel": "k_encode_tc (tq_encode: rotation (2 fp16 passes) + QJL (3) on "
-                              "tcgen05, fused epilogue)",
-                    "peak_source": "measured bf16 burst (MEASURED_PEAKS.json) / 2.5 passes "
-                                   "(fp16 = bf16 rate)",
-                    "frac_of_3xtf32_fp32_equivalent": round(ach / (pk["bf16"] * 0.5 / 3.0), 4),
-                    "hbm_gbs": round(ab["enc_bytes"] / enc_ms / 1e6, 1),
-                    "hbm_frac": round(ab["enc_bytes"] / enc_ms / 1e6 / pk["hbm"], 4)}
+
+def bench_config(args, name, rank, world, dist, headline):
+    """Time one workload; returns its JSON object (the headline's carries the
+    top-level keys of the line)."""
+    import kv_cache_embedding_b200 as K
+    cfg = CONFIGS[name]
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    sharded = name == "search" and world > 1
+    if sharded:  # one database across the ranks (strong scaling)
+        span = K.sharded.shard_bounds(cfg["n"], world, rank)
+        x, q = make_inputs(cfg, dev, rows=span)
+        shard = (cfg["n"], None)
     else:
-        roofline = {"bound": "alu", "achieved": round(ach, 3), "peak": round(FFMA_PEAK_TFLOPS, 1),
-                    "unit": "TFLOP/s", "frac": round(ach / FFMA_PEAK_TFLOPS, 4), "traffic": None,
-                    "kernel": "tq_encode portable path (fp32 FFMA GEMMs)",
-                    "peak_source": "derived: 148 SM x 128 FP32 lanes x 2 x 1965 MHz"}
+        x, q = make_inputs(cfg, dev, seed_offset=rank)
+        shard = None
+    tq = K.TurboQuant(cfg["d"], cfg["b"], seed=0, groups=cfg["G"], device=dev,
+                      variant=cfg.get("variant", "prod"))
+    step = Step(tq, cfg, x, q, shard)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    nlaunch, kernel_names = count_launches(step) if not args.no_count else (None, [])
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    # The step as one CUDA graph (the same public calls, captured once): its
+    # replays are the timed steps.  Per-call times come from a second pass of
+    # plain stream launches.  The sharded search (an NCCL all-gather in the
+    # step) runs as plain launches.
+    graph = None
+    if not args.no_graph and not sharded:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step.run()
+            torch.cuda.synchronize()
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture unsupported: plain launches
+            print(f"graph capture failed ({e}); timing plain launches", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+    run = graph.replay if graph is not None else step.run
+    # steps: exactly --steps for the headline; else enough for >= 1 s of timed region
+    K_ = args.steps
+    if not headline:
+        est = statistics.median(time_steps(run, flush, 3))
+        K_ = max(args.steps, min(20000, int(math.ceil(1000.0 / max(est, 1e-3)))))
+        K_ = int(rank_max(dist, [K_], dev)[0])
+    sampler = ClockSampler(dev)
+    sampler.start()
+    sampler.wait_first()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    tot_ms = sum(time_steps(run, flush, K_))
+    if dist:
+        dist.barrier()
+    t1 = time.time()
+    time.sleep(0.3)
+    sampler.stop()
+    # per-call breakdown, plain launches
+    nb = min(K_, 50)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
+    for i in range(nb):
+        flush.zero_()
+        step.run(evs[i])
+    torch.cuda.synchronize()
+    enc = sum(e[0].elapsed_time(e[1]) for e in evs) / nb
+    sco = sum(e[1].elapsed_time(e[2]) for e in evs) / nb
+    tpk = sum(e[2].elapsed_time(e[3]) for e in evs) / nb
+    tot_ms, enc, sco, tpk = rank_max(dist, [tot_ms, enc, sco, tpk], dev)
+    ms_step = tot_ms / K_
+    n_rank = x.shape[1]
+    units = cfg["G"] * cfg["n"] if sharded else cfg["G"] * n_rank * world
+    value = units * K_ / (tot_ms / 1e3) / 1e6
+
+    e2e_steps = max(2, min(args.steps, 5 if cfg["d"] >= 256 else 20))
+    e2e_ms, h2d, d2h = e2e_time(tq, cfg, x, q, e2e_steps, dist, dev, shard)
+
+    ab = alg_bytes_flops(cfg, n_rank)
+    pk = peaks()
     out = {
         "metric": METRIC, "value": round(value, 4), "unit": "Mvec/s", "n_gpus": world,
         "steps": K_, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak",
+        "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded; shapes of the pages' KV-cache / embedding workloads)",
-        "config": {"workload": f"{args.config}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
+        "config": {"workload": f"{name}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
                    "d": cfg["d"], "b": cfg["b"], "queries_per_group": cfg["nq"], "k": cfg["k"],
                    "l2": "flushed (256 MB write) between timed steps",
                    "launch": "CUDA graph of the step" if graph is not None else "stream launches",
-                   "parallelism": f"dp{world} (independent batches per GPU)"},
-        "encode": {"ms": round(enc_ms, 5),
-                   "mvec_s": round(cfg["G"] * cfg["n"] / enc_ms / 1e3, 3),
-                   "gbs": round(ab["enc_bytes"] / enc_ms / 1e6, 2),
-                   "hbm_frac": round(ab["enc_bytes"] / enc_ms / 1e6 / pk["hbm"], 4)},
-        "roofline": roofline,
+                   "parallelism": (f"sharded database over {world} ranks (local top-k, all-gather, "
+                                   f"merge)") if sharded else
+                   f"dp{world} (independent batches per GPU)"},
+        "encode": {"ms": round(enc, 5), "mvec_s": round(cfg["G"] * n_rank / enc / 1e3, 3),
+                   "gbs": round(ab["enc_bytes"] / enc / 1e6, 2),
+                   "hbm_frac": round(ab["enc_bytes"] / enc / 1e6 / pk["hbm"], 4)},
+        "roofline": None,
         "e2e": {"value": round(units / e2e_ms / 1e3, 4), "unit": "Mvec/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
@@ -541,27 +603,72 @@ def run_ours(args, cfg, rank, world, dist):
         "kernels": kernel_names,
         "clocks": sampler.summary(t0, t1),
         "peaks": pk,
+        "compression": {"record_bytes": ab["rec"], "input_bytes": ab["in_bytes"],
+                        "vs_input": round(ab["in_bytes"] / ab["rec"], 3),
+                        "vs_fp32": round(cfg["d"] * 4 / ab["rec"], 3)},
     }
+    out["roofline"] = encode_roofline(name, cfg, ab, enc, pk, out["clocks"])
     if step.combined:
         # tq_score_topk: the score matrix and the top-k lists from one scoring pass
-        sg = ab["score_bytes"] / score_ms / 1e6
-        out["score_topk"] = {"ms": round(score_ms, 5),
-                             "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / score_ms * 1e3, 1),
+        sg = ab["score_bytes"] / sco / 1e6
+        out["score_topk"] = {"ms": round(sco, 5),
+                             "scores_s": round(cfg["G"] * cfg["nq"] * n_rank / sco * 1e3, 1),
                              "gbs": round(sg, 2), "hbm_frac": round(sg / pk["hbm"], 4),
                              "call": "tq_score_topk (scores written + top-k of the same pass)"}
-    else:
-        if score_ms is not None:
-            sg = ab["score_bytes"] / score_ms / 1e6
-            out["score"] = {"ms": round(score_ms, 5),
-                            "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / score_ms * 1e3, 1),
-                            "gbs": round(sg, 2), "hbm_frac": round(sg / pk["hbm"], 4)}
-        if topk_ms is not None:
-            out["topk"] = {"ms": round(topk_ms, 5),
-                           "scores_s": round(cfg["G"] * cfg["nq"] * cfg["n"] / topk_ms * 1e3, 1)}
-    if args.config == "decode" and rank == 0:
+    elif cfg["topk"]:
+        out["topk"] = {"ms": round(tpk, 5),
+                       "scores_s": round(cfg["G"] * cfg["nq"] * n_rank / tpk * 1e3, 1),
+                       "call": "tq_topk" + (" per shard + all-gather + tq_topk_merge"
+                                            if sharded else "")}
+    if name in ("kv", "decode") and rank == 0:
+        out["score_alone"] = score_alone_time(tq, cfg, step, flush, args, nq=cfg["nq"])
+    if name == "decode" and rank == 0:
+        out["score_1q_per_kv_head"] = score_alone_time(tq, cfg, step, flush, args, nq=1)
         out["fp32_baseline"] = fp32_baseline(cfg, x, q, flush, args)
         out["attention"] = attention_decode_time(cfg, x, q, flush, args)
+    if name == "search":
+        out["recall_at_10"] = search_recall(tq, step, x, q, cfg, shard)
+    del graph, step
     return out
+
+
+def score_alone_time(tq, cfg, step, flush, args, nq):
+    """tq_score alone (query transform + scoring of nq queries per group over
+    the step's codes), L2 flushed before each call; bytes = the records read
+    and the scores written."""
+    q = step.q[:, :nq].contiguous()
+    out = torch.empty(cfg["G"], nq, step.codes.n, dtype=torch.float32, device=q.device)
+    for _ in range(3):
+        tq.score(step.codes, q, out=out)
+    ts = time_steps(lambda: tq.score(step.codes, q, out=out), flush, max(10, min(args.steps, 50)))
+    ms = statistics.median(ts)
+    rec = cfg["b"] * cfg["d"] // 8 + 8
+    byts = cfg["G"] * step.codes.n * rec + out.numel() * 4
+    pk = peaks()
+    return {"ms": round(ms, 5), "queries_per_group": nq, "gbs": round(byts / ms / 1e6, 1),
+            "hbm_frac": round(byts / ms / 1e6 / pk["hbm"], 4),
+            "scores_s": round(out.numel() / ms * 1e3, 1), "call": "tq_score"}
+
+
+def search_recall(tq, step, x, q, cfg, shard):
+    """recall@10 of the step's top-10 (estimates from 4-bit codes) against the
+    exact fp32 top-10 of the same database (tq_exact_topk), over every query;
+    sharded databases merge the exact lists like the estimated ones."""
+    import kv_cache_embedding_b200 as K
+    k = cfg["k"]
+    step.run()
+    est = step.topk[1]
+    if shard is not None:
+        _, ex = K.sharded.sharded_topk(None, x, q, k, shard[0], shard[1],
+                                       local_topk=lambda xs, qq, kk: K.exact_topk(xs, qq, kk))
+    else:
+        _, ex = K.exact_topk(x, q, k)
+    torch.cuda.synchronize()
+    e = est.reshape(-1, k).cpu()
+    t = ex.reshape(-1, k).cpu()
+    hits = sum(len(set(a.tolist()) & set(b.tolist())) for a, b in zip(e, t))
+    return {"value": round(hits / (k * e.shape[0]), 5), "queries": int(e.shape[0]),
+            "truth": "tq_exact_topk (fp32 inner products of the unquantized rows)"}
 
 
 def attention_decode_time(cfg, x, q, flush, args):
@@ -578,15 +685,8 @@ def attention_decode_time(cfg, x, q, flush, args):
     out = tk.attention_decode(kc, tv, vc, q)
     for _ in range(3):
         tk.attention_decode(kc, tv, vc, q, out=out)
-    ts = []
-    for _ in range(max(3, min(args.steps, 50))):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        tk.attention_decode(kc, tv, vc, q, out=out)
-        b.record()
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
+    ts = time_steps(lambda: tk.attention_decode(kc, tv, vc, q, out=out), flush,
+                    max(3, min(args.steps, 50)))
     ms = sum(ts) / len(ts)
     byts = (kc.codes.numel() * 4 + kc.xnorm.numel() * 8 + vc.codes.numel() * 4 +
             vc.xnorm.numel() * 4 + q.numel() * q.element_size() + out.numel() * 4)
@@ -601,54 +701,22 @@ def fp32_baseline(cfg, x, q, flush, args):
     out = torch.empty(cfg["G"], cfg["nq"], cfg["n"], dtype=torch.float32, device=x.device)
     for _ in range(3):
         K.logits_fp32(keys, q, out)
-    ts = []
-    for _ in range(max(3, min(args.steps, 50))):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        K.logits_fp32(keys, q, out)
-        b.record()
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
+    ts = time_steps(lambda: K.logits_fp32(keys, q, out), flush, max(3, min(args.steps, 50)))
     ms = sum(ts) / len(ts)
     byts = keys.numel() * 4 + out.numel() * 4
     return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1)}
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_sample(cfg, target_s=10.0, max_units=None):
-    """Run the oracle's encode -> score -> top-k on a bounded sample of the
-    workload; returns (vectors, seconds, description)."""
-    import numpy as np
-    from oracle import oracle as O
-    G, n, d, b, nq, k = cfg["G"], cfg["n"], cfg["d"], cfg["b"], cfg["nq"], cfg["k"]
-    x, q = make_inputs(cfg, "cpu", max_rows=65536)
-    n = min(n, x.shape[1])
-    mse = cfg.get("variant", "prod") == "mse"
-    # one group's parameters (built outside the timing)
-    params = O.MseParams(d, b, 0) if mse else O.Params(d, b, 0)
-
-    def run(rows):
-        xs = x[0, :rows].to(torch.float64).numpy()
-        qs = q[0].to(torch.float64).numpy()
-        t = time.perf_counter()
-        if mse:
-            codes, xn, rn = O.mse_encode(params, xs)
-            s = O.mse_score(params, codes, xn, qs)
-        else:
-            codes, xn, rn = O.encode(params, xs)
-            s = O.score(params, codes, xn, rn, qs)
-        O.topk(s, min(k, rows))
-        return time.perf_counter() - t
-
-    rows = min(n, 256)
-    dt = run(rows)
-    cap = max_units or n
-    while dt < target_s / 4 and rows < min(n, cap):
-        rows = min(n, cap, rows * 4)
-        dt = run(rows)
-    return rows, dt, (f"{rows} of the {G * n} vectors (group 0), oracle encode + score of "
-                      f"{nq} queries + top-{k}, extrapolated per vector")
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def cpu_cores():
@@ -658,25 +726,119 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def run_reference(args, cfg):
-    steps = []
+def omp_threads(n):
+    """Set the OpenMP thread count of the oracle library (libgomp); returns
+    False when that runtime cannot be reached."""
+    import ctypes
+    try:
+        ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+        return True
+    except OSError:
+        return False
+
+
+class OracleSample:
+    """The oracle's encode -> score -> top-k on a bounded sample of a
+    workload: the first rows of group 0, with one group's parameters built
+    once (outside the timing)."""
+
+    def __init__(self, cfg):
+        from oracle import oracle as O
+        self.O = O
+        self.cfg = cfg
+        x, q = make_inputs(cfg, "cpu", max_rows=65536)
+        self.x = x[0].to(torch.float64).numpy()
+        self.q = q[0].to(torch.float64).numpy()
+        self.mse = cfg.get("variant", "prod") == "mse"
+        d, b = cfg["d"], cfg["b"]
+        self.params = O.MseParams(d, b, 0) if self.mse else O.Params(d, b, 0)
+
+    def run(self, rows):
+        O, P = self.O, self.params
+        xs = self.x[:rows]
+        t = time.perf_counter()
+        if self.mse:
+            codes, xn, rn = O.mse_encode(P, xs)
+            s = O.mse_score(P, codes, xn, self.q)
+        else:
+            codes, xn, rn = O.encode(P, xs)
+            s = O.score(P, codes, xn, rn, self.q)
+        O.topk(s, min(self.cfg["k"], rows))
+        return time.perf_counter() - t
+
+    def sized(self, target_s):
+        """(rows, seconds) of a sample grown by 4x until it takes target_s / 4."""
+        n = self.x.shape[0]
+        rows = min(n, 256)
+        dt = self.run(rows)
+        while dt < target_s / 4 and rows < n:
+            rows = min(n, rows * 4)
+            dt = self.run(rows)
+        return rows, dt
+
+    def describe(self, rows):
+        c = self.cfg
+        return (f"{rows} of the {c['G'] * c['n']} vectors (group 0), oracle encode + score of "
+                f"{c['nq']} queries + top-{c['k']}, extrapolated per vector")
+
+    def flagged_rate(self, rows=None):
+        """Fraction of coordinates whose fp64 rotated value lies within 1e-5 sigma
+        of a Lloyd-Max boundary (the codes the parity rules exempt)."""
+        import numpy as np
+        rows = rows or (2048 if self.cfg["d"] <= 128 else 256)
+        if self.mse:
+            _, _, _, y, _ = self.O.mse_encode(self.params, self.x[:rows], diagnostics=True)
+        else:
+            _, _, _, y, _, _ = self.O.encode(self.params, self.x[:rows], diagnostics=True)
+        beta = np.asarray(self.params.beta, dtype=np.float64)
+        if beta.size == 0:
+            return {"value": 0.0, "coordinates": int(y.size)}
+        band = 1e-5 / math.sqrt(self.cfg["d"])
+        near = np.zeros(y.shape, dtype=bool)
+        for bj in beta:
+            near |= np.abs(y - bj) < band
+        return {"value": float(near.mean()), "coordinates": int(y.size),
+                "band": "1e-5 sigma, sigma = 1/sqrt(d)", "rows": int(y.shape[0])}
+
+
+def cpu_baseline(cfg, target_s):
+    """The oracle timed on the host cores (all of them, then one), for a
+    workload's line."""
+    o = OracleSample(cfg)
+    rows, dt = o.sized(target_s)
+    cores = int(os.environ.get("OMP_NUM_THREADS", cpu_cores()))
+    out = {"value": rows / dt / 1e6, "unit": "Mvec/s", "cores": cores, "kind": "oracle",
+           "sample": o.describe(rows), "cpu_model": cpu_model()}
+    if omp_threads(1):
+        r1 = max(16, rows // 16)
+        t1 = o.run(r1)
+        omp_threads(cores)
+        out["one_core"] = {"value": r1 / t1 / 1e6, "unit": "Mvec/s",
+                           "sample": f"{r1} vectors, OpenMP limited to 1 thread"}
+    out["flagged_coordinate_rate"] = o.flagged_rate()
+    return out
+
+
+def run_reference(args, cfg, name):
+    o = OracleSample(cfg)
+    rows, _ = o.sized(max(0.5, 60.0 / max(args.steps + args.warmup, 1)))
+    times = []
     for i in range(args.warmup + args.steps):
-        rows, dt, desc = oracle_sample(cfg, target_s=max(0.5, 8.0 / max(args.steps, 1)))
+        dt = o.run(rows)
         if i >= args.warmup:
-            steps.append((rows, dt))
-    rows = sum(r for r, _ in steps)
-    secs = sum(t for _, t in steps)
-    value = rows / secs / 1e6
+            times.append(dt)
+    secs = sum(times)
+    value = rows * len(times) / secs / 1e6
     cores = int(os.environ.get("OMP_NUM_THREADS", cpu_cores()))
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "Mvec/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": secs / len(steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": secs / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.config}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
+        "config": {"workload": f"{name}: {cfg['desc']}", "G": cfg["G"], "n": cfg["n"],
                    "d": cfg["d"], "b": cfg["b"]},
         "cpu_baseline": {"value": value, "unit": "Mvec/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": o.describe(rows), "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "Mvec/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -685,9 +847,10 @@ def run_reference(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="kv", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default=None, choices=sorted(CONFIGS),
+                    help="one workload only (default: all of them, large-d as the headline)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
@@ -697,13 +860,16 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    cfg = CONFIGS[args.config]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    names = (args.config,) if args.config else ALL
+    head = args.config or HEADLINE
     if args.impl == "reference":
         if rank != 0:
             return 0
-        print(json.dumps(run_reference(args, cfg)))
+        print(json.dumps(run_reference(args, CONFIGS[head], head)))
         return 0
 
     dist = None
@@ -712,14 +878,22 @@ def main():
 
         import torch.distributed as td
         torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        td.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         dist = td
-    out = run_ours(args, cfg, rank, world, dist)
+    results = {}
+    for name in names:
+        results[name] = bench_config(args, name, rank, world, dist, headline=(name == head))
+        torch.cuda.empty_cache()
+    out = results[head]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows, dt, desc = oracle_sample(cfg, target_s=10.0)
-        out["cpu_baseline"] = {"value": rows / dt / 1e6, "unit": "Mvec/s",
-                               "cores": int(os.environ.get("OMP_NUM_THREADS", cpu_cores())),
-                               "kind": "oracle", "sample": desc}
+        for name in names:
+            results[name]["cpu_baseline"] = cpu_baseline(CONFIGS[name],
+                                                         10.0 if name == head else 4.0)
+    if len(names) > 1:
+        out["configs"] = {nm: {k: v for k, v in r.items()
+                               if k not in ("metric", "higher_is_better", "vs_baseline", "data",
+                                            "peaks", "unit", "n_gpus", "warmup")}
+                          for nm, r in results.items() if nm != head}
     if rank == 0:
         print(json.dumps(out))
     if dist:

@@ -6,15 +6,26 @@
 // matrix); seeallochnaya #3476 steps 1-2 (rotate; round every coordinate on
 // the precomputed grid; residual -> random matrix -> sign).
 //
-// Portable path (any supported d; the only path of the MSE-only variant): per
-// group and row chunk
-//   k_rownorm      |x| in fp64 accumulation                       (E1)
-//   GEMM           Y = X Pi^T / |x|                                (E2)
-//   k_quantize     idx = #{beta_j <= y}, r = y - c[idx], |r|       (E3, E4)
-//   GEMM           P = R S^T                                       (E5)
-//   k_pack         fields idx | z -> code words                    (E3, E6)
-// The GEMMs run on the tensor cores (split bf16 pieces, tq_gemm_tc.cu) for
-// d >= 256, else as fp32 SIMT GEMMs (tq_gemm.cu).
+// General path (every d, fp32 rows, the MSE-only variant; bf16 keys at d = 128
+// take the fused kernel of tq_encode_tc.cu): per group and row chunk
+//   k_rownorm_split16   |x| in fp64 accumulation; fp16 pieces of 2^e x    (E1)
+//   GEMM                Y = X Pi^T / |x| on the tensor cores              (E2)
+//   k_quantize16        idx = #{beta_j <= y}, r = y - c[idx], |r|,
+//                       fp16 pieces of 2^s r                              (E3, E4)
+//   GEMM                P = R S^T on the tensor cores                     (E5)
+//   k_pack              fields idx | z -> code words                      (E3, E6)
+// The GEMMs (tq_gemm_tc.cu) take two fp16 pieces of each fp32 operand, every
+// operand scaled by a power of two into fp16's range: rows of x so that
+// |x| 2^e is in [2^10, 2^11) (then |2^e x_i| <= 2^11), Pi by 2^8 (its
+// entries are ~ 1/sqrt(d); the scale keeps the low pieces normal), S by 2^4,
+// r by 2^s with 2^s ~ 64 sqrt(d) (|r_i| <= 1.2 for |y| = 1).  The three
+// products hi*hi + hi*lo + lo*hi leave ~2^-22 of each term: ~5e-7 sigma on a
+// rotated coordinate and ~5e-7 |r| on a projection, far inside the 1e-5
+// bands of the code parity.  The scales are exact and cancel: Y is divided by
+// |x| 2^(e + 8); P only gives its signs.  Without the tensor-map encoder the
+// products run as fp32 SIMT GEMMs (tq_gemm.cu) on the unsplit rows.
+#include <cuda_fp16.h>
+
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -35,6 +46,82 @@ __global__ void k_rownorm(const T* __restrict__ x, int64_t rows, int d,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) xnorm[row] = (float)sqrt(acc);
+}
+
+// One warp per row: |x| (fp64 accumulation), the row scale |x| 2^(e + 8) of the
+// rotation's output (2^8: the scale of Pi's pieces), and the fp16 pieces of
+// 2^e x with |x| 2^e in [2^10, 2^11) -- hi to out[0], lo to out[1] (fp32 rows
+// only: a bf16 row scaled by 2^e is one exact fp16 piece).  x = 0 gives zero
+// pieces and scale 0 (the GEMM then writes y = 0).
+template <typename T>
+__global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
+                                  float* __restrict__ xnorm, float* __restrict__ rs,
+                                  __half* __restrict__ out) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const T* xr = x + row * d;
+    double acc = 0.0;
+    for (int i = lane; i < d; i += 32) {
+        const double v = (double)load_f32(xr, i);
+        acc = fma(v, v, acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const double nrm = sqrt(acc);
+    const float nf = (float)nrm;
+    int E = 0;
+    if (nf > 0.f) frexp((double)nf, &E);  // nf = m 2^E, m in [0.5, 1)
+    const int e = nf > 0.f ? 11 - E : 0;
+    const double sc = ldexp(1.0, e);      // exact; 2^e may exceed fp32's range
+    if (lane == 0) {
+        xnorm[row] = nf;
+        rs[row] = (float)ldexp((double)nf, e + 8);  // in [2^18, 2^19), or 0
+    }
+    __half* hi = out + row * d;
+    __half* lo = out + rows * d + row * d;
+    for (int i = lane; i < d; i += 32) {
+        const float v = (float)((double)load_f32(xr, i) * sc);  // exact, |v| <= 2^11
+        const __half h = __float2half_rn(v);
+        hi[i] = h;
+        if (sizeof(T) == 4) lo[i] = __float2half_rn(v - __half2float(h));
+    }
+}
+
+// One warp per row: bucketize each rotated coordinate, the cell index to a byte
+// array, |r|, and the fp16 pieces of rscale * r (r = y - c[idx]) -- hi to
+// rp[0], lo to rp[1] -- as the operand of the QJL product.
+__global__ void k_quantize16(const float* __restrict__ yr, uint8_t* __restrict__ idx, int64_t rows,
+                             int d, KCodebook cb, float rscale, float* __restrict__ rnorm,
+                             __half* __restrict__ rp) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const float* y = yr + row * d;
+    uint8_t* ix = idx + row * d;
+    __half* hi = rp + row * d;
+    __half* lo = rp + rows * d + row * d;
+    float rr = 0.f;
+    for (int i = lane; i < d; i += 32) {
+        const float v = y[i];
+        int cell = 0;
+        float r = v;
+        if (cb.levels > 0) {
+#pragma unroll
+            for (int j = 0; j < 15; ++j)
+                if (j + 1 < cb.levels && cb.beta[j] <= v) ++cell;
+            r = v - cb.c[cell];
+        }
+        ix[i] = (uint8_t)cell;
+        rr = fmaf(r, r, rr);
+        const float t = r * rscale;  // exact: a power of two
+        const __half h = __float2half_rn(t);
+        hi[i] = h;
+        lo[i] = __float2half_rn(t - __half2float(h));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);
+    if (lane == 0) rnorm[row] = sqrtf(rr);
 }
 
 // One warp per row: bucketize each rotated coordinate, write the residual over
@@ -140,16 +227,22 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     const size_t esz = (x_dtype == TQ_F32) ? 4 : 2;
     const size_t dd = (size_t)d * d;
     // tensor-core GEMMs: bf16 pieces of Pi_g, S_g and of the chunk's operand
-    const bool tcg = encode_gemm_tc(d) && gemm_tc_supported(d, d);
-    __nv_bfloat16* PiP = (__nv_bfloat16*)(IX + align256((size_t)chunk * d));
-    __nv_bfloat16* SP = (__nv_bfloat16*)((char*)PiP + align256(3 * dd * 2));
-    __nv_bfloat16* AP = (__nv_bfloat16*)((char*)SP + align256(3 * dd * 2));
+    const bool tcg = gemm_tc_supported(d, d);
+    // tensor-core GEMMs: fp16 pieces [2][d][d] of 2^8 Pi_g and of 2^4 S_g, the
+    // chunk's operand pieces [2][chunk][d] (x, then r) and its row scales
+    __half* PiP = (__half*)(IX + align256((size_t)chunk * d));
+    __half* SP = (__half*)((char*)PiP + align256(3 * dd * 2));
+    __half* AP = (__half*)((char*)SP + align256(3 * dd * 2));
+    float* RS = (float*)((char*)AP + align256((size_t)2 * chunk * d * 2));
+    int sr = 6;  // 2^sr ~ 64 sqrt(d)
+    while ((1 << (2 * (sr - 6))) < d) ++sr;
+    const float rscale = ldexpf(1.f, sr);
     for (int g = 0; g < G; ++g) {
         if (tcg) {
-            int rc = split_bf16x3(d_Pi + g * dd, (int64_t)dd, PiP, s);
+            int rc = split_f16x2(d_Pi + g * dd, (int64_t)dd, 256.f, PiP, s);
             if (rc) return rc;
             if (!mse) {
-                rc = split_bf16x3(d_S + g * dd, (int64_t)dd, SP, s);
+                rc = split_f16x2(d_S + g * dd, (int64_t)dd, 16.f, SP, s);
                 if (rc) return rc;
             }
         }
@@ -160,32 +253,33 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
             float* xn = d_xnorm + off;
             float* rn = d_rnorm + off;
             const unsigned wblocks = (unsigned)((rows + 7) / 8);
-            if (x_dtype == TQ_F32)
-                k_rownorm<float><<<wblocks, 256, 0, s>>>((const float*)xg, rows, d, xn);
-            else
-                k_rownorm<__nv_bfloat16><<<wblocks, 256, 0, s>>>((const __nv_bfloat16*)xg, rows,
-                                                                 d, xn);
-            TQ_CHECK_LAUNCH();
             int rc;
-            if (tcg) {  // Y = X Pi^T / |x| on the tensor cores
-                const __nv_bfloat16* A = (const __nv_bfloat16*)xg;  // bf16 keys: one exact piece
-                int pa = 1;
-                if (x_dtype == TQ_F32) {
-                    rc = split_bf16x3((const float*)xg, rows * d, AP, s);
-                    if (rc) return rc;
-                    A = AP;
-                    pa = 3;
-                }
-                rc = launch_gemm_tc((int)rows, d, d, A, pa, PiP, Y, d, xn, 1, err, s);
+            if (tcg) {  // Y = X Pi^T / |x| on the tensor cores (fp16 pieces)
+                if (x_dtype == TQ_F32)
+                    k_rownorm_split16<float><<<wblocks, 256, 0, s>>>((const float*)xg, rows, d, xn,
+                                                                     RS, AP);
+                else
+                    k_rownorm_split16<__nv_bfloat16><<<wblocks, 256, 0, s>>>(
+                        (const __nv_bfloat16*)xg, rows, d, xn, RS, AP);
+                TQ_CHECK_LAUNCH();
+                rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP,
+                                    x_dtype == TQ_F32 ? 2 : 1, (const __nv_bfloat16*)PiP, Y, d, RS,
+                                    1, err, s, 2, false, 0, nullptr, 0, true);
             } else {
+                if (x_dtype == TQ_F32)
+                    k_rownorm<float><<<wblocks, 256, 0, s>>>((const float*)xg, rows, d, xn);
+                else
+                    k_rownorm<__nv_bfloat16><<<wblocks, 256, 0, s>>>((const __nv_bfloat16*)xg,
+                                                                     rows, d, xn);
+                TQ_CHECK_LAUNCH();
                 rc = launch_sgemm((int)rows, d, d, xg, x_dtype, d, d_Pi + g * dd, true, d, Y, d,
                                   xn, 1, s);
             }
             if (rc) return rc;
-            k_quantize<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rn);
-            TQ_CHECK_LAUNCH();
             uint32_t* cg = d_codes + (size_t)off * W;
             if (mse) {  // no QJL projection
+                k_quantize<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rn);
+                TQ_CHECK_LAUNCH();
                 switch (b) {
                     case 1: k_pack<1, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
                     case 2: k_pack<2, true><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
@@ -195,11 +289,15 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                 TQ_CHECK_LAUNCH();
                 continue;
             }
-            if (tcg) {  // P = R S^T on the tensor cores
-                rc = split_bf16x3(Y, rows * d, AP, s);
-                if (rc) return rc;
-                rc = launch_gemm_tc((int)rows, d, d, AP, 3, SP, P, d, nullptr, 0, err, s);
+            if (tcg) {  // P = (2^sr R)(2^4 S)^T on the tensor cores: only its signs are kept
+                k_quantize16<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rscale, rn, AP);
+                TQ_CHECK_LAUNCH();
+                rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP, 2,
+                                    (const __nv_bfloat16*)SP, P, d, nullptr, 0, err, s, 2, false,
+                                    0, nullptr, 0, true);
             } else {
+                k_quantize<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rn);
+                TQ_CHECK_LAUNCH();
                 rc = launch_sgemm((int)rows, d, d, Y, TQ_F32, d, d_S + g * dd, true, d, P, d,
                                   nullptr, 0, s);
             }

@@ -14,12 +14,15 @@
 // multiply the residual by a random matrix, keep the sign); RecSysChannel #256
 // caveat 1 (normalise, multiply by a random matrix).
 //
-// Precision: both operands are split into bf16 pieces, A = a1 + a2 + a3 (one
-// piece when A is bf16 already) and B = b1 + b2 + b3 (each to ~2^-24 of the
-// value); the MMAs sum the products a_i b_j with i + j < max(pa, pb) (pa, pb
-// pieces of A and B: 3 x 3 -> a1 b1 + a1 b2 + a2 b1 + a1 b3 + a2 b2 + a3 b1;
-// 1 x 3 -> a1 b1 + a1 b2 + a1 b3; 2 x 2 -> a1 b1 + a1 b2 + a2 b1, ~2^-16);
-// bf16 x bf16 products are exact in fp32.  The accumulator in tensor memory is
+// Precision: both operands are split into 16-bit pieces and the MMAs sum the
+// products a_i b_j with i + j < max(pa, pb) (pa, pb pieces of A and B); 16-bit
+// x 16-bit products are exact in fp32.
+//  * fp16 pieces (the encode path): each operand scaled by a power of two into
+//    fp16's range, A = a1 + a2 and B = b1 + b2 (~2^-22 of the value; a bf16
+//    input scaled this way is one exact fp16 piece): 2 x 2 -> a1 b1 + a1 b2 +
+//    a2 b1 (3 passes), 1 x 2 -> a1 b1 + a1 b2 (2 passes).
+//  * bf16 pieces (the decoded-key scoring): 2 x 2 -> a1 b1 + a1 b2 + a2 b1
+//    (~2^-16); 3 x 3 pieces (~2^-24) -> 6 products.  The accumulator in tensor memory is
 // restarted every 128 of K and the chunk sums are added in fp32 registers,
 // so the rounding of an output stays near that of a 128-term fp32 sum for
 // any K, as in the SIMT path.
@@ -32,6 +35,7 @@
 // (1 s); a warp that gives up sets the abort flag and the status word.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -51,7 +55,6 @@ constexpr int kThreads = 32 * 6;
 constexpr int kThreadsDecode = 32 * 8;                // + 2 warps decoding A from records
 constexpr uint32_t kTmemCols = 2 * kTN;               // two chunk accumulators
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr uint32_t kIdesc = idesc_f16(1, kTM, kTN);   // bf16 x bf16 -> f32, K-major A and B
 
 struct SmemG {
     // stage s holds pieces [s (pa + pb), (s + 1)(pa + pb)): A's pa, then B's pb
@@ -240,7 +243,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
           int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
           const float* __restrict__ row_scale, int scale_mode, int transposed, int n_store,
           float* __restrict__ tmax, int64_t ldt, int* __restrict__ err, KeyDecode kd,
-          int decode) {
+          int decode, uint32_t idesc) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     SmemG& sm = *reinterpret_cast<SmemG*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -364,7 +367,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
 #pragma unroll
                         for (int ks = 0; ks < kKB / 16; ++ks)
                             mma_f16_ss(d, smem_desc_kmajor_sw128(as + ks * 32),
-                                   smem_desc_kmajor_sw128(bs + ks * 32), kIdesc,
+                                   smem_desc_kmajor_sw128(bs + ks * 32), idesc,
                                    (h | q | ks) != 0);
                     }
                     tc_commit(&sm.empty[s]);
@@ -496,6 +499,18 @@ __global__ void k_split3(const float* __restrict__ x, int64_t count, __nv_bfloat
     out[2 * count + i] = p3;
 }
 
+// out[p][i]: the fp16 pieces of scale * x (scale a power of two, so the
+// product is exact): out[0] + out[1] = scale * x to ~2^-22 of its magnitude.
+__global__ void k_split2h(const float* __restrict__ x, int64_t count, float scale,
+                          __half* __restrict__ out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= count) return;
+    const float v = x[i] * scale;
+    const __half p1 = __float2half_rn(v);
+    out[i] = p1;
+    out[count + i] = __float2half_rn(v - __half2float(p1));
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -543,10 +558,17 @@ int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t
     return TQ_OK;
 }
 
+int split_f16x2(const float* x, int64_t count, float scale, __half* out, cudaStream_t s) {
+    if (count <= 0) return TQ_OK;
+    k_split2h<<<(unsigned)((count + 255) / 256), 256, 0, s>>>(x, count, scale, out);
+    TQ_CHECK_LAUNCH();
+    return TQ_OK;
+}
+
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb, bool transposed, int n_store, float* tmax,
-                   int64_t ldt) {
+                   int64_t ldt, bool fp16) {
     if (M <= 0) return TQ_OK;
     if (!gemm_tc_supported(N, K) || pa < 1 || pa > 3 || pb < 1 || pb > 3) return TQ_ERR_ARG;
     if (!transposed && ldc % 4) return TQ_ERR_ARG;
@@ -561,7 +583,8 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
                                      (int)kSmemBytes));
     k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
                                                   scale_mode, transposed ? 1 : 0, n_store, tmax,
-                                                  ldt, d_err, KeyDecode{}, 0);
+                                                  ldt, d_err, KeyDecode{}, 0,
+                                                  idesc_f16(fp16 ? 0u : 1u, kTM, kTN));
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -583,7 +606,8 @@ int launch_gemm_tc_decoded(int M, int N, const KeyDecode& kd, const __nv_bfloat1
                                      (int)kSmemBytes));
     // the A map is unused in this mode: the B map stands in for the parameter
     k_gemm_tc<<<nctas, kThreadsDecode, kSmemBytes, s>>>(mb, mb, M, N, K, 2, 2, C, ldc, row_scale,
-                                                        2, 1, n_store, tmax, ldt, d_err, kd, 1);
+                                                        2, 1, n_store, tmax, ldt, d_err, kd, 1,
+                                                        idesc_f16(1u, kTM, kTN));
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }

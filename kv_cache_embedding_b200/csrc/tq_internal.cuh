@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -87,15 +88,18 @@ int check_common(const tq_codebook_t* cb, int G, int64_t n, int nq, int q_dtype)
 // Decode attention (tq_attention.cu): workspace of tq_attention_decode.
 size_t attn_workspace_bytes(int b, int G, int64_t n, int nq);
 bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n);
-// Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from bf16
-// pieces of A ([pa][M][K], pa = 1 or 3) and B ([3][N][K]); d_err as the
-// encode kernels' status word.
+// Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from
+// 16-bit pieces of A ([pa][M][K]) and B ([pb][N][K]) -- bf16, or fp16 with
+// `fp16` (the pointers then address __half data); d_err as the encode
+// kernels' status word.
 bool gemm_tc_supported(int N, int K);
 int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t s);
+// fp16 pieces [2][count] of scale * x (scale a power of two).
+int split_f16x2(const float* x, int64_t count, float scale, __half* out, cudaStream_t s);
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb = 3, bool transposed = false, int n_store = 0,
-                   float* tmax = nullptr, int64_t ldt = 0);
+                   float* tmax = nullptr, int64_t ldt = 0, bool fp16 = false);
 // A operand decoded from code records inside the GEMM (scoring of many
 // queries): row m of A = (c[idx] | kappa_m (2z - 1)) over K = 2d as bf16
 // pieces hi, lo (kappa_m = kscale |r_m|; the MSE-only variant has c[cell] and
@@ -111,8 +115,9 @@ struct KeyDecode {
 int launch_gemm_tc_decoded(int M, int N, const KeyDecode& kd, const __nv_bfloat16* B, float* C,
                            int64_t ldc, const float* row_scale, int* d_err, cudaStream_t s,
                            int n_store, float* tmax, int64_t ldt);
-// The encode path's dense products run on the tensor-core GEMM for d >= 256.
-inline bool encode_gemm_tc(int d) { return d >= 256; }
+// The general encode path's dense products run on the tensor-core GEMM (fp16
+// pieces) at every d; its workspace holds their operands.
+inline bool encode_gemm_tc(int d) { return d >= kMinD; }
 // Scoring of many queries at d >= 256 as a GEMM over decoded keys
 // (tq_score_gemm.cu): scores [G][nq][n] (and per-128-key maxima [G][nq][ntm]).
 constexpr int kScoreGemmMinQueries = 64;

@@ -43,15 +43,22 @@ def merge_lists(gvals, gids, k):
     return out_v, out_i
 
 
-def sharded_topk(tq, codes, q, k, n_total, group=None):
+def sharded_topk(tq, codes, q, k, n_total, group=None, local_topk=None, merge=None):
     """Top-k over a database of n_total records of which this rank holds its
     shard_bounds() slice as `codes` (a Codes of [G, n_shard, ...]); q is the
     same [G, nq, d] on every rank.  Returns the global (vals, ids) [G, nq, k]
-    on every rank."""
+    on every rank.
+
+    local_topk(codes, q, k) -> (vals, ids) and merge(gvals, gids, k) -> (vals,
+    ids) default to tq.topk and merge_lists (libtq); a caller may pass other
+    implementations of the same contract (the CPU tests pass the oracle's)."""
     world, rank = dist.get_world_size(group), dist.get_rank(group)
     start, _ = shard_bounds(n_total, world, rank)
-    vals, ids = tq.topk(codes, q, k)
-    ids = ids + start
+    local_topk = local_topk or tq.topk
+    merge = merge or merge_lists
+    vals, ids = local_topk(codes, q, k)
+    # missing entries (a shard with fewer than k records) keep their marker
+    ids = torch.where(ids == torch.iinfo(torch.int64).max, ids, ids + start)
     gv, gi = gather_lists(vals, ids, group)
-    mv, mi = merge_lists(gv, gi, k)
+    mv, mi = merge(gv, gi, k)
     return mv.reshape(vals.shape), mi.reshape(ids.shape)

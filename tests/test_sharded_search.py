@@ -66,6 +66,55 @@ def _rank_main(rank, world, port, out):
         td.destroy_process_group()
 
 
+def _rank_main_sharded_topk(rank, world, port, out):
+    """sharded_topk itself: the oracle's top-k of this rank's shard in place of
+    tq_topk, and a numpy merge in place of tq_topk_merge (both take and return
+    torch tensors, as the library calls do); the id offsets, the all-gather
+    and the layouts are the package's."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    from kv_cache_embedding_b200 import sharded
+    from oracle import oracle as O
+    td.init_process_group("gloo", rank=rank, world_size=world,
+                          timeout=datetime.timedelta(seconds=60))
+    try:
+        P, codes, xn, rn, q = _database()
+        start, stop = sharded.shard_bounds(N, world, rank)
+
+        def local_topk(shard, qq, k):
+            c, x, r = shard
+            v, i = O.topk(O.score(P, c, x, r, qq[0].numpy()), k)
+            return torch.from_numpy(v)[None], torch.from_numpy(i)[None]
+
+        def merge(gv, gi, k):
+            v, i = _merge_lists(gv.numpy(), gi.numpy(), k)
+            return torch.from_numpy(v), torch.from_numpy(i)
+
+        shard = (codes[start:stop], xn[start:stop], rn[start:stop])
+        mv, mi = sharded.sharded_topk(None, shard, torch.from_numpy(q)[None], K, N,
+                                      local_topk=local_topk, merge=merge)
+        assert mv.shape == (1, NQ, K) and mi.shape == (1, NQ, K)
+        out[rank] = (mv[0].numpy(), mi[0].numpy())
+    finally:
+        td.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_topk_function_equals_whole_database(world):
+    """sharded.sharded_topk (the call bench.py makes for the search at N > 1)
+    over gloo ranks equals the oracle's top-k over the whole database."""
+    from oracle import oracle as O
+    port = _free_port()
+    out = mp.Manager().dict()
+    mp.spawn(_rank_main_sharded_topk, args=(world, port, out), nprocs=world, join=True)
+    P, codes, xn, rn, q = _database()
+    ev, ei = O.topk(O.score(P, codes, xn, rn, q), K)
+    for rank in range(world):
+        mv, mi = out[rank]
+        np.testing.assert_array_equal(mi, ei)
+        np.testing.assert_array_equal(mv, ev)
+
+
 @pytest.mark.parametrize("world", [2, 3])
 def test_sharded_topk_equals_whole_database(world):
     from oracle import oracle as O
