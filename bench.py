@@ -495,11 +495,21 @@ def e2e_time(tq, cfg, x, q, steps, dist, dev, shard):
     return ms, h2d, d2h
 
 
+def workload(name, args):
+    """A workload's config, with its rows per group set by --rows (small cases
+    of the same kernels for profiler captures)."""
+    cfg = dict(CONFIGS[name])
+    if getattr(args, "rows", None):
+        cfg["n"] = int(args.rows)
+        cfg["desc"] = cfg["desc"] + f" [rows per group set to {cfg['n']}]"
+    return cfg
+
+
 def bench_config(args, name, rank, world, dist, headline):
     """Time one workload; returns its JSON object (the headline's carries the
     top-level keys of the line)."""
     import kv_cache_embedding_b200 as K
-    cfg = CONFIGS[name]
+    cfg = workload(name, args)
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     sharded = name == "search" and world > 1
@@ -857,6 +867,8 @@ def main():
                     help="time plain stream launches instead of replays of the step's CUDA graph")
     ap.add_argument("--no-count", action="store_true",
                     help="skip the profiler-based launch count (for runs under ncu)")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="rows per group instead of the workload's (small cases for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -869,7 +881,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        print(json.dumps(run_reference(args, CONFIGS[head], head)))
+        print(json.dumps(run_reference(args, workload(head, args), head)))
         return 0
 
     dist = None
@@ -887,7 +899,7 @@ def main():
     out = results[head]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         for name in names:
-            results[name]["cpu_baseline"] = cpu_baseline(CONFIGS[name],
+            results[name]["cpu_baseline"] = cpu_baseline(workload(name, args),
                                                          10.0 if name == head else 4.0)
     if len(names) > 1:
         out["configs"] = {nm: {k: v for k, v in r.items()

@@ -284,17 +284,30 @@ TQ_API int tq_attention_decode(const tq_codebook_t *cb_k, const float *d_Pi_k,
  * the process exits.
  *
  * Same arguments, results, ordering and errors as tq_topk, without d_ws and
- * ws_bytes.  Returns TQ_ERR_SCRATCH_LIMIT, having launched nothing, when
- * tq_workspace_bytes(TQ_OP_TOPK, d, b, G, n, nq, k) exceeds the array (for
- * d = 128, b = 4: e.g. 8 KV heads x 4 query heads x 131072 tokens, k = 10 fits).
+ * ws_bytes.  Which scratch form it takes:
+ *  - tq_topk's own choice when that fits the array (for searches up to 2^24
+ *    scores, the full score matrix: tq_workspace_bytes(TQ_OP_TOPK, ...));
+ *  - otherwise the form tq_topk takes beyond 2^24 scores, whose scratch holds
+ *    the transformed queries and per-range candidate lists (at d = 128 with
+ *    b >= 2 it scores chunks of keys sized to what is left of the array, with
+ *    the same results as tq_topk);
+ *  - TQ_ERR_SCRATCH_LIMIT, having launched nothing, only when that second
+ *    form does not fit either (e.g. more than ~8000 queries, whose two
+ *    transforms alone fill the array).  For d = 128, b = 4, 8 KV heads x 4
+ *    query heads x 131072 tokens and k = 10 take the second form.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  It allocates nothing: no cudaMalloc, cudaFree
- * or allocating library routine.  Every call on a device shares the one
- * array, which keeps the last call's contents (each call overwrites all of
- * the scratch it reads, nothing relies on it starting at zero): calls that
- * overlap on the GPU (different streams, or host threads) race on it and
- * must be serialised by the caller. */
+ * before any stream capture.  A device reset (cudaDeviceReset) unloads the
+ * library's module and invalidates the looked-up address: do not call this
+ * entry point on a device after resetting it.  It allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library routine.  Every call on a device
+ * shares the one array, which keeps the last call's contents (each call
+ * overwrites all of the scratch it reads, nothing relies on it starting at
+ * zero): calls that overlap on the GPU (different streams, or host threads)
+ * race on it and must be serialised by the caller.  A bounded device-side
+ * wait that gives up is recorded in the array, which the caller cannot read:
+ * on this path such a time-out is not reported (tq_topk reports it through
+ * tq_device_status). */
 #define TQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 TQ_API int tq_topk_noalloc(const tq_codebook_t *cb, const float *d_Pi, const float *d_S,
                            int G, int64_t n, const uint32_t *d_codes, const float *d_xnorm,

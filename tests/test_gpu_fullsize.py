@@ -142,3 +142,40 @@ def test_large_d_full_size(tq_lib, cuda, b):
     s_ora = O.score(O.Params(d, b, 0), c[r], xn[r], rn[r], qs)
     PT.compare_scores(_np(s[0][:, rows.to(cuda)]), s_ora, np.linalg.norm(qs, axis=1),
                       xn[r].astype(np.float64))
+
+
+@pytest.mark.parametrize("b,n", [(4, 1_000_000), (2, 262_144)])
+def test_search_chain_on_encoded_database(tq_lib, cuda, b, n):
+    """The search chain on one database: fp32 unit rows (d = 1536) encoded on
+    the GPU, the top-10 of the 1024 queries over those codes, and the exact
+    fp32 top-10 of the same rows.  For 64 sampled queries the oracle scores
+    the GPU's own records (it is given the codes and norms, never x) and takes
+    its top-10: the id sets agree on every query that is not a near tie, so
+    recall@10 against the exact top-10 is the same for the GPU and the
+    oracle on those queries."""
+    d, nq, k = 1536, 1024, 10
+    x = synth.gaussian_rows(n, d, seed=1, device=cuda, unit=True)[None]
+    q = synth.gaussian_rows(nq, d, seed=2, device=cuda, unit=True)[None]
+    quant = tq_lib.TurboQuant(d, b, seed=0, groups=1, device=cuda)
+    codes = quant.encode(x)
+    vals, ids = quant.topk(codes, q, k)
+    _, exact = tq_lib.exact_topk(x, q, k)
+    torch.cuda.synchronize()
+    pick = np.sort(synth.sample_rows(nq, 64, seed=11).numpy())
+    c = _np(codes.codes[0]).view(np.uint32)
+    xn, rn = _np(codes.xnorm[0]), _np(codes.rnorm[0])
+    qs = q[0, pick].cpu().to(torch.float64).numpy()
+    s_ora = O.score(O.Params(d, b, 0), c, xn, rn, qs)
+    rep = PT.compare_topk(_np(vals[0, pick]), _np(ids[0, pick]), s_ora, k, np.ones(len(pick)),
+                          float(xn.max()))
+    assert rep["near_tie_queries"] <= len(pick) // 4
+    _, o_ids = O.topk(s_ora, k)
+    g_ids, ex = _np(ids[0, pick]), _np(exact[0, pick])
+    r_gpu, r_ora = [], []
+    for t in range(len(pick)):
+        order = np.sort(s_ora[t])[::-1]
+        if order[k - 1] - order[k] <= 1e-5 * float(xn.max()):
+            continue  # near tie: the id sets may legitimately differ
+        r_gpu.append(len(set(g_ids[t]) & set(ex[t])) / k)
+        r_ora.append(len(set(o_ids[t]) & set(ex[t])) / k)
+    assert r_gpu == r_ora and len(r_gpu) >= 3 * len(pick) // 4
