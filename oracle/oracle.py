@@ -48,6 +48,12 @@ def lib():
         L.tqo_mse_score.argtypes = [i32, i32, P, i64, P, P, i64, P, P]
         L.tqo_mse_decode.argtypes = [i32, i32, P, P, i64, P, P, P]
         L.tqo_softmax_weighted_sum.argtypes = [i64, i64, i32, P, P, P]
+        L.tqo_split_words_per_vector.restype = i64
+        L.tqo_split_words_per_vector.argtypes = [i32, i32]
+        L.tqo_split_encode.argtypes = [i32, i32, P, P, P, P, P, P, i64, P, P, P, P, P, P, P]
+        L.tqo_split_unpack.argtypes = [i32, i32, i64, P, P, P]
+        L.tqo_split_decode.argtypes = [i32, i32, P, P, P, P, i64, P, P, P, P]
+        L.tqo_split_score.argtypes = [i32, i32, P, P, i64, P, P, P, i64, P, P, P]
         _lib = L
     return _lib
 
@@ -304,3 +310,80 @@ def attention_decode(kparams, kcodes, kxnorm, krnorm, vparams, vcodes, vxnorm, q
     values = mse_decode(vparams, vcodes, vxnorm)
     return softmax_weighted_sum(logits, values)
 
+
+
+# ---------------------------------------------------------------- fractional widths
+class SplitParams:
+    """The oracle's parameters of the fractional width b - 1/2 for (d, b, seed):
+    the first d/2 rotated coordinates on the grid of b total bits (c_hi,
+    beta_hi: 2^(b-1) levels), the last d/2 on that of b - 1 (c_lo, beta_lo),
+    and the Pi and S of the inner-product quantizer of that seed."""
+
+    def __init__(self, d, b, seed):
+        self.d, self.b, self.seed = d, b, seed
+        self.c_hi, self.beta_hi = codebook(d, b)
+        self.c_lo, self.beta_lo = codebook(d, b - 1)
+        self.Pi = rotation(d, seed)
+        self.S = qjl_matrix(d, seed)
+
+
+def split_words_per_vector(d, b):
+    return int(lib().tqo_split_words_per_vector(d, b))
+
+
+def _tab(a):
+    return a if a.size else np.zeros(1, np.float32)
+
+
+def split_encode(params, x, diagnostics=False):
+    """Records of the fractional width: codes [n, d/64 (2b - 1)] uint32, xnorm,
+    rnorm; with diagnostics also y, p [n, d] float64 and idx [n, d] int32."""
+    d, b = params.d, params.b
+    x = _f64(x).reshape(-1, d)
+    n = x.shape[0]
+    codes = np.empty((n, split_words_per_vector(d, b)), dtype=np.uint32)
+    xn = np.empty(n, dtype=np.float32)
+    rn = np.empty(n, dtype=np.float32)
+    y = np.empty((n, d), np.float64) if diagnostics else None
+    p = np.empty((n, d), np.float64) if diagnostics else None
+    idx = np.empty((n, d), np.int32) if diagnostics else None
+    _check(lib().tqo_split_encode(d, b, _p(_tab(params.c_hi)), _p(_tab(params.beta_hi)),
+                                  _p(_tab(params.c_lo)), _p(_tab(params.beta_lo)), _p(params.Pi),
+                                  _p(params.S), n, _p(x), _p(codes), _p(xn), _p(rn), _p(y),
+                                  _p(p), _p(idx)), "split_encode")
+    if diagnostics:
+        return codes, xn, rn, y, p, idx
+    return codes, xn, rn
+
+
+def split_unpack(d, b, codes):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32).reshape(-1, split_words_per_vector(d, b))
+    n = codes.shape[0]
+    idx = np.empty((n, d), np.int32)
+    z = np.empty((n, d), np.int32)
+    _check(lib().tqo_split_unpack(d, b, n, _p(codes), _p(idx), _p(z)), "split_unpack")
+    return idx, z
+
+
+def split_decode(params, codes, xnorm, rnorm):
+    d, b = params.d, params.b
+    codes = np.ascontiguousarray(codes, dtype=np.uint32).reshape(-1, split_words_per_vector(d, b))
+    n = codes.shape[0]
+    out = np.empty((n, d), np.float64)
+    _check(lib().tqo_split_decode(d, b, _p(_tab(params.c_hi)), _p(_tab(params.c_lo)),
+                                  _p(params.Pi), _p(params.S), n, _p(codes), _p(_f32(xnorm)),
+                                  _p(_f32(rnorm)), _p(out)), "split_decode")
+    return out
+
+
+def split_score(params, codes, xnorm, rnorm, q):
+    """Estimated <q_t, x_v> from split records: [nq, n]."""
+    d, b = params.d, params.b
+    qr, u = query(params, q)
+    codes = np.ascontiguousarray(codes, dtype=np.uint32).reshape(-1, split_words_per_vector(d, b))
+    n = codes.shape[0]
+    out = np.empty((qr.shape[0], n), np.float64)
+    _check(lib().tqo_split_score(d, b, _p(_tab(params.c_hi)), _p(_tab(params.c_lo)), n,
+                                 _p(codes), _p(_f32(xnorm)), _p(_f32(rnorm)), qr.shape[0],
+                                 _p(qr), _p(u), _p(out)), "split_score")
+    return out

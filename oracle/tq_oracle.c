@@ -534,6 +534,184 @@ int tqo_score(int d, int b, const float *c, int64_t n, const uint32_t *codes,
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Fractional bit widths ([QPD] experiments: quality neutral at 3.5 bits per */
+/* channel on LongBench, a mild loss at 2.5; comuna.ru, the KV-cache         */
+/* paragraph).  The pages give only the average width.  Reading (R13): the   */
+/* first d/2 rotated coordinates take b total bits (b-1 index bits and the   */
+/* sign), the last d/2 take b-1 (b-2 index bits and the sign), each half     */
+/* rounded on the Lloyd-Max grid of its own level count for the same         */
+/* N(0, 1/d) marginal; the QJL sign covers every coordinate.  The record is  */
+/* the first half's d/64 blocks in the R7 layout of width b, then the second */
+/* half's d/64 blocks in the layout of width b-1: b - 1/2 bits a coordinate. */
+/* ------------------------------------------------------------------------ */
+int64_t tqo_split_words_per_vector(int d, int b)
+{
+    return (int64_t)(d / 64) * (2 * b - 1);
+}
+
+static int tqo_check_split(int d, int b)
+{
+    if (d <= 0 || d % 64 != 0) return -1;
+    if (b < 2 || b > 4) return -1;
+    return 0;
+}
+
+/* width and first word of 32-coordinate block w of a split record */
+static int tqo_split_block_bits(int d, int b, int w)
+{
+    return (w < d / 64) ? b : b - 1;
+}
+
+static int64_t tqo_split_block_offset(int d, int b, int w)
+{
+    const int h = d / 64;
+    return (w < h) ? (int64_t)w * b : (int64_t)h * b + (int64_t)(w - h) * (b - 1);
+}
+
+/* Encode with the steps of tqo_encode; coordinate i is rounded on the grid of
+ * its half (c_hi, beta_hi: 2^(b-1) levels for i < d/2; c_lo, beta_lo:
+ * 2^(b-2) levels after, none when b = 2). */
+int tqo_split_encode(int d, int b, const float *c_hi, const float *beta_hi,
+                     const float *c_lo, const float *beta_lo, const float *Pi,
+                     const float *S, int64_t n, const double *x, uint32_t *codes,
+                     float *xnorm, float *rnorm, double *y_out, double *p_out,
+                     int32_t *idx_out)
+{
+    int64_t wpv, v;
+    if (tqo_check_split(d, b)) return -1;
+    wpv = tqo_split_words_per_vector(d, b);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (v = 0; v < n; v++) {
+        const double *xv = x + (size_t)v * d;
+        double *y = (double *)malloc(sizeof(double) * (size_t)d);
+        double *r = (double *)malloc(sizeof(double) * (size_t)d);
+        double *p = (double *)malloc(sizeof(double) * (size_t)d);
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        int32_t *z = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        double nx = 0.0, nr = 0.0;
+        int i, j, w;
+        for (j = 0; j < d; j++) nx += xv[j] * xv[j];
+        nx = sqrt(nx);
+        for (i = 0; i < d; i++) {
+            double acc = 0.0;
+            for (j = 0; j < d; j++) acc += (double)Pi[(size_t)i * d + j] * xv[j];
+            y[i] = (nx > 0.0) ? acc / nx : 0.0;
+        }
+        for (i = 0; i < d; i++) {
+            const int hi = i < d / 2;
+            const int k = hi ? b - 1 : b - 2;
+            const float *c = hi ? c_hi : c_lo, *beta = hi ? beta_hi : beta_lo;
+            int cnt = 0;
+            for (j = 0; j + 1 < (1 << k); j++)
+                if ((double)beta[j] <= y[i]) cnt++;
+            idx[i] = cnt;
+            r[i] = y[i] - ((k > 0) ? (double)c[cnt] : 0.0);
+            nr += r[i] * r[i];
+        }
+        nr = sqrt(nr);
+        for (i = 0; i < d; i++) {
+            double acc = 0.0;
+            for (j = 0; j < d; j++) acc += (double)S[(size_t)i * d + j] * r[j];
+            p[i] = acc;
+            z[i] = (acc >= 0.0) ? 1 : 0;
+        }
+        for (w = 0; w < d / 32; w++)
+            tqo_pack_block(tqo_split_block_bits(d, b, w), idx + 32 * w, z + 32 * w,
+                           codes + (size_t)v * wpv + tqo_split_block_offset(d, b, w));
+        xnorm[v] = (float)nx;
+        rnorm[v] = (float)nr;
+        if (y_out) memcpy(y_out + (size_t)v * d, y, sizeof(double) * (size_t)d);
+        if (p_out) memcpy(p_out + (size_t)v * d, p, sizeof(double) * (size_t)d);
+        if (idx_out) memcpy(idx_out + (size_t)v * d, idx, sizeof(int32_t) * (size_t)d);
+        free(y); free(r); free(p); free(idx); free(z);
+    }
+    return 0;
+}
+
+int tqo_split_unpack(int d, int b, int64_t n, const uint32_t *codes, int32_t *idx, int32_t *z)
+{
+    int64_t wpv, v;
+    if (tqo_check_split(d, b)) return -1;
+    wpv = tqo_split_words_per_vector(d, b);
+    for (v = 0; v < n; v++)
+        for (int w = 0; w < d / 32; w++)
+            tqo_unpack_block(tqo_split_block_bits(d, b, w),
+                             codes + (size_t)v * wpv + tqo_split_block_offset(d, b, w),
+                             idx + (size_t)v * d + 32 * w, z + (size_t)v * d + 32 * w);
+    return 0;
+}
+
+/* yhat_i of a split record: the centroid of coordinate i's half (0 where that
+ * half has no index bits). */
+static double tqo_split_yhat(int d, int b, const float *c_hi, const float *c_lo, int i,
+                             int32_t idx)
+{
+    if (i < d / 2) return (double)c_hi[idx];
+    return (b - 2 > 0) ? (double)c_lo[idx] : 0.0;
+}
+
+/* Dequantization of a split record, as tqo_decode. */
+int tqo_split_decode(int d, int b, const float *c_hi, const float *c_lo, const float *Pi,
+                     const float *S, int64_t n, const uint32_t *codes, const float *xnorm,
+                     const float *rnorm, double *xhat)
+{
+    int64_t v;
+    const double kappa0 = sqrt(3.14159265358979323846 / 2.0) / (double)d;
+    if (tqo_check_split(d, b)) return -1;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (v = 0; v < n; v++) {
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        int32_t *z = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        double *e = (double *)malloc(sizeof(double) * (size_t)d);
+        double kap = kappa0 * (double)rnorm[v];
+        int i, j;
+        tqo_split_unpack(d, b, 1, codes + (size_t)v * tqo_split_words_per_vector(d, b), idx, z);
+        for (j = 0; j < d; j++) {
+            double acc = 0.0;
+            for (i = 0; i < d; i++)
+                acc += (double)S[(size_t)i * d + j] * (z[i] ? 1.0 : -1.0);
+            e[j] = tqo_split_yhat(d, b, c_hi, c_lo, j, idx[j]) + kap * acc;
+        }
+        for (j = 0; j < d; j++) {
+            double acc = 0.0;
+            for (i = 0; i < d; i++) acc += (double)Pi[(size_t)i * d + j] * e[i];
+            xhat[(size_t)v * d + j] = (double)xnorm[v] * acc;
+        }
+        free(idx); free(z); free(e);
+    }
+    return 0;
+}
+
+/* The estimator of tqo_score on split records. */
+int tqo_split_score(int d, int b, const float *c_hi, const float *c_lo, int64_t n,
+                    const uint32_t *codes, const float *xnorm, const float *rnorm, int64_t nq,
+                    const double *qr, const double *u, double *scores)
+{
+    int64_t wpv, v;
+    const double kappa0 = sqrt(3.14159265358979323846 / 2.0) / (double)d;
+    if (tqo_check_split(d, b)) return -1;
+    wpv = tqo_split_words_per_vector(d, b);
+#pragma omp parallel for schedule(dynamic, 64)
+    for (v = 0; v < n; v++) {
+        int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        int32_t *z = (int32_t *)malloc(sizeof(int32_t) * (size_t)d);
+        tqo_split_unpack(d, b, 1, codes + (size_t)v * wpv, idx, z);
+        for (int64_t t = 0; t < nq; t++) {
+            const double *a = qr + (size_t)t * d, *bb = u + (size_t)t * d;
+            double mse = 0.0, qjl = 0.0;
+            for (int i = 0; i < d; i++) {
+                mse += a[i] * tqo_split_yhat(d, b, c_hi, c_lo, i, idx[i]);
+                qjl += bb[i] * (z[i] ? 1.0 : -1.0);
+            }
+            scores[(size_t)t * n + v] =
+                (double)xnorm[v] * (mse + kappa0 * (double)rnorm[v] * qjl);
+        }
+        free(idx); free(z);
+    }
+    return 0;
+}
+
 /* Top-k per query: order by score descending, then id ascending; by plain
  * selection (k passes over the row). */
 int tqo_topk(int64_t nq, int64_t n, const double *scores, int k,

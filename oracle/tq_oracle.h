@@ -78,6 +78,22 @@ int tqo_mse_score(int d, int b, const float *c, int64_t n, const uint32_t *codes
 int tqo_mse_decode(int d, int b, const float *c, const float *Pi, int64_t n,
                    const uint32_t *codes, const float *xnorm, double *out);
 
+/* Fractional widths (b - 1/2 bits a coordinate): the first d/2 rotated
+ * coordinates at b bits, the last d/2 at b - 1 (b = 2..4, d % 64 == 0). */
+int64_t tqo_split_words_per_vector(int d, int b);
+int tqo_split_encode(int d, int b, const float *c_hi, const float *beta_hi,
+                     const float *c_lo, const float *beta_lo, const float *Pi,
+                     const float *S, int64_t n, const double *x, uint32_t *codes,
+                     float *xnorm, float *rnorm, double *y_out, double *p_out,
+                     int32_t *idx_out);
+int tqo_split_unpack(int d, int b, int64_t n, const uint32_t *codes, int32_t *idx, int32_t *z);
+int tqo_split_decode(int d, int b, const float *c_hi, const float *c_lo, const float *Pi,
+                     const float *S, int64_t n, const uint32_t *codes, const float *xnorm,
+                     const float *rnorm, double *xhat);
+int tqo_split_score(int d, int b, const float *c_hi, const float *c_lo, int64_t n,
+                    const uint32_t *codes, const float *xnorm, const float *rnorm, int64_t nq,
+                    const double *qr, const double *u, double *scores);
+
 /* Decode attention: out_t = sum_j softmax_j(logits_t) values_j (fp64). */
 int tqo_softmax_weighted_sum(int64_t nq, int64_t n, int d, const double *logits,
                              const double *values, double *out);
