@@ -112,6 +112,13 @@ typedef struct tq_codebook {
     double   distortion;   /* Lloyd-Max mean squared error for N(0,1)        */
     int32_t  variant;      /* TQ_VARIANT_PROD or TQ_VARIANT_MSE              */
     int32_t  reserved;     /* 0                                              */
+    /* fractional widths (tq_build_codebook_split; all 0 otherwise): split = 1
+     * when the last d/2 rotated coordinates use the tables below, of
+     * levels_lo levels (0 when they keep only the sign) */
+    int32_t  split;
+    int32_t  levels_lo;
+    float    centroids_lo[16];
+    float    boundaries_lo[16];
 } tq_codebook_t;
 
 /* Bytes of device workspace an operation needs for the given sizes (0 when
@@ -150,6 +157,25 @@ TQ_API int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook_t *
  * Same arguments, sizes and errors as tq_build_codebook otherwise. */
 TQ_API int tq_build_codebook_mse(int d, int b, uint64_t seed, int G, tq_codebook_t *cb,
                           float *d_Pi, void *d_ws, size_t ws_bytes, void *stream);
+
+/* E0 of the fractional widths.  quant_prune_distill #674 (experiments) and
+ * comuna.ru "Google speeds up LLMs 8x" report KV caches at 3.5 and 2.5 bits
+ * per channel; the pages give only the average.  Here b - 1/2 bits a
+ * coordinate: the first d/2 rotated coordinates take b total bits (b-1 index
+ * bits and the QJL sign), the last d/2 take b - 1, each half rounded on the
+ * Lloyd-Max grid of its own level count for the same N(0, 1/d) marginal:
+ * centroids/boundaries hold 2^(b-1) levels, centroids_lo/boundaries_lo 2^(b-2)
+ * (none for b = 2, whose second half keeps only the sign).  Pi_g and S_g are
+ * tq_build_codebook's.  b in 2..4 (1.5, 2.5 and 3.5 bits); cb->split = 1.
+ * Records hold W = d/64 (2b - 1) words: the first half's d/64 blocks in the
+ * layout of width b (above), then the second half's in the layout of width
+ * b - 1.  tq_encode, tq_score, tq_topk, tq_score_topk, tq_topk_noalloc and
+ * tq_decode take such a codebook (same arguments; records of this layout);
+ * tq_attention_decode returns TQ_ERR_UNSUPPORTED for it.  Same errors as
+ * tq_build_codebook otherwise (b outside 2..4: TQ_ERR_UNSUPPORTED). */
+TQ_API int tq_build_codebook_split(int d, int b, uint64_t seed, int G, tq_codebook_t *cb,
+                                   float *d_Pi, float *d_S, void *d_ws, size_t ws_bytes,
+                                   void *stream);
 
 /* E1-E6, encode (quant_prune_distill #674 inner-product quantizer;
  * RecSysChannel #256 caveat 1: normalise, multiply by a random matrix):

@@ -8,7 +8,8 @@ The compute lives in libtq.so (include/tq.h); this package is its binding.
 """
 from . import _binding as binding  # noqa: F401  (raises if libtq.so is missing)
 from ._binding import (  # noqa: F401
-    TQError, tq_attention_decode, tq_build_codebook, tq_build_codebook_mse, tq_decode, tq_encode,
+    TQError, tq_attention_decode, tq_build_codebook, tq_build_codebook_mse,
+    tq_build_codebook_split, tq_decode, tq_encode,
     tq_exact_topk, tq_logits_fp32, tq_score, tq_score_topk, tq_status_str, tq_topk, tq_topk_merge,
     tq_topk_noalloc, tq_workspace_bytes)
 from .quantizer import Codes, TurboQuant, Workspace, exact_topk, logits_fp32  # noqa: F401

@@ -30,6 +30,7 @@ TQ_VARIANT_MSE = 1
  TQ_OP_ATTENTION, TQ_OP_SCORE_TOPK) = range(8)
 
 EXPORTS = ("tq_workspace_bytes", "tq_status_str", "tq_build_codebook", "tq_build_codebook_mse",
+           "tq_build_codebook_split",
            "tq_encode", "tq_score",
            "tq_topk", "tq_decode", "tq_logits_fp32", "tq_exact_topk", "tq_topk_noalloc",
            "tq_device_status", "tq_selftest_wait_timeout", "tq_attention_decode",
@@ -48,6 +49,10 @@ class tq_codebook_t(C.Structure):
         ("distortion", C.c_double),
         ("variant", C.c_int32),
         ("reserved", C.c_int32),
+        ("split", C.c_int32),
+        ("levels_lo", C.c_int32),
+        ("centroids_lo", C.c_float * 16),
+        ("boundaries_lo", C.c_float * 16),
     ]
 
 
@@ -72,6 +77,8 @@ def _load():
     L.tq_build_codebook.argtypes = [i32, i32, u64, i32, cbp, P, P, P, sz, P]
     L.tq_build_codebook_mse.restype = i32
     L.tq_build_codebook_mse.argtypes = [i32, i32, u64, i32, cbp, P, P, sz, P]
+    L.tq_build_codebook_split.restype = i32
+    L.tq_build_codebook_split.argtypes = [i32, i32, u64, i32, cbp, P, P, P, sz, P]
     L.tq_encode.restype = i32
     L.tq_encode.argtypes = [cbp, P, P, i32, i64, P, i32, P, P, P, P, sz, P]
     L.tq_score.restype = i32
@@ -125,6 +132,12 @@ def tq_build_codebook(d, b, seed, G, cb, d_Pi, d_S, d_ws, ws_bytes, stream):
 def tq_build_codebook_mse(d, b, seed, G, cb, d_Pi, d_ws, ws_bytes, stream):
     return _ok("tq_build_codebook_mse",
                lib.tq_build_codebook_mse(d, b, seed, G, C.byref(cb), d_Pi, d_ws, ws_bytes, stream))
+
+
+def tq_build_codebook_split(d, b, seed, G, cb, d_Pi, d_S, d_ws, ws_bytes, stream):
+    return _ok("tq_build_codebook_split",
+               lib.tq_build_codebook_split(d, b, seed, G, C.byref(cb), d_Pi, d_S, d_ws, ws_bytes,
+                                           stream))
 
 
 def tq_encode(cb, d_Pi, d_S, G, n, d_x, x_dtype, d_codes, d_xnorm, d_rnorm, d_ws, ws_bytes,

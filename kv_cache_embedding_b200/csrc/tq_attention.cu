@@ -279,6 +279,7 @@ extern "C" int tq_attention_decode(const tq_codebook_t* cb_k, const float* d_Pi_
     if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
     if (is_mse(cb_k) || !is_mse(cb_v)) return TQ_ERR_ARG;
     if (cb_k->d != kAD || cb_v->d != kAD) return TQ_ERR_UNSUPPORTED;
+    if (is_split(cb_k) || is_split(cb_v)) return TQ_ERR_UNSUPPORTED;
     if (!valid_db(cb_k->d, cb_k->b) || !valid_db(cb_v->d, cb_v->b)) return TQ_ERR_UNSUPPORTED;
     if (cb_k->groups < G || cb_v->groups < G) return TQ_ERR_MISMATCH;
     if (!d_Pi_k || !d_S_k || !d_Pi_v || !d_kcodes || !d_kxnorm || !d_krnorm || !d_vcodes ||

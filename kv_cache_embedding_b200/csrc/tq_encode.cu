@@ -90,10 +90,11 @@ __global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
 
 // One warp per row: bucketize each rotated coordinate, the cell index to a byte
 // array, |r|, and the fp16 pieces of rscale * r (r = y - c[idx]) -- hi to
-// rp[0], lo to rp[1] -- as the operand of the QJL product.
+// rp[0], lo to rp[1] -- as the operand of the QJL product.  Coordinates from
+// `half` on take the second grid of a fractional width (c_lo, beta_lo).
 __global__ void k_quantize16(const float* __restrict__ yr, uint8_t* __restrict__ idx, int64_t rows,
                              int d, KCodebook cb, float rscale, float* __restrict__ rnorm,
-                             __half* __restrict__ rp) {
+                             __half* __restrict__ rp, int half) {
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (row >= rows) return;
@@ -104,13 +105,15 @@ __global__ void k_quantize16(const float* __restrict__ yr, uint8_t* __restrict__
     float rr = 0.f;
     for (int i = lane; i < d; i += 32) {
         const float v = y[i];
+        const bool second = i >= half;  // the second grid of a fractional width
+        const int levels = second ? cb.levels_lo : cb.levels;
         int cell = 0;
         float r = v;
-        if (cb.levels > 0) {
+        if (levels > 0) {
 #pragma unroll
             for (int j = 0; j < 15; ++j)
-                if (j + 1 < cb.levels && cb.beta[j] <= v) ++cell;
-            r = v - cb.c[cell];
+                if (j + 1 < levels && (second ? cb.beta_lo[j] : cb.beta[j]) <= v) ++cell;
+            r = v - (second ? cb.c_lo[cell] : cb.c[cell]);
         }
         ix[i] = (uint8_t)cell;
         rr = fmaf(r, r, rr);
@@ -153,8 +156,31 @@ __global__ void k_quantize(float* __restrict__ yr, uint8_t* __restrict__ idx, in
     if (lane == 0) rnorm[row] = sqrtf(rr);
 }
 
-// One warp per row; lane j handles coordinate 32w + j of block w.  Fields of
-// neighbouring lanes are OR-combined with a butterfly inside each word's lanes.
+// One 32-coordinate block of a record: lane j holds coordinate j's cell index
+// field `iv` and sign z; the warp ORs neighbouring lanes' fields together with
+// a butterfly inside each word's lanes and writes the block's B words.
+template <int B>
+__device__ __forceinline__ void pack_block(int lane, uint32_t iv, uint32_t z, uint32_t* out) {
+    if (B == 1) {
+        const uint32_t word = __ballot_sync(0xffffffffu, z != 0u);
+        if (lane == 0) out[0] = word;
+    } else if (B == 2 || B == 4) {
+        constexpr int per = 32 / B;  // coordinates per word
+        uint32_t f = (iv | (z << (B - 1))) << (B * (lane % per));
+#pragma unroll
+        for (int o = 1; o < per; o <<= 1) f |= __shfl_xor_sync(0xffffffffu, f, o);
+        if (lane % per == 0) out[lane / per] = f;
+    } else {  // B == 3: 2-bit index fields (16 per word), then the sign word
+        uint32_t f = iv << (2 * (lane % 16));
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) f |= __shfl_xor_sync(0xffffffffu, f, o);
+        const uint32_t zw = __ballot_sync(0xffffffffu, z != 0u);
+        if (lane % 16 == 0) out[lane / 16] = f;
+        if (lane == 0) out[2] = zw;
+    }
+}
+
+// One warp per row; lane j handles coordinate 32w + j of block w.
 // MSE: no projection; the b-bit cell is split into its low b-1 bits (idx
 // field) and its top bit (the z position).
 template <int B, bool MSE>
@@ -169,24 +195,26 @@ __global__ void k_pack(const float* __restrict__ p, const uint8_t* __restrict__ 
         const uint32_t cell = idx[row * d + i];
         const uint32_t z = MSE ? (cell >> (B - 1)) : ((p[row * d + i] >= 0.f) ? 1u : 0u);
         const uint32_t iv = MSE ? (cell & ((1u << (B - 1)) - 1u)) : cell;
-        uint32_t* out = codes + row * W + w * B;
-        if (B == 1) {
-            const uint32_t word = __ballot_sync(0xffffffffu, z != 0u);
-            if (lane == 0) out[0] = word;
-        } else if (B == 2 || B == 4) {
-            constexpr int per = 32 / B;  // coordinates per word
-            uint32_t f = (iv | (z << (B - 1))) << (B * (lane % per));
-#pragma unroll
-            for (int o = 1; o < per; o <<= 1) f |= __shfl_xor_sync(0xffffffffu, f, o);
-            if (lane % per == 0) out[lane / per] = f;
-        } else {  // B == 3: 2-bit index fields (16 per word), then the sign word
-            uint32_t f = iv << (2 * (lane % 16));
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) f |= __shfl_xor_sync(0xffffffffu, f, o);
-            const uint32_t zw = __ballot_sync(0xffffffffu, z != 0u);
-            if (lane % 16 == 0) out[lane / 16] = f;
-            if (lane == 0) out[2] = zw;
-        }
+        pack_block<B>(lane, iv, z, codes + row * W + w * B);
+    }
+}
+
+// Fractional width b - 1/2: the first d/64 blocks in the layout of width B,
+// the last d/64 in the layout of width B - 1, d/64 (2B - 1) words a record.
+template <int B>
+__global__ void k_pack_split(const float* __restrict__ p, const uint8_t* __restrict__ idx,
+                             int64_t rows, int d, uint32_t* __restrict__ codes) {
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const int h = d / 64;  // blocks per half
+    uint32_t* rec = codes + row * (int64_t)(h * (2 * B - 1));
+    for (int w = 0; w < d / 32; ++w) {
+        const int i = 32 * w + lane;
+        const uint32_t cell = idx[row * d + i];
+        const uint32_t z = (p[row * d + i] >= 0.f) ? 1u : 0u;
+        if (w < h) pack_block<B>(lane, cell, z, rec + w * B);
+        else pack_block<B - 1>(lane, cell, z, rec + h * B + (w - h) * (B - 1));
     }
 }
 
@@ -212,7 +240,9 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     // the first 256 bytes of the workspace hold the device status word
     // d = 128 bf16 keys: fused tensor-core kernel (TMA source and 16-byte code
     // stores need 16-byte aligned buffers)
-    if (!mse && encode_tc_supported(cb, x_dtype, G, n) && (uintptr_t)d_x % 16 == 0 &&
+    const bool split = is_split(cb);
+    if (split && (mse || b < 2 || d % 64)) return TQ_ERR_UNSUPPORTED;
+    if (!mse && !split && encode_tc_supported(cb, x_dtype, G, n) && (uintptr_t)d_x % 16 == 0 &&
         (uintptr_t)d_codes % 16 == 0)
         return launch_encode_tc(cb, d_Pi, d_S, G, n, d_x, d_codes, d_xnorm, d_rnorm,
                                 (int*)d_ws, s);
@@ -223,11 +253,12 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     float* Y = (float*)((char*)d_ws + 256);
     float* P = (float*)((char*)Y + align256((size_t)chunk * d * 4));
     uint8_t* IX = (uint8_t*)((char*)P + align256((size_t)chunk * d * 4));
-    const int W = words_per_vector(d, b);
+    const int W = record_words(cb);
     const size_t esz = (x_dtype == TQ_F32) ? 4 : 2;
     const size_t dd = (size_t)d * d;
-    // tensor-core GEMMs: bf16 pieces of Pi_g, S_g and of the chunk's operand
+    // the rotation and QJL products on the tensor cores, else fp32 SIMT GEMMs
     const bool tcg = gemm_tc_supported(d, d);
+    if (split && !tcg) return TQ_ERR_UNSUPPORTED;  // the SIMT fallback has one grid
     // tensor-core GEMMs: fp16 pieces [2][d][d] of 2^8 Pi_g and of 2^4 S_g, the
     // chunk's operand pieces [2][chunk][d] (x, then r) and its row scales
     __half* PiP = (__half*)(IX + align256((size_t)chunk * d));
@@ -290,7 +321,8 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                 continue;
             }
             if (tcg) {  // P = (2^sr R)(2^4 S)^T on the tensor cores: only its signs are kept
-                k_quantize16<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rscale, rn, AP);
+                k_quantize16<<<wblocks, 256, 0, s>>>(Y, IX, rows, d, kc, rscale, rn, AP,
+                                                      split ? d / 2 : d);
                 TQ_CHECK_LAUNCH();
                 rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP, 2,
                                     (const __nv_bfloat16*)SP, P, d, nullptr, 0, err, s, 2, false,
@@ -302,11 +334,19 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                                   nullptr, 0, s);
             }
             if (rc) return rc;
-            switch (b) {
-                case 1: k_pack<1, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                case 2: k_pack<2, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                case 3: k_pack<3, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
-                default: k_pack<4, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+            if (split) {
+                switch (b) {
+                    case 2: k_pack_split<2><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    case 3: k_pack_split<3><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    default: k_pack_split<4><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                }
+            } else {
+                switch (b) {
+                    case 1: k_pack<1, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    case 2: k_pack<2, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    case 3: k_pack<3, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                    default: k_pack<4, false><<<wblocks, 256, 0, s>>>(P, IX, rows, d, cg); break;
+                }
             }
             TQ_CHECK_LAUNCH();
         }

@@ -21,8 +21,12 @@ constexpr int64_t kEncodeChunk = 65536;  // rows per encode/decode chunk
 struct KCodebook {
     float c[16];
     float beta[16];
+    float c_lo[16];     // fractional widths: the last d/2 coordinates' grid
+    float beta_lo[16];
     int levels;   // PROD: 2^(b-1), 0 for b = 1; MSE: 2^b
+    int levels_lo;
     int mse;      // 1: MSE-only variant (b-bit index, no QJL)
+    int split;    // 1: fractional width (b - 1/2 bits a coordinate)
 };
 
 inline KCodebook make_kcodebook(const tq_codebook_t* cb) {
@@ -30,15 +34,24 @@ inline KCodebook make_kcodebook(const tq_codebook_t* cb) {
     for (int i = 0; i < 16; ++i) {
         k.c[i] = cb->centroids[i];
         k.beta[i] = cb->boundaries[i];
+        k.c_lo[i] = cb->split ? cb->centroids_lo[i] : 0.f;
+        k.beta_lo[i] = cb->split ? cb->boundaries_lo[i] : 0.f;
     }
     k.levels = cb->levels;
+    k.levels_lo = cb->split ? cb->levels_lo : 0;
     k.mse = cb->variant == TQ_VARIANT_MSE ? 1 : 0;
+    k.split = cb->split ? 1 : 0;
     return k;
 }
 
 inline bool is_mse(const tq_codebook_t* cb) { return cb->variant == TQ_VARIANT_MSE; }
+inline bool is_split(const tq_codebook_t* cb) { return cb->split != 0; }
 
 __host__ __device__ inline int words_per_vector(int d, int b) { return d / 32 * b; }
+// Record words of a codebook: d/32 b, or d/64 (2b - 1) for a fractional width.
+inline int record_words(const tq_codebook_t* cb) {
+    return is_split(cb) ? cb->d / 64 * (2 * cb->b - 1) : words_per_vector(cb->d, cb->b);
+}
 
 __device__ __forceinline__ float load_f32(const float* p, int64_t i) { return p[i]; }
 __device__ __forceinline__ float load_f32(const __nv_bfloat16* p, int64_t i) {

@@ -244,6 +244,30 @@ extern "C" int tq_build_codebook(int d, int b, uint64_t seed, int G, tq_codebook
     return TQ_OK;
 }
 
+extern "C" int tq_build_codebook_split(int d, int b, uint64_t seed, int G, tq_codebook_t* cb,
+                                       float* d_Pi, float* d_S, void* d_ws, size_t ws_bytes,
+                                       void* stream) {
+    using namespace tq;
+    if (!cb || G < 1) return TQ_ERR_ARG;
+    if (!valid_db(d, b) || b < 2) return TQ_ERR_UNSUPPORTED;
+    if (!d_Pi || !d_S || !d_ws) return TQ_ERR_ARG;
+    if (ws_bytes < tq_workspace_bytes(TQ_OP_BUILD, d, b, G, 0, 0, 0)) return TQ_ERR_WORKSPACE;
+    const int rc = build_matrices(d, seed, G, d_Pi, d_S, d_ws, (cudaStream_t)stream);
+    if (rc) return rc;
+    // the first half's grid (b bits: 2^(b-1) levels), the second half's (b - 1 bits)
+    tq_codebook_t out = make_codebook(d, b, seed, G, 1 << (b - 1), TQ_VARIANT_PROD);
+    const tq_codebook_t lo = make_codebook(d, b - 1, seed, G, (b == 2) ? 0 : (1 << (b - 2)),
+                                           TQ_VARIANT_PROD);
+    out.split = 1;
+    out.levels_lo = lo.levels;
+    for (int i = 0; i < 16; ++i) {
+        out.centroids_lo[i] = lo.centroids[i];
+        out.boundaries_lo[i] = lo.boundaries[i];
+    }
+    *cb = out;
+    return TQ_OK;
+}
+
 extern "C" int tq_build_codebook_mse(int d, int b, uint64_t seed, int G, tq_codebook_t* cb,
                                      float* d_Pi, void* d_ws, size_t ws_bytes, void* stream) {
     using namespace tq;

@@ -21,7 +21,7 @@ namespace {
 
 using namespace sc;
 
-template <int B, int NQ, int KP, bool F2>
+template <int B, int NQ, int KP, bool F2, bool SPLIT>
 __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ codes,
                                                 const float* __restrict__ xnorm,
                                                 const float* __restrict__ rnorm, int64_t n, int d,
@@ -31,14 +31,14 @@ __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ cod
                                                 float* __restrict__ cmax, int nchunks,
                                                 int* __restrict__ zero_cnt) {
     extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d] pairs (qr_i, u_i)
-    __shared__ float2 s_tab[16];
+    __shared__ float2 s_tab[SPLIT ? 32 : 16];
     __shared__ float s_max[4][NQ];
     const int g = blockIdx.y;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
-    load_score_smem<B, NQ>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
+    load_score_smem<B, NQ, SPLIT>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
     __syncthreads();
-    const int W = words_per_vector(d, B);
+    const int W = SPLIT ? d / 64 * (2 * B - 1) : words_per_vector(d, B);
     int64_t v[KP];
     bool ok[KP];
 #pragma unroll
@@ -55,7 +55,7 @@ __global__ __launch_bounds__(128) void k_score2(const uint32_t* __restrict__ cod
 #pragma unroll
     for (int k = 0; k < KP; ++k) rec[k] = codes + ((int64_t)g * n + (ok[k] ? v[k] : 0)) * W;
 
-    score_keys<B, NQ, KP, F2>(rec, d, s_qu, s_tab, acc);
+    score_record<B, NQ, KP, F2, SPLIT>(rec, d, s_qu, s_tab, acc);
     const float k0 = kSqrtHalfPi / (float)d;
     float mx[NQ];
 #pragma unroll
@@ -193,14 +193,14 @@ struct WarpList {
 // combined in shared memory.  Output: the range's best K per query (value,
 // global key id; -inf / INT64_MAX where the range has fewer) in
 // part_vals/part_ids [G][nq][nblk][K].
-template <int B, int NQ, bool F2>
+template <int B, int NQ, bool F2, bool SPLIT>
 __global__ __launch_bounds__(256) void k_score_topk(
     const uint32_t* __restrict__ codes, const float* __restrict__ xnorm,
     const float* __restrict__ rnorm, int64_t n, int d, int nq, const float* __restrict__ qr,
     const float* __restrict__ u, KCodebook cb, int K, int nblk, int64_t span,
     float* __restrict__ part_vals, int64_t* __restrict__ part_ids) {
     extern __shared__ __align__(16) float2 s_qu[];  // [NQ][d]
-    __shared__ float2 s_tab[16];
+    __shared__ float2 s_tab[SPLIT ? 32 : 16];
     __shared__ float s_lv[NQ][8][kMaxK];
     __shared__ uint32_t s_li[NQ][8][kMaxK];
     const int g = blockIdx.y;
@@ -209,9 +209,9 @@ __global__ __launch_bounds__(256) void k_score_topk(
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int64_t kb0 = (int64_t)blockIdx.x * span;
     const int64_t kb1 = min(n, kb0 + span);
-    load_score_smem<B, NQ>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
+    load_score_smem<B, NQ, SPLIT>(cb, qr, u, (int64_t)g * nq + q0, qn, d, s_qu, s_tab);
     __syncthreads();
-    const int W = words_per_vector(d, B);
+    const int W = SPLIT ? d / 64 * (2 * B - 1) : words_per_vector(d, B);
     const float k0 = kSqrtHalfPi / (float)d;
     WarpList<uint32_t> L[NQ];
 #pragma unroll
@@ -224,7 +224,7 @@ __global__ __launch_bounds__(256) void k_score_topk(
         float2 acc[1][NQ];
 #pragma unroll
         for (int qq = 0; qq < NQ; ++qq) acc[0][qq] = make_float2(0.f, 0.f);
-        score_keys<B, NQ, 1, F2>(rec, d, s_qu, s_tab, acc);
+        score_record<B, NQ, 1, F2, SPLIT>(rec, d, s_qu, s_tab, acc);
         const float xn = xnorm[gv];
         const float kap = k0 * rnorm[gv];
 #pragma unroll
@@ -436,45 +436,70 @@ __global__ __launch_bounds__(128) void k_topk_merge(const float* __restrict__ pa
 }
 
 // ---- dequantization -------------------------------------------------------
-// T = 2z - 1 (fp32 rows) for the rows of a chunk.
-template <int B>
+// T = 2z - 1 (fp32 rows) for the rows of a chunk.  SPLIT: records of a
+// fractional width (the last d/64 blocks at width B - 1).
+template <int B, bool SPLIT>
 __global__ void k_signs(const uint32_t* __restrict__ codes, int64_t rows, int d,
                         float* __restrict__ T) {
+    constexpr int BL = B > 1 ? B - 1 : 1;
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= rows * (d / 32)) return;
     const int64_t row = e / (d / 32);
     const int blk = (int)(e % (d / 32));
+    const int W = SPLIT ? d / 64 * (2 * B - 1) : words_per_vector(d, B);
+    const uint32_t* rec = codes + row * W;
+    float* t = T + row * d + blk * 32;
     uint32_t w[4];
-    load_block<B>(codes + row * words_per_vector(d, B), blk, w);
-    for (int j = 0; j < 32; ++j) {
-        int cell;
-        uint32_t z;
-        field<B>(w, j, cell, z);
-        T[row * d + blk * 32 + j] = z ? 1.f : -1.f;
+    int cell;
+    uint32_t z;
+    if (SPLIT && blk >= d / 64) {
+        load_block<BL, false>(rec + (d / 64) * B, blk - d / 64, w);
+        for (int j = 0; j < 32; ++j) {
+            field<BL>(w, j, cell, z);
+            t[j] = z ? 1.f : -1.f;
+        }
+    } else {
+        load_block<B, !SPLIT>(rec, blk, w);
+        for (int j = 0; j < 32; ++j) {
+            field<B>(w, j, cell, z);
+            t[j] = z ? 1.f : -1.f;
+        }
     }
 }
 
-// E = c[idx] + |r| sqrt(pi/2)/d * E  (E holds S^T (2z - 1) on entry).
-template <int B>
+// E = c[idx] + |r| sqrt(pi/2)/d * E  (E holds S^T (2z - 1) on entry); the
+// second half of a fractional-width record takes c_lo.
+template <int B, bool SPLIT>
 __global__ void k_combine(const uint32_t* __restrict__ codes, const float* __restrict__ rnorm,
                           int64_t rows, int d, KCodebook cb, float* __restrict__ E) {
+    constexpr int BL = B > 1 ? B - 1 : 1;
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= rows * (d / 32)) return;
     const int64_t row = e / (d / 32);
     const int blk = (int)(e % (d / 32));
-    uint32_t w[4];
-    load_block<B>(codes + row * words_per_vector(d, B), blk, w);
+    const int W = SPLIT ? d / 64 * (2 * B - 1) : words_per_vector(d, B);
+    const uint32_t* rec = codes + row * W;
     const float kap = kSqrtHalfPi / (float)d * rnorm[row];
+    float* p = E + row * d + blk * 32;
+    uint32_t w[4];
+    int cell;
+    uint32_t z;
+    if (SPLIT && blk >= d / 64) {
+        load_block<BL, false>(rec + (d / 64) * B, blk - d / 64, w);
+        for (int j = 0; j < 32; ++j) {
+            field<BL>(w, j, cell, z);
+            p[j] = ((BL == 1) ? 0.f : cb.c_lo[cell]) + kap * p[j];
+        }
+        return;
+    }
+    load_block<B, !SPLIT>(rec, blk, w);
     for (int j = 0; j < 32; ++j) {
-        int cell;
-        uint32_t z;
         field<B>(w, j, cell, z);
-        float* p = E + row * d + blk * 32 + j;
         if (cb.mse) {  // MSE-only variant: the b-bit cell is (idx | z << (b-1)); no QJL term
-            *p = cb.c[(B == 1) ? (int)z : (cell | (int)(z << (B - 1)))];
+            p[j] = cb.c[(B == 1) ? (int)z : (cell | (int)(z << (B - 1)))];
         } else {
             const float yh = (B == 1) ? 0.f : cb.c[cell];
-            *p = yh + kap * (*p);
+            p[j] = yh + kap * p[j];
         }
     }
 }
@@ -533,19 +558,19 @@ __global__ __launch_bounds__(256) void k_logits_fp32(const float* __restrict__ k
 
 // ---- helpers ----------------------------------------------------------------
 
-template <int B, int NQ, bool F2>
+template <int B, int NQ, bool F2, bool SPLIT>
 int launch_score2_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                     int G, int nq, const float* qr, const float* u, const KCodebook& kc,
                     float* scores, float* cmax, int* zero_cnt, cudaStream_t s) {
     constexpr int KP = 2;
     static_assert(128 * KP == kTopkTile, "one score block per top-k chunk");
     const size_t smem = (size_t)NQ * d * sizeof(float2);
-    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score2<B, NQ, KP, F2>,
+    TQ_TRY_CUDA(cudaFuncSetAttribute(k_score2<B, NQ, KP, F2, SPLIT>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     const int nchunks = (int)((n + 128 * KP - 1) / (128 * KP));
     dim3 grid((unsigned)nchunks, (unsigned)G, (unsigned)((nq + NQ - 1) / NQ));
-    k_score2<B, NQ, KP, F2><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc, scores,
-                                                    cmax, nchunks, zero_cnt);
+    k_score2<B, NQ, KP, F2, SPLIT><<<grid, 128, smem, s>>>(codes, xn, rn, n, d, nq, qr, u, kc,
+                                                           scores, cmax, nchunks, zero_cnt);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -562,9 +587,12 @@ template <int B>
 int launch_score_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                    int G, int nq, const float* qr, const float* u, const KCodebook& kc,
                    float* scores, float* cmax, int* zero_cnt, cudaStream_t s) {
-#define TQ_SC(NQV) \
-    return launch_score2_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, scores, cmax, \
-                                         zero_cnt, s)
+#define TQ_SC(NQV)                                                                              \
+    return (B >= 2 && kc.split)                                                                 \
+               ? launch_score2_t<B, NQV, true, (B >= 2)>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
+                                                         scores, cmax, zero_cnt, s)             \
+               : launch_score2_t<B, NQV, true, false>(codes, xn, rn, n, d, G, nq, qr, u, kc,    \
+                                                      scores, cmax, zero_cnt, s)
     switch (score_nq(d, nq)) {
         case 1: TQ_SC(1);
         case 2: TQ_SC(2);
@@ -581,12 +609,12 @@ struct TopkGrid {
     int64_t span;
 };
 
-template <int B, int NQ, bool F2>
+template <int B, int NQ, bool F2, bool SPLIT>
 int launch_topk_t(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
                   float* pv, int64_t* pi, TopkGrid* out, cudaStream_t s) {
     const size_t smem = (size_t)NQ * d * sizeof(float2);
-    auto kern = k_score_topk<B, NQ, F2>;
+    auto kern = k_score_topk<B, NQ, F2, SPLIT>;
     TQ_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     int dev = 0, nsm = 0, occ = 0;
     TQ_TRY_CUDA(cudaGetDevice(&dev));
@@ -611,8 +639,12 @@ template <int B>
 int launch_topk_b(const uint32_t* codes, const float* xn, const float* rn, int64_t n, int d,
                   int G, int nq, const float* qr, const float* u, const KCodebook& kc, int K,
                   float* pv, int64_t* pi, TopkGrid* tg, cudaStream_t s) {
-#define TQ_TK(NQV) \
-    return launch_topk_t<B, NQV, true>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, pv, pi, tg, s)
+#define TQ_TK(NQV)                                                                         \
+    return (B >= 2 && kc.split)                                                            \
+               ? launch_topk_t<B, NQV, true, (B >= 2)>(codes, xn, rn, n, d, G, nq, qr, u, kc, \
+                                                       K, pv, pi, tg, s)                    \
+               : launch_topk_t<B, NQV, true, false>(codes, xn, rn, n, d, G, nq, qr, u, kc, K, \
+                                                    pv, pi, tg, s)
     switch (score_nq(d, nq)) {
         case 1: TQ_TK(1);
         case 2: TQ_TK(2);
@@ -759,7 +791,7 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     float* u = (float*)((char*)qr + align256((size_t)G * nq * d * 4));
     rc = query_prep(d_Pi, d_S, G, d, nq, d_q, q_dtype, qr, u, err, s);
     if (rc) return rc;
-    if (score_gemm_supported(d, nq)) {  // many queries at d >= 256: decoded-key GEMM
+    if (!is_split(cb) && score_gemm_supported(d, nq)) {  // many queries at d >= 256: decoded-key GEMM
         void* op = (char*)u + align256((size_t)G * nq * d * 4);
         return score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr, 0,
                           op, err, s);
@@ -767,7 +799,7 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
     if (score_i8_supported(cb, G, n, nq, d_codes))
         return launch_score_i8(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
-    if (!is_mse(cb) && score_tc_supported(d, b, G, n, nq))
+    if (!is_mse(cb) && !is_split(cb) && score_tc_supported(d, b, G, n, nq))
         return launch_score_tc(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, d_scores, nullptr,
                                nullptr, err, s);
     const KCodebook kc = make_kcodebook(cb);
@@ -805,7 +837,7 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
     if (materialize) {
         // scores [G][nq][n], row maxima per chunk, counters, candidates; then
         // the per-row selection
-        const bool tc = !is_mse(cb) && score_tc_supported(d, b, G, n, nq);
+        const bool tc = !is_mse(cb) && !is_split(cb) && score_tc_supported(d, b, G, n, nq);
         const int64_t ntm = (n + 127) / 128;
         float* sc = scores_out;  // the caller's score output, else the workspace
         if (!sc) {
@@ -820,7 +852,7 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         p += align256((size_t)rows * kCandCapG * 4);
         int* ci = (int*)p;
         int nchunks;
-        if (score_gemm_supported(d, nq)) {  // decoded-key GEMM, maxima per 128-key tile
+        if (!is_split(cb) && score_gemm_supported(d, nq)) {  // decoded-key GEMM, maxima per 128-key tile
             p = (char*)ci + align256((size_t)rows * kCandCapG * 4);
             TQ_TRY_CUDA(cudaMemsetAsync(cnt, 0, (size_t)rows * 2 * 4, s));
             rc = score_gemm(cb, G, n, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, ntm, p, err, s);
@@ -995,7 +1027,8 @@ extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float
     const int64_t chunk = n < kEncodeChunk ? n : kEncodeChunk;
     float* T = (float*)d_ws;
     float* E = (float*)((char*)d_ws + align256((size_t)chunk * d * 4));
-    const int W = words_per_vector(d, b);
+    const int W = record_words(cb);
+    const bool split = is_split(cb);
     const size_t dd = (size_t)d * d;
     for (int g = 0; g < G; ++g) {
         for (int64_t r0 = 0; r0 < n; r0 += chunk) {
@@ -1004,11 +1037,19 @@ extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float
             const uint32_t* cg = d_codes + off * W;
             const unsigned blocks = (unsigned)((rows * (d / 32) + 255) / 256);
             if (!mse) {
-                switch (b) {
-                    case 1: k_signs<1><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                    case 2: k_signs<2><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                    case 3: k_signs<3><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
-                    default: k_signs<4><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                if (split) {
+                    switch (b) {
+                        case 2: k_signs<2, true><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                        case 3: k_signs<3, true><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                        default: k_signs<4, true><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                    }
+                } else {
+                    switch (b) {
+                        case 1: k_signs<1, false><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                        case 2: k_signs<2, false><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                        case 3: k_signs<3, false><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                        default: k_signs<4, false><<<blocks, 256, 0, s>>>(cg, rows, d, T); break;
+                    }
                 }
                 TQ_CHECK_LAUNCH();
                 // E = T S   (E[v][j] = sum_i T[v][i] S[i][j])
@@ -1016,11 +1057,19 @@ extern "C" int tq_decode(const tq_codebook_t* cb, const float* d_Pi, const float
                                   nullptr, 0, s);
                 if (rc) return rc;
             }
-            switch (b) {
-                case 1: k_combine<1><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
-                case 2: k_combine<2><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
-                case 3: k_combine<3><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
-                default: k_combine<4><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+            if (split) {
+                switch (b) {
+                    case 2: k_combine<2, true><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                    case 3: k_combine<3, true><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                    default: k_combine<4, true><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                }
+            } else {
+                switch (b) {
+                    case 1: k_combine<1, false><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                    case 2: k_combine<2, false><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                    case 3: k_combine<3, false><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                    default: k_combine<4, false><<<blocks, 256, 0, s>>>(cg, d_rnorm + off, rows, d, kc, E); break;
+                }
             }
             TQ_CHECK_LAUNCH();
             // xhat = |x| E Pi   (xhat[v][j] = |x_v| sum_i E[v][i] Pi[i][j])

@@ -518,7 +518,8 @@ void score_i8_tables(const tq_codebook_t* cb, uint4* ctab, float* scale_c) {
 }
 
 bool score_i8_supported(const tq_codebook_t* cb, int G, int64_t n, int nq, const void* d_codes) {
-    return !is_mse(cb) && cb->d == kD && cb->b >= 2 && cb->b <= 4 && nq > 0 && n > 0 &&
+    return !is_mse(cb) && !is_split(cb) && cb->d == kD && cb->b >= 2 && cb->b <= 4 && nq > 0 &&
+           n > 0 &&
            n < ((int64_t)1 << 31) / 128 * 128 && (int64_t)G * n < ((int64_t)1 << 40) &&
            ((uintptr_t)d_codes & 15u) == 0;
 }

@@ -60,12 +60,20 @@ class TurboQuant:
     variant="prod" (default): the inner-product quantizer, (b-1)-bit
     Lloyd-Max index + 1 QJL sign bit, unbiased inner products.
     variant="mse": the MSE-only quantizer, b-bit Lloyd-Max index, no QJL
-    (no S; biased inner products)."""
+    (no S; biased inner products).
+    A fractional b (1.5, 2.5, 3.5; inner-product quantizer only) gives the
+    first d/2 rotated coordinates ceil(b) bits and the rest floor(b)
+    (tq_build_codebook_split); self.b is then ceil(b) and self.split True."""
 
     def __init__(self, d, b, seed=0, groups=1, device="cuda", variant="prod"):
         if variant not in ("prod", "mse"):
             raise ValueError(f"variant must be 'prod' or 'mse', got {variant!r}")
-        self.d, self.b, self.seed, self.G = int(d), int(b), int(seed), int(groups)
+        self.split = float(b) != int(b)
+        if self.split and (variant != "prod" or float(b) * 2 != int(float(b) * 2)):
+            raise ValueError(f"fractional widths are b - 1/2 of the inner-product quantizer, "
+                             f"got b={b!r}, variant={variant!r}")
+        self.d, self.seed, self.G = int(d), int(seed), int(groups)
+        self.b = int(float(b) + 0.5) if self.split else int(b)
         self.variant = variant
         self.device = torch.device(device)
         self.Pi = torch.empty(self.G, d, d, dtype=torch.float32, device=self.device)
@@ -73,9 +81,12 @@ class TurboQuant:
                   if variant == "prod" else None)
         self.cb = B.tq_codebook_t()
         self.ws = Workspace(self.device)
-        nbytes = B.tq_workspace_bytes(B.TQ_OP_BUILD, d, b, self.G, 0, 0, 0)
+        nbytes = B.tq_workspace_bytes(B.TQ_OP_BUILD, d, self.b, self.G, 0, 0, 0)
         wp, wn = self.ws.get(nbytes)
-        if variant == "prod":
+        if self.split:
+            B.tq_build_codebook_split(self.d, self.b, self.seed, self.G, self.cb, _ptr(self.Pi),
+                                      _ptr(self.S), wp, wn, _stream())
+        elif variant == "prod":
             B.tq_build_codebook(self.d, self.b, self.seed, self.G, self.cb, _ptr(self.Pi),
                                 _ptr(self.S), wp, wn, _stream())
         else:
@@ -84,6 +95,8 @@ class TurboQuant:
 
     @property
     def words(self):
+        if self.split:
+            return self.d // 64 * (2 * self.b - 1)
         return self.b * self.d // 32
 
     def centroids(self):

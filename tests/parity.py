@@ -56,19 +56,48 @@ def compare_encode(d, b, beta, gpu, ora, check=True, bound_flags=True):
     Returns a report; with check, asserts the parity rules.  bound_flags=False
     drops the 1e-4 bound on the flagged fraction (for crafted inputs such as a
     zero vector, whose coordinates all sit on the middle boundary)."""
-    g_codes, g_xn, g_rn = gpu
-    o_codes, o_xn, o_rn, y, p, o_idx = ora
-    n = o_codes.shape[0]
-    sigma = 1.0 / math.sqrt(d)
+    g_codes = gpu[0]
+    o_codes, y, o_idx = ora[0], ora[3], ora[5]
     g_idx, g_z = read_layout(d, b, g_codes)
     o_idx2, o_z = read_layout(d, b, o_codes)
     assert np.array_equal(o_idx2, o_idx)
+    return _compare_fields(d, gpu, ora, g_idx, g_z, o_z, _near_boundary(d, y, beta), check,
+                           bound_flags)
+
+
+def _near_boundary(d, y, beta):
+    """Coordinates whose rotated value lies within BAND sigma of a boundary."""
+    if not beta.size:
+        return np.zeros_like(y, dtype=bool)
+    dist = np.min(np.abs(y[:, :, None] - beta.astype(np.float64)[None, None, :]), axis=2)
+    return dist < BAND / math.sqrt(d)
+
+
+def compare_encode_split(d, b, beta_hi, beta_lo, gpu, ora, check=True, bound_flags=True):
+    """Records of the fractional width b - 1/2: the first d/64 blocks are the
+    first d/2 coordinates in the b-bit layout, the rest the last d/2 in the
+    (b-1)-bit layout; each half is read with read_layout and flagged against
+    its own boundaries, then the rules of compare_encode apply."""
+    h = d // 64
+    g_codes = np.ascontiguousarray(np.asarray(gpu[0])).view(np.uint32).reshape(-1, h * (2 * b - 1))
+    o_codes, y, o_idx = ora[0], ora[3], ora[5]
+    gi_hi, gz_hi = read_layout(d // 2, b, np.ascontiguousarray(g_codes[:, :h * b]))
+    gi_lo, gz_lo = read_layout(d // 2, b - 1, np.ascontiguousarray(g_codes[:, h * b:]))
+    oi_hi, oz_hi = read_layout(d // 2, b, np.ascontiguousarray(o_codes[:, :h * b]))
+    oi_lo, oz_lo = read_layout(d // 2, b - 1, np.ascontiguousarray(o_codes[:, h * b:]))
+    assert np.array_equal(np.concatenate([oi_hi, oi_lo], 1), o_idx)
+    flag = np.concatenate([_near_boundary(d, y[:, :d // 2], beta_hi),
+                           _near_boundary(d, y[:, d // 2:], beta_lo)], 1)
+    return _compare_fields(d, (g_codes, gpu[1], gpu[2]), ora, np.concatenate([gi_hi, gi_lo], 1),
+                           np.concatenate([gz_hi, gz_lo], 1), np.concatenate([oz_hi, oz_lo], 1),
+                           flag, check, bound_flags)
+
+
+def _compare_fields(d, gpu, ora, g_idx, g_z, o_z, flag_idx, check, bound_flags):
+    g_codes, g_xn, g_rn = gpu
+    o_codes, o_xn, o_rn, y, p, o_idx = ora
+    n = o_codes.shape[0]
     rep = EncodeReport(n=n, coords=n * d)
-    if beta.size:
-        dist = np.min(np.abs(y[:, :, None] - beta.astype(np.float64)[None, None, :]), axis=2)
-        flag_idx = dist < BAND * sigma
-    else:
-        flag_idx = np.zeros_like(y, dtype=bool)
     idx_diff = g_idx != o_idx
     rep["idx_flagged"] = int(flag_idx.sum())
     rep["idx_mismatch"] = int(idx_diff.sum())

@@ -51,7 +51,7 @@ def test_codebook_struct_layout(tq_lib, tmp_path):
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
     got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
-    assert got[0] == C.sizeof(B.tq_codebook_t) == 168
+    assert got[0] == C.sizeof(B.tq_codebook_t) == 304
     assert got[1:] == [getattr(B.tq_codebook_t, f).offset for f in fields]
 
 
@@ -90,6 +90,16 @@ def test_bad_arguments_rejected_without_device_work(tq_lib):
     assert lib.tq_build_codebook(128, 4, 0, 0, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
     assert lib.tq_build_codebook(128, 4, 0, 1, None, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_ARG
     assert lib.tq_build_codebook(128, 4, 0, 1, C.byref(cb), 1, 1, 1, 16, None) == B.TQ_ERR_WORKSPACE
+    # fractional widths: b - 1/2 with 2 <= b <= 4, inner-product quantizer only
+    assert lib.tq_build_codebook_split(128, 1, 0, 1, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    assert lib.tq_build_codebook_split(96, 3, 0, 1, C.byref(cb), 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    assert lib.tq_build_codebook_split(128, 3, 0, 1, C.byref(cb), 1, None, 1, 1 << 30, None) == B.TQ_ERR_ARG
+    assert lib.tq_build_codebook_split(128, 3, 0, 1, C.byref(cb), 1, 1, 1, 16, None) == B.TQ_ERR_WORKSPACE
+    scb = B.tq_codebook_t()
+    scb.d, scb.b, scb.groups, scb.levels, scb.variant, scb.split = 128, 3, 1, 4, B.TQ_VARIANT_MSE, 1
+    assert lib.tq_encode(C.byref(scb), 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
+    scb.variant, scb.b = B.TQ_VARIANT_PROD, 1
+    assert lib.tq_encode(C.byref(scb), 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
     # a codebook that was never built: d = 0
     assert lib.tq_encode(C.byref(cb), 1, 1, 1, 10, 1, 0, 1, 1, 1, 1, 1 << 30, None) == B.TQ_ERR_UNSUPPORTED
     cb.d, cb.b, cb.groups, cb.levels = 128, 4, 1, 8
@@ -133,6 +143,9 @@ def test_bad_arguments_rejected_without_device_work(tq_lib):
     assert attn(G=2) == B.TQ_ERR_MISMATCH
     assert attn(scale=float("nan")) == B.TQ_ERR_ARG
     assert attn(ws=64) == B.TQ_ERR_WORKSPACE
+    kcb.split = 1
+    assert attn() == B.TQ_ERR_UNSUPPORTED
+    kcb.split = 0
     kcb.d = 96
     assert attn() == B.TQ_ERR_UNSUPPORTED
 
