@@ -484,6 +484,227 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
+// ---- the CTA-pair form (row-major products with N % 256 == 0) --------------
+// One 256 x 256 tile per cluster of two CTAs: CTA r stages rows m0 + 128 r of
+// A and rows n0 + 128 r of B (its halves of the pair's operands), the
+// leader's thread issues cta_group::2 MMAs of M = 256, N = 256, and each CTA's
+// tensor memory holds its 128 rows x 256 columns.  Per SM that is twice the
+// MMA work per staged byte of the 128 x 128 form above, whose MMA warp waits
+// on its stages (ncu: tensor pipe ~46 %, TMA reads ~31 % of peak), and half
+// the MMA instructions.  The accumulation and its 128-wide K chunks are the
+// same.  Warps: 0 TMA (both CTAs), 1 tensor memory (both) and the MMA issue
+// (leader), 4-11 chunk sums and stores (TMEM lane quarter warp % 4, column
+// half (warp - 4) / 4); 2-3 idle.  The leader's full barrier counts the
+// bytes of both CTAs; the leader's MMA commits release both CTAs' stages and
+// accumulators; every epilogue warp of the pair arrives on the leader's
+// accumulator-empty barrier.  Every wait is bounded.
+constexpr int kPN = 256;                       // tile columns (MMA N); tile rows 2 x kTM
+constexpr int kPairThreads = 32 * 12;
+constexpr uint32_t kPairTmemCols = 2 * kPN;    // two chunk accumulators
+constexpr uint32_t kPairEpiWarps = 8;
+
+struct SmemP {
+    uint8_t pool[kPool][kPieceBytes];  // stage s: A's pa pieces, then B's pb (1024-aligned)
+    uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done;
+    uint32_t tmem_base;
+    int abort;
+    int zero;
+};
+constexpr size_t kSmemPairBytes = sizeof(SmemP) + 1024;
+
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort) {
+    const bool ok = mbar_wait_cluster(bar, parity, abort, kWaitNs);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+            int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
+            const float* __restrict__ row_scale, int scale_mode, int* __restrict__ err,
+            uint32_t idesc) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = smem_u32(smem_raw);
+    // the same offset in both CTAs: the MMA reads the peer's operands there
+    SmemP& sm = *reinterpret_cast<SmemP*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    volatile int* abort = &sm.abort;
+    const int tm = (M + 2 * kTM - 1) / (2 * kTM), tn = N / kPN;
+    const int tiles = tm * tn;
+    const int pair = blockIdx.x / 2, npairs = gridDim.x / 2;
+    const int nkb = K / kKB;   // K blocks per tile
+    const int nch = nkb / 2;   // 128-wide K chunks per tile
+    const uint32_t stage_tx = (uint32_t)(pa + pb) * kPieceBytes;  // one CTA's bytes per stage
+    const int ns = min(kMaxStages, kPool / (pa + pb));
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMaxStages; ++s) {
+            mbar_init(&sm.full[s], 1);   // the leader's producer; the bytes of both CTAs
+            mbar_init(&sm.empty[s], 1);  // the pair's MMA commit
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.acc_full[i], 1);
+            mbar_init(&sm.acc_empty[i], 2 * kPairEpiWarps);  // used in the leader
+        }
+        mbar_init(&sm.mma_done, 1);
+        sm.abort = 0;
+        sm.zero = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&sm.tmem_base, kPairTmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barriers initialised and tensor memory allocated in both CTAs
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = pair; t < tiles && ok; t += npairs) {
+            const int m0 = (t / tn) * 2 * kTM + (int)rank * kTM;
+            const int n0 = (t % tn) * kPN + (int)rank * kTM;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = (int)(it % (uint32_t)ns);
+                if (it >= (uint32_t)ns &&
+                    !mbar_wait_cluster(&sm.empty[s], ((it / ns) - 1) & 1, abort, kWaitNs)) {
+                    ok = give_up(abort, err, 51);
+                    break;
+                }
+                if (leader) mbar_arrive_expect_tx(&sm.full[s], 2 * stage_tx);
+                const uint32_t fb = mapa_shared(smem_u32(&sm.full[s]), 0);
+                uint8_t* st = sm.pool[s * (pa + pb)];
+                for (int p = 0; p < pa; ++p)
+                    tma_load_3d_pair(st + p * kPieceBytes, &tmap_a, kb * kKB, m0, p, fb);
+                for (int p = 0; p < pb; ++p)
+                    tma_load_3d_pair(st + (pa + p) * kPieceBytes, &tmap_b, kb * kKB, n0, p, fb);
+            }
+        }
+        // no TMA write may still be in flight when the pair exits: the leader's
+        // barriers count both CTAs' bytes
+        if (leader)
+            for (uint32_t j = (it > (uint32_t)ns ? it - ns : 0); j < it; ++j)
+                mbar_wait(&sm.full[j % ns], (j / ns) & 1, &sm.zero, kWaitNs);
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ---------------- MMA issuer (leader) ----------------
+        int pi_[6], pj_[6], np = 0;
+        const int pmax = pa > pb ? pa : pb;
+        for (int sij = 0; sij < pmax; ++sij)
+            for (int i = 0; i <= sij; ++i)
+                if (i < pa && sij - i < pb) {
+                    pi_[np] = i;
+                    pj_[np] = sij - i;
+                    ++np;
+                }
+        uint32_t it = 0, cc = 0;
+        bool ok = true;
+        for (int t = pair; t < tiles && ok; t += npairs) {
+            for (int c = 0; c < nch && ok; ++c, ++cc) {
+                const uint32_t ab = cc & 1;
+                if (cc >= 2 &&
+                    !mbar_wait_cluster(&sm.acc_empty[ab], ((cc >> 1) - 1) & 1, abort, kWaitNs)) {
+                    ok = give_up(abort, err, 52);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tbase + ab * kPN;
+                for (int h = 0; h < 2; ++h, ++it) {
+                    const int s = (int)(it % (uint32_t)ns);
+                    if (!mbar_wait(&sm.full[s], (it / ns) & 1, abort, kWaitNs)) {
+                        ok = give_up(abort, err, 53);
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int q = 0; q < np; ++q) {
+                        const uint32_t as = smem_u32(sm.pool[s * (pa + pb) + pi_[q]]),
+                                       bs = smem_u32(sm.pool[s * (pa + pb) + pa + pj_[q]]);
+#pragma unroll
+                        for (int ks = 0; ks < kKB / 16; ++ks)
+                            mma_f16_ss_pair(d, smem_desc_kmajor_sw128(as + ks * 32),
+                                            smem_desc_kmajor_sw128(bs + ks * 32), idesc,
+                                            (h | q | ks) != 0);
+                    }
+                    tc_commit_pair(&sm.empty[s], 0x3);
+                }
+                if (ok) tc_commit_pair(&sm.acc_full[ab], 0x3);
+            }
+        }
+        // every issued MMA completes before either CTA releases tensor memory
+        tc_commit_pair(&sm.mma_done, 0x3);
+        mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
+    } else if (warp == 1 && lane == 0) {
+        // the leader's MMAs write this CTA's tensor memory and read its stages
+        mbar_wait_cluster(&sm.mma_done, 0, &sm.zero, kWaitNs);
+    } else if (warp >= 4) {
+        // ---------------- chunk sums and stores (both CTAs) ----------------
+        const int q = warp & 3;               // TMEM lane quarter: rows 32 q .. 32 q + 31
+        const int hc = (warp - 4) >> 2;       // column half of the tile
+        const uint32_t lane_addr = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(hc * kTN);
+        const uint32_t empty_c[2] = {mapa_shared(smem_u32(&sm.acc_empty[0]), 0),
+                                     mapa_shared(smem_u32(&sm.acc_empty[1]), 0)};
+        uint32_t cc = 0;
+        bool ok = true;
+        for (int t = pair; t < tiles && ok; t += npairs) {
+            const int m0 = (t / tn) * 2 * kTM + (int)rank * kTM;
+            const int n0 = (t % tn) * kPN + hc * kTN;
+            float sum[kTN];
+#pragma unroll
+            for (int j = 0; j < kTN; ++j) sum[j] = 0.f;
+            for (int c = 0; c < nch; ++c, ++cc) {
+                const uint32_t ab = cc & 1;
+                if (!warp_wait_cluster(&sm.acc_full[ab], (cc >> 1) & 1, abort)) {
+                    ok = give_up(abort, err, 54);
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int j0 = 0; j0 < kTN; j0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + ab * kPN + (uint32_t)j0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sum[j0 + j] += __uint_as_float(v[j]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_c[ab]);
+            }
+            if (!ok) break;
+            const int64_t row = (int64_t)m0 + 32 * q + lane;
+            if (row < M) {
+                float sc = 1.f;
+                if (scale_mode == 1) {
+                    const float r = row_scale[row];
+                    sc = (r != 0.f) ? 1.f / r : 0.f;
+                } else if (scale_mode == 2) {
+                    sc = row_scale[row];
+                }
+                float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
+#pragma unroll
+                for (int j = 0; j < kTN; j += 4)
+                    dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
+                                             sum[j + 3] * sc);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // neither CTA leaves while the pair's MMAs or arrivals may touch it
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tbase, kPairTmemCols);
+}
+
 // out[p][r][k]: the bf16 pieces of x (fp32), x = out[0] + out[1] + out[2] to
 // ~2^-24 of |x| (each piece the bf16 rounding of what the previous ones left).
 __global__ void k_split3(const float* __restrict__ x, int64_t count, __nv_bfloat16* __restrict__ out) {
@@ -568,7 +789,7 @@ int split_f16x2(const float* x, int64_t count, float scale, __half* out, cudaStr
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb, bool transposed, int n_store, float* tmax,
-                   int64_t ldt, bool fp16) {
+                   int64_t ldt, bool fp16, bool pair_form) {
     if (M <= 0) return TQ_OK;
     if (!gemm_tc_supported(N, K) || pa < 1 || pa > 3 || pb < 1 || pb > 3) return TQ_ERR_ARG;
     if (!transposed && ldc % 4) return TQ_ERR_ARG;
@@ -577,6 +798,28 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     int dev = 0, nsm = 0;
     TQ_TRY_CUDA(cudaGetDevice(&dev));
     TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    if (!transposed && !tmax && N % kPN == 0 && nsm >= 2 && pair_form) {
+        const int64_t ptiles = (int64_t)((M + 2 * kTM - 1) / (2 * kTM)) * (N / kPN);
+        const int npairs = (int)(ptiles < nsm / 2 ? ptiles : nsm / 2);
+        TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemPairBytes));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * npairs));
+        cfg.blockDim = dim3(kPairThreads);
+        cfg.dynamicSmemBytes = kSmemPairBytes;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        TQ_TRY_CUDA(cudaLaunchKernelEx(&cfg, k_gemm_pair, ma, mb, M, N, K, pa, pb, C, ldc,
+                                       row_scale, scale_mode, d_err,
+                                       idesc_f16(fp16 ? 0u : 1u, 2 * kTM, kPN)));
+        return TQ_OK;
+    }
     const int64_t tiles = (int64_t)((M + kTM - 1) / kTM) * (N / kTN);
     const int nctas = (int)(tiles < nsm ? tiles : nsm);
     TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,

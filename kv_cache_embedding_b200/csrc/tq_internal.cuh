@@ -104,7 +104,8 @@ bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n)
 // Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from
 // 16-bit pieces of A ([pa][M][K]) and B ([pb][N][K]) -- bf16, or fp16 with
 // `fp16` (the pointers then address __half data); d_err as the encode
-// kernels' status word.
+// kernels' status word.  Row-major products with N % 256 == 0 run on CTA
+// pairs (256 x 256 tiles) unless pair_form is false.
 bool gemm_tc_supported(int N, int K);
 int split_bf16x3(const float* x, int64_t count, __nv_bfloat16* out, cudaStream_t s);
 // fp16 pieces [2][count] of scale * x (scale a power of two).
@@ -112,7 +113,8 @@ int split_f16x2(const float* x, int64_t count, float scale, __half* out, cudaStr
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb = 3, bool transposed = false, int n_store = 0,
-                   float* tmax = nullptr, int64_t ldt = 0, bool fp16 = false);
+                   float* tmax = nullptr, int64_t ldt = 0, bool fp16 = false,
+                   bool pair_form = true);
 // A operand decoded from code records inside the GEMM (scoring of many
 // queries): row m of A = (c[idx] | kappa_m (2z - 1)) over K = 2d as bf16
 // pieces hi, lo (kappa_m = kscale |r_m|; the MSE-only variant has c[cell] and
