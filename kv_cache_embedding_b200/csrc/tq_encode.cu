@@ -91,36 +91,59 @@ __global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
 // One warp per row: bucketize each rotated coordinate, the cell index to a byte
 // array, |r|, and the fp16 pieces of rscale * r (r = y - c[idx]) -- hi to
 // rp[0], lo to rp[1] -- as the operand of the QJL product.  Coordinates from
-// `half` on take the second grid of a fractional width (c_lo, beta_lo).
-__global__ void k_quantize16(const float* __restrict__ yr, uint8_t* __restrict__ idx, int64_t rows,
-                             int d, KCodebook cb, float rscale, float* __restrict__ rnorm,
-                             __half* __restrict__ rp, int half) {
+// `half` on take the second grid of a fractional width (c_lo, beta_lo).  A
+// lane takes 4 consecutive coordinates per step (16-byte loads, 4-byte cell
+// and 8-byte piece stores; d and `half` are multiples of 4); the grids sit in
+// shared memory, read as broadcasts.
+__global__ void __launch_bounds__(256)
+k_quantize16(const float* __restrict__ yr, uint8_t* __restrict__ idx, int64_t rows, int d,
+             KCodebook cb, float rscale, float* __restrict__ rnorm, __half* __restrict__ rp,
+             int half) {
+    __shared__ float s_c[2][16], s_b[2][16];
+    if (threadIdx.x < 16) {
+        s_c[0][threadIdx.x] = cb.c[threadIdx.x];
+        s_b[0][threadIdx.x] = cb.beta[threadIdx.x];
+    } else if (threadIdx.x < 32) {
+        s_c[1][threadIdx.x - 16] = cb.c_lo[threadIdx.x - 16];
+        s_b[1][threadIdx.x - 16] = cb.beta_lo[threadIdx.x - 16];
+    }
+    __syncthreads();
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     if (row >= rows) return;
-    const float* y = yr + row * d;
-    uint8_t* ix = idx + row * d;
-    __half* hi = rp + row * d;
-    __half* lo = rp + rows * d + row * d;
+    const float4* y = reinterpret_cast<const float4*>(yr + row * d);
+    uint32_t* ix = reinterpret_cast<uint32_t*>(idx + row * d);
+    uint2* hi = reinterpret_cast<uint2*>(rp + row * d);
+    uint2* lo = reinterpret_cast<uint2*>(rp + rows * d + row * d);
     float rr = 0.f;
-    for (int i = lane; i < d; i += 32) {
-        const float v = y[i];
-        const bool second = i >= half;  // the second grid of a fractional width
-        const int levels = second ? cb.levels_lo : cb.levels;
-        int cell = 0;
-        float r = v;
-        if (levels > 0) {
+    for (int i4 = lane; i4 < d / 4; i4 += 32) {
+        const float4 v4 = y[i4];
+        const int g = (4 * i4 >= half) ? 1 : 0;  // the second grid of a fractional width
+        const int levels = g ? cb.levels_lo : cb.levels;
+        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+        uint32_t cells = 0u;
+        __half h[4], l[4];
 #pragma unroll
-            for (int j = 0; j < 15; ++j)
-                if (j + 1 < levels && (second ? cb.beta_lo[j] : cb.beta[j]) <= v) ++cell;
-            r = v - (second ? cb.c_lo[cell] : cb.c[cell]);
+        for (int e = 0; e < 4; ++e) {
+            int cell = 0;
+            float r = v[e];
+            if (levels > 0) {
+#pragma unroll
+                for (int j = 0; j < 15; ++j)
+                    if (j + 1 < levels && s_b[g][j] <= v[e]) ++cell;
+                r = v[e] - s_c[g][cell];
+            }
+            cells |= (uint32_t)cell << (8 * e);
+            rr = fmaf(r, r, rr);
+            const float t = r * rscale;  // exact: a power of two
+            h[e] = __float2half_rn(t);
+            l[e] = __float2half_rn(t - __half2float(h[e]));
         }
-        ix[i] = (uint8_t)cell;
-        rr = fmaf(r, r, rr);
-        const float t = r * rscale;  // exact: a power of two
-        const __half h = __float2half_rn(t);
-        hi[i] = h;
-        lo[i] = __float2half_rn(t - __half2float(h));
+        ix[i4] = cells;
+        hi[i4] = make_uint2((uint32_t)__half_as_ushort(h[0]) | ((uint32_t)__half_as_ushort(h[1]) << 16),
+                            (uint32_t)__half_as_ushort(h[2]) | ((uint32_t)__half_as_ushort(h[3]) << 16));
+        lo[i4] = make_uint2((uint32_t)__half_as_ushort(l[0]) | ((uint32_t)__half_as_ushort(l[1]) << 16),
+                            (uint32_t)__half_as_ushort(l[2]) | ((uint32_t)__half_as_ushort(l[3]) << 16));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) rr += __shfl_xor_sync(0xffffffffu, rr, o);

@@ -512,12 +512,6 @@ struct SmemP {
 };
 constexpr size_t kSmemPairBytes = sizeof(SmemP) + 1024;
 
-__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
-    const bool ok = mbar_wait_cluster(bar, parity, abort, kWaitNs);
-    return __all_sync(0xffffffffu, ok);
-}
-
 __global__ void __launch_bounds__(kPairThreads, 1)
 k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
             int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
@@ -577,7 +571,7 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = (int)(it % (uint32_t)ns);
                 if (it >= (uint32_t)ns &&
-                    !mbar_wait_cluster(&sm.empty[s], ((it / ns) - 1) & 1, abort, kWaitNs)) {
+                    !mbar_wait(&sm.empty[s], ((it / ns) - 1) & 1, abort, kWaitNs)) {
                     ok = give_up(abort, err, 51);
                     break;
                 }
@@ -612,7 +606,7 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             for (int c = 0; c < nch && ok; ++c, ++cc) {
                 const uint32_t ab = cc & 1;
                 if (cc >= 2 &&
-                    !mbar_wait_cluster(&sm.acc_empty[ab], ((cc >> 1) - 1) & 1, abort, kWaitNs)) {
+                    !mbar_wait(&sm.acc_empty[ab], ((cc >> 1) - 1) & 1, abort, kWaitNs)) {
                     ok = give_up(abort, err, 52);
                     break;
                 }
@@ -644,7 +638,7 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
     } else if (warp == 1 && lane == 0) {
         // the leader's MMAs write this CTA's tensor memory and read its stages
-        mbar_wait_cluster(&sm.mma_done, 0, &sm.zero, kWaitNs);
+        mbar_wait(&sm.mma_done, 0, &sm.zero, kWaitNs);
     } else if (warp >= 4) {
         // ---------------- chunk sums and stores (both CTAs) ----------------
         const int q = warp & 3;               // TMEM lane quarter: rows 32 q .. 32 q + 31
@@ -662,7 +656,7 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             for (int j = 0; j < kTN; ++j) sum[j] = 0.f;
             for (int c = 0; c < nch; ++c, ++cc) {
                 const uint32_t ab = cc & 1;
-                if (!warp_wait_cluster(&sm.acc_full[ab], (cc >> 1) & 1, abort)) {
+                if (!warp_wait(&sm.acc_full[ab], (cc >> 1) & 1, abort)) {
                     ok = give_up(abort, err, 54);
                     break;
                 }

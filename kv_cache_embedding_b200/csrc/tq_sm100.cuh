@@ -65,26 +65,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// The same, acquiring at cluster scope: for mbarriers that the other CTA of
-// a pair arrives on.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer();
-    while (true) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.b32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
-            : "memory");
-        if (ok) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > limit_ns) return false;
-    }
-}
-
 // ---- TMA ---------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
                                             int32_t y, uint64_t* bar) {
@@ -320,10 +300,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 }
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly the
-// other CTA's), releasing this thread's prior accesses at cluster scope.
+// other CTA's).  The epilogue arrives after tcgen05.wait::ld, so its tensor
+// memory reads are complete; no cluster-scope fence is needed.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 
 // All threads of both CTAs; orders the barrier inits and tensor-memory
