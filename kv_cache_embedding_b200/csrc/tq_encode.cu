@@ -282,6 +282,12 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
     // the rotation and QJL products on the tensor cores, else fp32 SIMT GEMMs
     const bool tcg = gemm_tc_supported(d, d);
     if (split && !tcg) return TQ_ERR_UNSUPPORTED;  // the SIMT fallback has one grid
+    // inner-product records at d % 256 == 0: the CTA-pair GEMMs with the
+    // bucketize and packing in their epilogues
+    int nsm_dev = 0, dev_id = 0;
+    TQ_TRY_CUDA(cudaGetDevice(&dev_id));
+    TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm_dev, cudaDevAttrMultiProcessorCount, dev_id));
+    const bool fused = tcg && !mse && d % 256 == 0 && nsm_dev >= 2;
     // tensor-core GEMMs: fp16 pieces [2][d][d] of 2^8 Pi_g and of 2^4 S_g, the
     // chunk's operand pieces [2][chunk][d] (x, then r) and its row scales
     __half* PiP = (__half*)(IX + align256((size_t)chunk * d));
@@ -316,6 +322,34 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                     k_rownorm_split16<__nv_bfloat16><<<wblocks, 256, 0, s>>>(
                         (const __nv_bfloat16*)xg, rows, d, xn, RS, AP);
                 TQ_CHECK_LAUNCH();
+                if (fused) {
+                    // the bucketize in the rotation's epilogue (cells, pieces of
+                    // r in Y's space, |r|^2 partials in P's), the packing in the
+                    // QJL product's: Y and P never reach HBM
+                    uint32_t* cgf = d_codes + (size_t)off * W;
+                    EncodeEpi e1 = {};
+                    e1.mode = 1;
+                    e1.b = b;
+                    e1.rscale = rscale;
+                    e1.idx = IX;
+                    e1.rp = (__half*)Y;
+                    e1.rn2 = P;
+                    e1.cb = kc;
+                    rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP,
+                                        x_dtype == TQ_F32 ? 2 : 1, (const __nv_bfloat16*)PiP,
+                                        nullptr, d, RS, 1, err, s, 2, false, 0, nullptr, 0, true,
+                                        true, &e1);
+                    if (rc) return rc;
+                    EncodeEpi e2 = e1;
+                    e2.mode = 2;
+                    e2.codes = cgf;
+                    e2.rnorm = rn;
+                    rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)Y, 2,
+                                        (const __nv_bfloat16*)SP, nullptr, d, nullptr, 0, err, s,
+                                        2, false, 0, nullptr, 0, true, true, &e2);
+                    if (rc) return rc;
+                    continue;
+                }
                 rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP,
                                     x_dtype == TQ_F32 ? 2 : 1, (const __nv_bfloat16*)PiP, Y, d, RS,
                                     1, err, s, 2, false, 0, nullptr, 0, true);

@@ -505,6 +505,8 @@ constexpr uint32_t kPairEpiWarps = 8;
 
 struct SmemP {
     uint8_t pool[kPool][kPieceBytes];  // stage s: A's pa pieces, then B's pb (1024-aligned)
+    float g_c[2][16], g_b[2][16];      // encode epilogues: the grids (second: fractional width)
+    int g_levels[2];
     uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done;
     uint32_t tmem_base;
     int abort;
@@ -512,11 +514,92 @@ struct SmemP {
 };
 constexpr size_t kSmemPairBytes = sizeof(SmemP) + 1024;
 
+// Rotation epilogue: coordinates n0 .. n0 + 127 of row `row`, y = sum * sc:
+// the cell (the count of boundaries <= y, by binary search over the sorted
+// grid of 2^k levels), r = y - c[cell], the fp16 pieces of rscale * r and the
+// segment's |r|^2 -- the arithmetic of k_quantize16, per coordinate.
+__device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, const SmemP& sm,
+                                             const EncodeEpi& ep, int M, int N, int64_t row,
+                                             int n0) {
+    const int g = (ep.cb.split && n0 >= N / 2) ? 1 : 0;
+    const int L = sm.g_levels[g];
+    const float* bt = sm.g_b[g];
+    const float* ct = sm.g_c[g];
+    uint8_t* ix = ep.idx + row * N + n0;
+    __half* hi = ep.rp + row * N + n0;
+    __half* lo = ep.rp + (int64_t)M * N + row * N + n0;
+    float rr = 0.f;
+#pragma unroll
+    for (int j0 = 0; j0 < kTN; j0 += 8) {
+        uint32_t cw[2] = {0u, 0u}, hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float y = sum[j0 + e] * sc;
+            int cell = 0;
+            float r = y;
+            if (L > 0) {
+                for (int step = L >> 1; step > 0; step >>= 1)
+                    if (bt[cell + step - 1] <= y) cell += step;
+                r = y - ct[cell];
+            }
+            cw[e >> 2] |= (uint32_t)cell << (8 * (e & 3));
+            rr = fmaf(r, r, rr);
+            const float t = r * ep.rscale;  // exact: a power of two
+            const __half h = __float2half_rn(t);
+            const __half l = __float2half_rn(t - __half2float(h));
+            hw[e >> 1] |= (uint32_t)__half_as_ushort(h) << (16 * (e & 1));
+            lw[e >> 1] |= (uint32_t)__half_as_ushort(l) << (16 * (e & 1));
+        }
+        *reinterpret_cast<uint2*>(ix + j0) = make_uint2(cw[0], cw[1]);
+        *reinterpret_cast<uint4*>(hi + j0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lo + j0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    ep.rn2[(int64_t)(n0 / kTN) * M + row] = rr;
+}
+
+// QJL epilogue: coordinates n0 .. n0 + 127 (4 blocks of 32) of row `row` --
+// z = [P >= 0] with the cells into 4 blocks of BB words at `rec` (the record
+// layout of width BB: a sign plane; 2-bit [idx | z] fields; 2-bit idx fields
+// and a sign plane; 4-bit [idx | z] nibbles).
+template <int BB>
+__device__ __forceinline__ void epi_pack(const float (&sum)[kTN], const uint8_t* cells,
+                                         uint32_t* rec) {
+    uint32_t out[4 * BB];
+#pragma unroll
+    for (int i = 0; i < 4 * BB; ++i) out[i] = 0u;
+    const uint4* cp = reinterpret_cast<const uint4*>(cells);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint4 c0 = cp[2 * w], c1 = cp[2 * w + 1];
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t cell = (cw[j >> 2] >> (8 * (j & 3))) & 0xFFu;
+            const uint32_t z = sum[32 * w + j] >= 0.f ? 1u : 0u;
+            if (BB == 1) {
+                out[w] |= z << j;
+            } else if (BB == 2) {
+                out[2 * w + (j >> 4)] |= ((cell & 1u) | (z << 1)) << (2 * (j & 15));
+            } else if (BB == 3) {
+                out[3 * w + (j >> 4)] |= (cell & 3u) << (2 * (j & 15));
+                out[3 * w + 2] |= z << j;
+            } else {
+                out[4 * w + (j >> 3)] |= ((cell & 7u) | (z << 3)) << (4 * (j & 7));
+            }
+        }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(rec);
+#pragma unroll
+    for (int i = 0; i < BB; ++i)
+        dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+}
+
+template <int EPI>
 __global__ void __launch_bounds__(kPairThreads, 1)
 k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
             int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
             const float* __restrict__ row_scale, int scale_mode, int* __restrict__ err,
-            uint32_t idesc) {
+            uint32_t idesc, const __grid_constant__ EncodeEpi ep) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     // the same offset in both CTAs: the MMA reads the peer's operands there
@@ -546,6 +629,20 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         sm.abort = 0;
         sm.zero = 0;
         fence_mbar_init();
+    }
+    if (EPI != 0 && threadIdx.x >= 32 && threadIdx.x < 64) {
+        const int i = threadIdx.x - 32;
+        if (i < 16) {
+            sm.g_c[0][i] = ep.cb.c[i];
+            sm.g_b[0][i] = ep.cb.beta[i];
+        } else {
+            sm.g_c[1][i - 16] = ep.cb.c_lo[i - 16];
+            sm.g_b[1][i - 16] = ep.cb.beta_lo[i - 16];
+        }
+        if (i == 0) {
+            sm.g_levels[0] = ep.cb.levels;
+            sm.g_levels[1] = ep.cb.levels_lo;
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(&sm.tmem_base, kPairTmemCols);
@@ -683,11 +780,36 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
                 } else if (scale_mode == 2) {
                     sc = row_scale[row];
                 }
-                float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
+                if constexpr (EPI == 0) {
+                    float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
 #pragma unroll
-                for (int j = 0; j < kTN; j += 4)
-                    dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
-                                             sum[j + 3] * sc);
+                    for (int j = 0; j < kTN; j += 4)
+                        dst[j / 4] = make_float4(sum[j] * sc, sum[j + 1] * sc, sum[j + 2] * sc,
+                                                 sum[j + 3] * sc);
+                } else if constexpr (EPI == 1) {
+                    epi_quantize(sum, sc, sm, ep, M, N, row, n0);
+                } else {
+                    // the record words of these 4 blocks: width b, or for a
+                    // fractional width b in the first half and b - 1 after
+                    const int b = ep.b;
+                    const bool second = ep.cb.split && n0 >= N / 2;
+                    const int W = ep.cb.split ? N / 64 * (2 * b - 1) : b * N / 32;
+                    const int wb = n0 / 32;
+                    const int off = !second ? wb * b : (N / 64) * b + (wb - N / 64) * (b - 1);
+                    uint32_t* rec = ep.codes + row * W + off;
+                    const uint8_t* cells = ep.idx + row * N + n0;
+                    switch (second ? b - 1 : b) {
+                        case 1: epi_pack<1>(sum, cells, rec); break;
+                        case 2: epi_pack<2>(sum, cells, rec); break;
+                        case 3: epi_pack<3>(sum, cells, rec); break;
+                        default: epi_pack<4>(sum, cells, rec); break;
+                    }
+                    if (n0 == 0) {  // |r| from the rotation epilogue's partial sums, in order
+                        float rr = 0.f;
+                        for (int t = 0; t < N / kTN; ++t) rr += ep.rn2[(int64_t)t * M + row];
+                        ep.rnorm[row] = sqrtf(rr);
+                    }
+                }
             }
         }
     }
@@ -783,7 +905,7 @@ int split_f16x2(const float* x, int64_t count, float scale, __half* out, cudaStr
 int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __nv_bfloat16* B,
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb, bool transposed, int n_store, float* tmax,
-                   int64_t ldt, bool fp16, bool pair_form) {
+                   int64_t ldt, bool fp16, bool pair_form, const EncodeEpi* epi) {
     if (M <= 0) return TQ_OK;
     if (!gemm_tc_supported(N, K) || pa < 1 || pa > 3 || pb < 1 || pb > 3) return TQ_ERR_ARG;
     if (!transposed && ldc % 4) return TQ_ERR_ARG;
@@ -792,10 +914,14 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     int dev = 0, nsm = 0;
     TQ_TRY_CUDA(cudaGetDevice(&dev));
     TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
+    const int epi_mode = epi ? epi->mode : 0;
+    if (epi_mode != 0 && (transposed || tmax || N % kPN != 0 || nsm < 2 || !pair_form))
+        return TQ_ERR_ARG;
     if (!transposed && !tmax && N % kPN == 0 && nsm >= 2 && pair_form) {
         const int64_t ptiles = (int64_t)((M + 2 * kTM - 1) / (2 * kTM)) * (N / kPN);
         const int npairs = (int)(ptiles < nsm / 2 ? ptiles : nsm / 2);
-        TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        auto kern = epi_mode == 1 ? k_gemm_pair<1> : epi_mode == 2 ? k_gemm_pair<2> : k_gemm_pair<0>;
+        TQ_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemPairBytes));
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * npairs));
@@ -809,9 +935,11 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        TQ_TRY_CUDA(cudaLaunchKernelEx(&cfg, k_gemm_pair, ma, mb, M, N, K, pa, pb, C, ldc,
-                                       row_scale, scale_mode, d_err,
-                                       idesc_f16(fp16 ? 0u : 1u, 2 * kTM, kPN)));
+        EncodeEpi e = {};
+        if (epi) e = *epi;
+        TQ_TRY_CUDA(cudaLaunchKernelEx(&cfg, kern, ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
+                                       scale_mode, d_err, idesc_f16(fp16 ? 0u : 1u, 2 * kTM, kPN),
+                                       e));
         return TQ_OK;
     }
     const int64_t tiles = (int64_t)((M + kTM - 1) / kTM) * (N / kTN);

@@ -102,6 +102,22 @@ int check_common(const tq_codebook_t* cb, int G, int64_t n, int nq, int q_dtype)
 size_t attn_workspace_bytes(int b, int G, int64_t n, int nq);
 bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n);
 // Split-precision tcgen05 GEMM (tq_gemm_tc.cu): C = scale(m) * A B^T from
+// Encode epilogues of the CTA-pair GEMM over one chunk of M rows (N = K = d,
+// d % 256 == 0, inner-product records).  Mode 1, on the rotation product:
+// bucketize y = C, write the cells, the fp16 pieces of rscale * r and |r|^2 of
+// every 128 coordinates.  Mode 2, on the QJL product: the signs of C with the
+// cells -> code records, and |r| from the partial sums.  Mode 0 stores C.
+struct EncodeEpi {
+    int mode;
+    int b;
+    float rscale;      // power of two
+    uint8_t* idx;      // [M][d] cells (mode 1 writes, mode 2 reads)
+    __half* rp;        // [2][M][d] fp16 pieces hi, lo of rscale * r (mode 1)
+    float* rn2;        // [d/128][M] |r|^2 per 128 coordinates (mode 1 writes, mode 2 sums)
+    float* rnorm;      // [M] |r| (mode 2)
+    uint32_t* codes;   // [M][record words] (mode 2)
+    KCodebook cb;
+};
 // 16-bit pieces of A ([pa][M][K]) and B ([pb][N][K]) -- bf16, or fp16 with
 // `fp16` (the pointers then address __half data); d_err as the encode
 // kernels' status word.  Row-major products with N % 256 == 0 run on CTA
@@ -114,7 +130,7 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
                    float* C, int64_t ldc, const float* row_scale, int scale_mode, int* d_err,
                    cudaStream_t s, int pb = 3, bool transposed = false, int n_store = 0,
                    float* tmax = nullptr, int64_t ldt = 0, bool fp16 = false,
-                   bool pair_form = true);
+                   bool pair_form = true, const EncodeEpi* epi = nullptr);
 // A operand decoded from code records inside the GEMM (scoring of many
 // queries): row m of A = (c[idx] | kappa_m (2z - 1)) over K = 2d as bf16
 // pieces hi, lo (kappa_m = kscale |r_m|; the MSE-only variant has c[cell] and
