@@ -531,24 +531,30 @@ __device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, 
     float rr = 0.f;
 #pragma unroll
     for (int j0 = 0; j0 < kTN; j0 += 8) {
-        uint32_t cw[2] = {0u, 0u}, hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+        uint32_t cw[2] = {0u, 0u}, hw[4], lw[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float y = sum[j0 + e] * sc;
-            int cell = 0;
-            float r = y;
-            if (L > 0) {
-                for (int step = L >> 1; step > 0; step >>= 1)
-                    if (bt[cell + step - 1] <= y) cell += step;
-                r = y - ct[cell];
+        for (int e = 0; e < 8; e += 2) {
+            float t[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float y = sum[j0 + e + u] * sc;
+                int cell = 0;
+                float r = y;
+                if (L > 0) {
+                    for (int step = L >> 1; step > 0; step >>= 1)
+                        if (bt[cell + step - 1] <= y) cell += step;
+                    r = y - ct[cell];
+                }
+                cw[e >> 2] |= (uint32_t)cell << (8 * ((e + u) & 3));
+                rr = fmaf(r, r, rr);
+                t[u] = r * ep.rscale;  // exact: a power of two
             }
-            cw[e >> 2] |= (uint32_t)cell << (8 * (e & 3));
-            rr = fmaf(r, r, rr);
-            const float t = r * ep.rscale;  // exact: a power of two
-            const __half h = __float2half_rn(t);
-            const __half l = __float2half_rn(t - __half2float(h));
-            hw[e >> 1] |= (uint32_t)__half_as_ushort(h) << (16 * (e & 1));
-            lw[e >> 1] |= (uint32_t)__half_as_ushort(l) << (16 * (e & 1));
+            // two coordinates' pieces at once (round to nearest, as __float2half_rn)
+            const __half2 h = __floats2half2_rn(t[0], t[1]);
+            const float2 hf = __half22float2(h);
+            const __half2 l = __floats2half2_rn(t[0] - hf.x, t[1] - hf.y);
+            hw[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            lw[e >> 1] = *reinterpret_cast<const uint32_t*>(&l);
         }
         *reinterpret_cast<uint2*>(ix + j0) = make_uint2(cw[0], cw[1]);
         *reinterpret_cast<uint4*>(hi + j0) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
