@@ -13,14 +13,12 @@
 //
 // Design: the logits come from tq_score itself (its scoring kernels for the
 // group's query count) into the workspace; then split-K over the keys of a
-// group (flash-decoding).  A block takes `split` keys in tiles of 256, keeps a
-// running maximum and sum per query, and
-// accumulates sum_j p_j |v_j| c_v[cell_j] in the rotated value domain: thread
-// (coordinate pair, quarter of the tile) walks the tile's value records staged
-// in shared memory and updates both coordinates with packed fp32x2 FMAs (at
-// b_v = 4 one byte-indexed table load gives both centroids).  Because Pi_v^T
-// is linear it is applied once per query, after the splits are merged
-// (k_attn_combine), instead of once per value.
+// group (flash-decoding).  A block takes `split` keys: the split's maximum per
+// query first, then in tiles of 256 the weights e^(l - M) |v_j| and
+// sum_j w_j c_v[cell_j] in the rotated value domain, a thread owning 8
+// coordinates (one code word of every record) and a sixteenth of the keys.
+// Because Pi_v^T is linear it is applied once per query, after the splits are
+// merged (k_attn_combine), instead of once per value.
 #include <cmath>
 
 #include "tq_internal.cuh"
@@ -45,18 +43,28 @@ __device__ __forceinline__ uint32_t value_cell(const uint32_t* blk, int j) {
     return (blk[0] >> j) & 1u;
 }
 
+// One split of `split` keys of group g for queries q0 .. q0 + NQ - 1:
+//   M_q = max_j l_qj over the split (one pass over its logits, so the
+//         weights need no rescaling as the tiles go by),
+//   w_qj = e^(l_qj - M_q) |v_j|,  L_q = sum_j e^(l_qj - M_q),
+//   acc_q = sum_j w_qj c_v[cell_j]   (the rotated value domain).
+// Per tile of 256 keys, thread t forms key t's weights (shared memory); then
+// thread (8-coordinate word wi = t % 16, key lane kl = t / 16) walks keys
+// kl, kl + 16, ... of the tile: one code word of the record (coalesced: 16
+// threads read one record), 8 centroids from a 16-entry table (one entry per
+// bank: no conflicts), 16 packed fp32x2 FMAs for the 4 queries.  The 16 key
+// lanes' sums are merged once per split.
 template <int BV, int NQ>
-__global__ __launch_bounds__(kAT, 8) void k_attn_partial(
+__global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     const float* __restrict__ logits, const uint32_t* __restrict__ vcodes,
     const float* __restrict__ vxn, int64_t n, int nq, KCodebook vcb, float scale, int split,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_acc) {
-    constexpr int WV = BV * kAD / 32;
+    constexpr int WV = BV * kAD / 32;  // record words
     __shared__ float s_vc[16];
     __shared__ float2 s_vpair[256];  // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble])
-    __shared__ uint32_t s_vcodes[kAT * WV];
-    __shared__ __align__(16) float s_w[kAT][NQ];
-    __shared__ float s_red[kAT / 32][NQ];
-    __shared__ float2 s_part[3][NQ][kAD / 2];
+    __shared__ __align__(16) float s_w[kAT][4];
+    __shared__ float s_red[kAT / 32][4];
+    __shared__ float2 s_acc[16][4][NQ][16];  // [key lane][coordinate pair of the word][query][word]
     const int g = blockIdx.y, sp = blockIdx.x, nsplit = gridDim.x;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
@@ -73,119 +81,132 @@ __global__ __launch_bounds__(kAT, 8) void k_attn_partial(
     }
     __syncthreads();
     if (BV == 4) s_vpair[t] = make_float2(s_vc[t & 15], s_vc[t >> 4]);
-
     const int64_t r_beg = (int64_t)sp * split;
     const int64_t r_end = min(n, r_beg + split);
-    // value phase: coordinates 2 cp, 2 cp + 1 over quarter hq of every tile
-    const int cp = t % (kAD / 2), hq = t / (kAD / 2);
-    const int vblk = (2 * cp) / 32, vj = (2 * cp) % 32;
-    float M[NQ], L[NQ];
-    float2 accv[NQ];
+    const float* lg[NQ];
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-        M[q] = -INFINITY;
-        L[q] = 0.f;
-        accv[q] = make_float2(0.f, 0.f);
-    }
-    for (int64_t r = r_beg; r < r_end; r += kAT) {
-        const int cnt = (int)min((int64_t)kAT, r_end - r);
-        const int64_t j = r + t;
-        const bool ok = t < cnt;
-        const int64_t gj = (int64_t)g * n + (ok ? j : r);
-        // scaled logits of this thread's key
-        float l[NQ];
+    for (int q = 0; q < NQ; ++q) lg[q] = logits + ((int64_t)g * nq + q0 + (q < qn ? q : 0)) * n;
+
+    // ---- the split's maximum per query
+    float M[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) M[q] = -INFINITY;
+    for (int64_t j = r_beg + t; j < r_end; j += kAT)
 #pragma unroll
         for (int q = 0; q < NQ; ++q)
-            l[q] = (ok && q < qn) ? scale * logits[((int64_t)g * nq + q0 + q) * n + j] : -INFINITY;
-        // the tile's value records, staged whole (coalesced)
-        const uint32_t* vsrc = vcodes + ((int64_t)g * n + r) * WV;
-        for (int e = t; e < cnt * WV; e += kAT) s_vcodes[e] = vsrc[e];
-        const float vx = ok ? vxn[gj] : 0.f;
-        // running maximum per query
+            if (q < qn) M[q] = fmaxf(M[q], scale * lg[q][j]);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            float m = l[q];
+    for (int q = 0; q < NQ; ++q) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) s_red[warp][q] = m;
-        }
-        __syncthreads();
-        float alpha[NQ], p[NQ];
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            float mt = s_red[0][q];
-#pragma unroll
-            for (int w = 1; w < kAT / 32; ++w) mt = fmaxf(mt, s_red[w][q]);
-            const float mn = fmaxf(M[q], mt);
-            alpha[q] = (M[q] == -INFINITY) ? 0.f : __expf(M[q] - mn);
-            M[q] = mn;
-            p[q] = ok ? __expf(l[q] - mn) : 0.f;
-            s_w[t][q] = p[q] * vx;
-        }
-        __syncthreads();  // every thread has read s_red (maxima) and written s_w
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            float ps = p[q];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-            if (lane == 0) s_red[warp][q] = ps;
-        }
-        // value sums of this thread's coordinate pair over its quarter of the tile
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            accv[q].x *= alpha[q];
-            accv[q].y *= alpha[q];
-        }
-        const int jj1 = min(cnt, kAT / 4 * (hq + 1));
-        for (int jj = kAT / 4 * hq; jj < jj1; ++jj) {
-            const uint32_t* blk = s_vcodes + jj * WV + vblk * BV;
-            float2 c2;
-            if (BV == 4) {
-                c2 = s_vpair[__byte_perm(blk[vj >> 3], 0u, 0x4440u | ((vj >> 1) & 3))];
-            } else {
-                c2 = make_float2(s_vc[value_cell<BV>(blk, vj)], s_vc[value_cell<BV>(blk, vj + 1)]);
-            }
-            if (NQ == 4) {
-                const float4 w4 = *reinterpret_cast<const float4*>(&s_w[jj][0]);
-                accv[0] = ffma2(make_float2(w4.x, w4.x), c2, accv[0]);
-                accv[1 % NQ] = ffma2(make_float2(w4.y, w4.y), c2, accv[1 % NQ]);
-                accv[2 % NQ] = ffma2(make_float2(w4.z, w4.z), c2, accv[2 % NQ]);
-                accv[3 % NQ] = ffma2(make_float2(w4.w, w4.w), c2, accv[3 % NQ]);
-            } else {
-#pragma unroll
-                for (int q = 0; q < NQ; ++q)
-                    accv[q] = ffma2(make_float2(s_w[jj][q], s_w[jj][q]), c2, accv[q]);
-            }
-        }
-        __syncthreads();  // s_red holds the tile sums; s_vcodes / s_w may be reused
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            float ts = 0.f;
-#pragma unroll
-            for (int w = 0; w < kAT / 32; ++w) ts += s_red[w][q];
-            L[q] = L[q] * alpha[q] + ts;
-        }
-        __syncthreads();  // s_red is rewritten by the next tile
-    }
-    // merge the four quarters of every coordinate pair and write the split's partials
-    if (hq > 0) {
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) s_part[hq - 1][q][cp] = accv[q];
+        for (int o = 16; o > 0; o >>= 1) M[q] = fmaxf(M[q], __shfl_xor_sync(0xffffffffu, M[q], o));
+        if (lane == 0) s_red[warp][q] = M[q];
     }
     __syncthreads();
-    if (hq == 0) {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-            if (q >= qn) continue;
-            const int64_t row = (int64_t)g * nq + q0 + q;
-            const float2 a1 = s_part[0][q][cp], a2 = s_part[1][q][cp], a3 = s_part[2][q][cp];
-            const float2 sum = make_float2((accv[q].x + a1.x) + (a2.x + a3.x),
-                                           (accv[q].y + a1.y) + (a2.y + a3.y));
-            *reinterpret_cast<float2*>(&part_acc[(row * nsplit + sp) * kAD + 2 * cp]) = sum;
-            if (cp == 0) {
-                part_m[row * nsplit + sp] = M[q];
-                part_l[row * nsplit + sp] = L[q];
+    for (int q = 0; q < NQ; ++q) {
+        float m = s_red[0][q];
+#pragma unroll
+        for (int w = 1; w < kAT / 32; ++w) m = fmaxf(m, s_red[w][q]);
+        M[q] = m;
+    }
+
+    const int wi = t % 16, kl = t / 16;
+    float2 acc[4][NQ];  // coordinates 8 wi + 2 e, 8 wi + 2 e + 1
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) acc[e][q] = make_float2(0.f, 0.f);
+    float Lp[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) Lp[q] = 0.f;
+    const uint32_t* vg = vcodes + (int64_t)g * n * WV;
+    const float* vxg = vxn + (int64_t)g * n;
+    for (int64_t r = r_beg; r < r_end; r += kAT) {
+        const int cnt = (int)min((int64_t)kAT, r_end - r);
+        // the weights of key r + t
+        {
+            const bool ok = t < cnt;
+            const float vx = ok ? vxg[r + t] : 0.f;
+            float w4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const float pq = (ok && q < qn) ? __expf(scale * lg[q][r + t] - M[q]) : 0.f;
+                Lp[q] += pq;
+                w4[q] = pq * vx;
             }
+            *reinterpret_cast<float4*>(&s_w[t][0]) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        __syncthreads();  // s_w complete
+        // this thread's code word(s) of the tile's keys kl, kl + 16, ..., in two
+        // batches of 8 loads
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+            uint32_t cw[8][BV == 4 ? 1 : BV];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int key = kl + 16 * (8 * hb + kk);
+                const int64_t v = r + (key < cnt ? key : 0);
+#pragma unroll
+                for (int i = 0; i < (BV == 4 ? 1 : BV); ++i)
+                    cw[kk][i] = __ldg(vg + v * WV + (BV == 4 ? wi : (wi >> 2) * BV + i));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int key = kl + 16 * (8 * hb + kk);
+                if (key < cnt) {
+                    const float4 w = *reinterpret_cast<const float4*>(&s_w[key][0]);
+                    const float wq[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float2 c2;
+                        if (BV == 4) {  // one code byte = one coordinate pair
+                            c2 = s_vpair[__byte_perm(cw[kk][0], 0u, 0x4440u | e)];
+                        } else {
+                            const int j = 8 * (wi & 3) + 2 * e;
+                            c2 = make_float2(s_vc[value_cell<BV>(cw[kk], j)],
+                                             s_vc[value_cell<BV>(cw[kk], j + 1)]);
+                        }
+#pragma unroll
+                        for (int q = 0; q < NQ; ++q)
+                            acc[e][q] = ffma2(make_float2(wq[q], wq[q]), c2, acc[e][q]);
+                    }
+                }
+            }
+        }
+        __syncthreads();  // s_w is rewritten by the next tile
+    }
+    // ---- merge the 16 key lanes; the split's sums per query
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) s_acc[kl][e][q][wi] = acc[e][q];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        float ls = Lp[q];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+        if (lane == 0) s_red[warp][q] = ls;
+    }
+    __syncthreads();
+    // output o = ((q * 4 + e) * 16 + wi) * 2 + u is coordinate k = 8 wi + 2 e + u
+    for (int o = t; o < kAD * NQ; o += kAT) {
+        const int u = o & 1, wo = (o >> 1) & 15, e = (o >> 5) & 3, q = o >> 7;
+        const int k = 8 * wo + 2 * e + u;
+        if (q >= qn) continue;
+        float a = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+            const float2 v = s_acc[l][e][q][wo];
+            a += u ? v.y : v.x;
+        }
+        const int64_t row = (int64_t)g * nq + q0 + q;
+        part_acc[(row * nsplit + sp) * kAD + k] = a;
+        if (k == 0) {
+            float ls = 0.f;
+#pragma unroll
+            for (int w = 0; w < kAT / 32; ++w) ls += s_red[w][q];
+            part_m[row * nsplit + sp] = M[q];
+            part_l[row * nsplit + sp] = ls;
         }
     }
 }
