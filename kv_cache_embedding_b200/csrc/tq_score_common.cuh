@@ -64,16 +64,7 @@ __device__ __forceinline__ void load_block(const uint32_t* __restrict__ rec, int
 // two coordinates and reused by the thread's KP keys.  Accumulators are
 // (mse, qjl) pairs; with F2 they are updated by the packed fma.rn.f32x2.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\t"
-        "mov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
-        "mov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
+    return __ffma2_rn(a, b, c);  // fma.rn.f32x2: the register pairs stay packed
 }
 
 template <bool F2>
