@@ -54,6 +54,22 @@ __global__ void k_rownorm(const T* __restrict__ x, int64_t rows, int d,
 // only: a bf16 row scaled by 2^e is one exact fp16 piece).  x = 0 gives zero
 // pieces and scale 0 (the GEMM then writes y = 0).
 template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&v)[4]) {
+    if constexpr (sizeof(T) == 4) {
+        const float4 u = *reinterpret_cast<const float4*>(p);
+        v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+    } else {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        v[0] = __uint_as_float(u.x << 16);
+        v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+        v[2] = __uint_as_float(u.y << 16);
+        v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    }
+}
+
+// Rows whose start is 16-byte (fp32) or 8-byte (bf16) aligned are read 4
+// values a lane; d is a multiple of 128.
+template <typename T>
 __global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
                                   float* __restrict__ xnorm, float* __restrict__ rs,
                                   __half* __restrict__ out) {
@@ -61,10 +77,20 @@ __global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
     const int lane = threadIdx.x % 32;
     if (row >= rows) return;
     const T* xr = x + row * d;
+    const bool vec = ((uintptr_t)xr % (4 * sizeof(T))) == 0;  // the same for every row
     double acc = 0.0;
-    for (int i = lane; i < d; i += 32) {
-        const double v = (double)load_f32(xr, i);
-        acc = fma(v, v, acc);
+    if (vec) {
+        for (int i = 4 * lane; i < d; i += 128) {
+            float v[4];
+            load4(xr + i, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc = fma((double)v[e], (double)v[e], acc);
+        }
+    } else {
+        for (int i = lane; i < d; i += 32) {
+            const double v = (double)load_f32(xr, i);
+            acc = fma(v, v, acc);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -80,11 +106,31 @@ __global__ void k_rownorm_split16(const T* __restrict__ x, int64_t rows, int d,
     }
     __half* hi = out + row * d;
     __half* lo = out + rows * d + row * d;
-    for (int i = lane; i < d; i += 32) {
-        const float v = (float)((double)load_f32(xr, i) * sc);  // exact, |v| <= 2^11
-        const __half h = __float2half_rn(v);
-        hi[i] = h;
-        if (sizeof(T) == 4) lo[i] = __float2half_rn(v - __half2float(h));
+    if (vec) {
+        for (int i = 4 * lane; i < d; i += 128) {
+            float v[4];
+            load4(xr + i, v);
+            uint32_t hw[2], lw[2];
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const float a = (float)((double)v[2 * p] * sc);  // exact, |a| <= 2^11
+                const float b = (float)((double)v[2 * p + 1] * sc);
+                const __half2 h = __floats2half2_rn(a, b);
+                const float2 hf = __half22float2(h);
+                const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+                hw[p] = *reinterpret_cast<const uint32_t*>(&h);
+                lw[p] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            *reinterpret_cast<uint2*>(hi + i) = make_uint2(hw[0], hw[1]);
+            if (sizeof(T) == 4) *reinterpret_cast<uint2*>(lo + i) = make_uint2(lw[0], lw[1]);
+        }
+    } else {
+        for (int i = lane; i < d; i += 32) {
+            const float v = (float)((double)load_f32(xr, i) * sc);  // exact, |v| <= 2^11
+            const __half h = __float2half_rn(v);
+            hi[i] = h;
+            if (sizeof(T) == 4) lo[i] = __float2half_rn(v - __half2float(h));
+        }
     }
 }
 
