@@ -514,17 +514,10 @@ struct SmemP {
 };
 constexpr size_t kSmemPairBytes = sizeof(SmemP) + 1024;
 
-// Rotation epilogue: coordinates n0 .. n0 + 127 of row `row`, y = sum * sc:
-// the cell (the count of boundaries <= y, by binary search over the sorted
-// grid of 2^k levels), r = y - c[cell], the fp16 pieces of rscale * r and the
-// segment's |r|^2 -- the arithmetic of k_quantize16, per coordinate.
-__device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, const SmemP& sm,
-                                             const EncodeEpi& ep, int M, int N, int64_t row,
-                                             int n0) {
-    const int g = (ep.cb.split && n0 >= N / 2) ? 1 : 0;
-    const int L = sm.g_levels[g];
-    const float* bt = sm.g_b[g];
-    const float* ct = sm.g_c[g];
+template <int L>
+__device__ __forceinline__ void epi_quantize_l(const float (&sum)[kTN], float sc, const float* bt,
+                                               const float* ct, const EncodeEpi& ep, int M,
+                                               int N, int64_t row, int n0) {
     uint8_t* ix = ep.idx + row * N + n0;
     __half* hi = ep.rp + row * N + n0;
     __half* lo = ep.rp + (int64_t)M * N + row * N + n0;
@@ -540,7 +533,8 @@ __device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, 
                 const float y = sum[j0 + e + u] * sc;
                 int cell = 0;
                 float r = y;
-                if (L > 0) {
+                if constexpr (L > 0) {
+#pragma unroll
                     for (int step = L >> 1; step > 0; step >>= 1)
                         if (bt[cell + step - 1] <= y) cell += step;
                     r = y - ct[cell];
@@ -561,6 +555,24 @@ __device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, 
         *reinterpret_cast<uint4*>(lo + j0) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
     ep.rn2[(int64_t)(n0 / kTN) * M + row] = rr;
+}
+
+// Rotation epilogue: coordinates n0 .. n0 + 127 of row `row`, y = sum * sc:
+// the cell (the count of boundaries <= y, by binary search over the sorted
+// grid of 2^k levels), r = y - c[cell], the fp16 pieces of rscale * r and the
+// segment's |r|^2 -- the arithmetic of k_quantize16, per coordinate.
+__device__ __forceinline__ void epi_quantize(const float (&sum)[kTN], float sc, const SmemP& sm,
+                                             const EncodeEpi& ep, int M, int N, int64_t row,
+                                             int n0) {
+    const int g = (ep.cb.split && n0 >= N / 2) ? 1 : 0;
+    const float* bt = sm.g_b[g];
+    const float* ct = sm.g_c[g];
+    switch (sm.g_levels[g]) {  // inner-product grids: 2^(b-1) levels (none at b = 1)
+        case 0: epi_quantize_l<0>(sum, sc, bt, ct, ep, M, N, row, n0); break;
+        case 2: epi_quantize_l<2>(sum, sc, bt, ct, ep, M, N, row, n0); break;
+        case 4: epi_quantize_l<4>(sum, sc, bt, ct, ep, M, N, row, n0); break;
+        default: epi_quantize_l<8>(sum, sc, bt, ct, ep, M, N, row, n0); break;
+    }
 }
 
 // QJL epilogue: coordinates n0 .. n0 + 127 (4 blocks of 32) of row `row` --
