@@ -83,6 +83,18 @@ NCU_TRAFFIC = {
         "sha1": "d0fba32e71c4e1608d47cd281935347fa9eba732",
         "bytes": 68254208 + 4477696,
     },
+    # the encode call of the large-d workload: one 65,536-row chunk captured
+    # (k_rownorm_split16, k_gemm_pair<1>, k_gemm_pair<2>: 7,205,393,920 bytes)
+    # scaled by rows to 10^6, plus the once-per-call fp16 pieces of Pi and S
+    # (k_split2h x 2: 77,169,664 bytes)
+    ("larged", "encode"): {
+        "sources": ["kv_cache_embedding_b200/csrc/tq_encode.cu",
+                    "kv_cache_embedding_b200/csrc/tq_gemm_tc.cu",
+                    "kv_cache_embedding_b200/csrc/tq_sm100.cuh",
+                    "kv_cache_embedding_b200/csrc/tq_internal.cuh"],
+        "sha1": "411c04b786ffce29b3a17959fa12d3d1aef4023a",
+        "bytes": 110022755602,
+    },
 }
 
 
@@ -408,10 +420,17 @@ def encode_roofline(name, cfg, ab, enc_ms, pk, clocks):
     p_rot = 2 if cfg["x"] == "kv" else 3
     passes = [p_rot] if mse else [p_rot, 3]
     peak = bf16 * len(passes) / sum(passes)
+    if cfg["d"] % 256 == 0 and not mse:
+        kernel = ("tq_encode call: k_gemm_pair<1> (rotation, bucketize in the epilogue) + "
+                  "k_gemm_pair<2> (QJL, record packing in the epilogue) -- CTA-pair tcgen05 "
+                  "GEMMs on fp16 pieces -- + k_rownorm_split16")
+    else:
+        kernel = ("tq_encode call: k_gemm_tc (rotation and QJL as tcgen05 GEMMs on fp16 "
+                  "pieces) + k_rownorm_split16 + k_quantize16 + k_pack")
     return {"bound": "tensor", "achieved": round(ach, 2), "peak": round(peak, 1),
-            "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
-            "kernel": "k_gemm_tc (tq_encode: rotation and QJL as tcgen05 GEMMs on fp16 pieces) "
-                      "+ k_rownorm_split16 + k_quantize16 + k_pack",
+            "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+            "traffic": ncu_traffic(name, "encode") if cfg["n"] == CONFIGS[name]["n"] else None,
+            "kernel": kernel,
             "peak_source": (f"measured bf16 {which} (MEASURED_PEAKS.json)" if pk["src"] == "measured"
                             else f"fallback bf16 {which}") +
                            f" / {sum(passes) / len(passes):g} passes (mean over the products)",
