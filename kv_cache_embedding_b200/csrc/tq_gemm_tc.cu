@@ -507,7 +507,9 @@ struct SmemP {
     uint8_t pool[kPool][kPieceBytes];  // stage s: A's pa pieces, then B's pb (1024-aligned)
     float g_c[2][16], g_b[2][16];      // encode epilogues: the grids (second: fractional width)
     int g_levels[2];
+    float tkey[2][4][kTN];             // transposed store: per column half, warp, column maxima
     uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done;
+    uint64_t tmax_bar[2], tmax_bar2[2];
     uint32_t tmem_base;
     int abort;
     int zero;
@@ -616,8 +618,9 @@ template <int EPI>
 __global__ void __launch_bounds__(kPairThreads, 1)
 k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
             int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
-            const float* __restrict__ row_scale, int scale_mode, int* __restrict__ err,
-            uint32_t idesc, const __grid_constant__ EncodeEpi ep) {
+            const float* __restrict__ row_scale, int scale_mode, int n_store,
+            float* __restrict__ tmax, int64_t ldt, int* __restrict__ err, uint32_t idesc,
+            const __grid_constant__ EncodeEpi ep) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     // the same offset in both CTAs: the MMA reads the peer's operands there
@@ -644,11 +647,15 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             mbar_init(&sm.acc_empty[i], 2 * kPairEpiWarps);  // used in the leader
         }
         mbar_init(&sm.mma_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.tmax_bar[i], 4);   // the 4 warps of a column half
+            mbar_init(&sm.tmax_bar2[i], 4);
+        }
         sm.abort = 0;
         sm.zero = 0;
         fence_mbar_init();
     }
-    if (EPI != 0 && threadIdx.x >= 32 && threadIdx.x < 64) {
+    if ((EPI == 1 || EPI == 2) && threadIdx.x >= 32 && threadIdx.x < 64) {
         const int i = threadIdx.x - 32;
         if (i < 16) {
             sm.g_c[0][i] = ep.cb.c[i];
@@ -761,7 +768,7 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
         const uint32_t lane_addr = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)(hc * kTN);
         const uint32_t empty_c[2] = {mapa_shared(smem_u32(&sm.acc_empty[0]), 0),
                                      mapa_shared(smem_u32(&sm.acc_empty[1]), 0)};
-        uint32_t cc = 0;
+        uint32_t cc = 0, tb = 0;
         bool ok = true;
         for (int t = pair; t < tiles && ok; t += npairs) {
             const int m0 = (t / tn) * 2 * kTM + (int)rank * kTM;
@@ -790,7 +797,50 @@ k_gemm_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             }
             if (!ok) break;
             const int64_t row = (int64_t)m0 + 32 * q + lane;
-            if (row < M) {
+            if constexpr (EPI == 3) {
+                // scores: column j of the tile -> C[(n0 + j) * ldc + row] (a warp writes 32
+                // consecutive rows of each column), times row_scale; the maximum of the
+                // CTA's 128 rows per column for the top-k threshold
+                const bool live = row < M;
+                const float sc = live ? row_scale[row] : 0.f;
+#pragma unroll
+                for (int j = 0; j < kTN; ++j) {
+                    const float v = sum[j] * sc;
+                    if (live && n0 + j < n_store) C[(int64_t)(n0 + j) * ldc + row] = v;
+                    if (tmax) {
+                        float m = live ? v : -INFINITY;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (lane == 0) sm.tkey[hc][q][j] = m;
+                    }
+                }
+                if (tmax) {
+                    // the 4 warps of this column half meet on a bounded barrier, then
+                    // each writes the maxima of 32 columns
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.tmax_bar[hc]);
+                    if (!warp_wait(&sm.tmax_bar[hc], tb & 1, abort)) {
+                        ok = give_up(abort, err, 55);
+                        break;
+                    }
+                    ++tb;
+                    const int j = 32 * q + lane;
+                    // a CTA whose 128 rows all lie past M (the second half of the
+                    // last pair tile) has no tile maximum to write
+                    if (n0 + j < n_store && m0 < M)
+                        tmax[(int64_t)(n0 + j) * ldt + m0 / kTM] =
+                            fmaxf(fmaxf(sm.tkey[hc][0][j], sm.tkey[hc][1][j]),
+                                  fmaxf(sm.tkey[hc][2][j], sm.tkey[hc][3][j]));
+                    // the slots are rewritten only after every warp has read them
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.tmax_bar2[hc]);
+                    if (!warp_wait(&sm.tmax_bar2[hc], (tb - 1) & 1, abort)) {
+                        ok = give_up(abort, err, 56);
+                        break;
+                    }
+                }
+            } else if (row < M) {
                 float sc = 1.f;
                 if (scale_mode == 1) {
                     const float r = row_scale[row];
@@ -935,10 +985,11 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     const int epi_mode = epi ? epi->mode : 0;
     if (epi_mode != 0 && (transposed || tmax || N % kPN != 0 || nsm < 2 || !pair_form))
         return TQ_ERR_ARG;
-    if (!transposed && !tmax && N % kPN == 0 && nsm >= 2 && pair_form) {
+    if ((transposed || !tmax) && N % kPN == 0 && nsm >= 2 && pair_form) {
         const int64_t ptiles = (int64_t)((M + 2 * kTM - 1) / (2 * kTM)) * (N / kPN);
         const int npairs = (int)(ptiles < nsm / 2 ? ptiles : nsm / 2);
-        auto kern = epi_mode == 1 ? k_gemm_pair<1> : epi_mode == 2 ? k_gemm_pair<2> : k_gemm_pair<0>;
+        auto kern = transposed ? k_gemm_pair<3>
+                    : epi_mode == 1 ? k_gemm_pair<1> : epi_mode == 2 ? k_gemm_pair<2> : k_gemm_pair<0>;
         TQ_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemPairBytes));
         cudaLaunchConfig_t cfg = {};
@@ -956,8 +1007,8 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
         EncodeEpi e = {};
         if (epi) e = *epi;
         TQ_TRY_CUDA(cudaLaunchKernelEx(&cfg, kern, ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
-                                       scale_mode, d_err, idesc_f16(fp16 ? 0u : 1u, 2 * kTM, kPN),
-                                       e));
+                                       scale_mode, n_store, tmax, ldt, d_err,
+                                       idesc_f16(fp16 ? 0u : 1u, 2 * kTM, kPN), e));
         return TQ_OK;
     }
     const int64_t tiles = (int64_t)((M + kTM - 1) / kTM) * (N / kTN);

@@ -10,13 +10,14 @@
 // (vector search over the quantized database).
 //
 // A and B are two bf16 pieces each (x = hi + lo to ~2^-16 of |x|) and the GEMM
-// sums hi hi + hi lo + lo hi, an error well inside the score tolerance.  Up
-// to 256 queries the keys' pieces are decoded from the records inside the
+// sums hi hi + hi lo + lo hi, an error well inside the score tolerance.  With
+// one 128-query tile the keys' pieces are decoded from the records inside the
 // GEMM (two warps write them into each shared-memory stage), so only the
-// records cross HBM; with more queries they are decoded once per chunk of
-// 32768 keys into the workspace.  The queries' pieces come by TMA.  Scores go out transposed
-// ([query][key], coalesced over keys) with the maximum of every 128-key tile
-// per query for the top-k threshold.
+// records cross HBM; with 256 or more queries they are decoded once per chunk
+// of 37,888 keys into the workspace and the product runs on CTA pairs
+// (256 x 256 tiles).  The queries' pieces come by TMA.  Scores go out
+// transposed ([query][key], coalesced over keys) with the maximum of every
+// 128-key tile per query for the top-k threshold.
 #include <cuda_bf16.h>
 
 #include "tq_internal.cuh"
@@ -128,16 +129,23 @@ bool topk_materialized(int d, int G, int64_t n, int nq) {
     return (int64_t)G * nq * n <= kTopkMaterialize || score_gemm_supported(d, nq);
 }
 
-// Up to 256 queries the keys are decoded inside the GEMM (two query tiles per
-// key tile); beyond that re-decoding every key tile for each query tile costs
-// more than writing the decoded keys once per chunk and reading them back.
+// Query counts padded to a multiple of 256 take the decoded keys through HBM,
+// once per chunk of keys, and the CTA-pair GEMM (256 x 256 tiles: each key
+// tile is read once per 256 queries); a single 128-query tile decodes the keys
+// inside the one-CTA GEMM, so only the records cross HBM.  Beyond 256 queries
+// re-decoding every key tile for each query tile costs more than the round
+// trip of the decoded keys.
 constexpr int kDecodeInGemmMaxQueries = 256;
-constexpr int64_t kScoreGemmChunk = 32768;  // keys decoded per GEMM (materialised form)
+constexpr int64_t kScoreGemmChunk = 148 * 256;  // keys decoded per GEMM: 2 row tiles per pair
+
+bool score_gemm_materialises(int64_t nq_pad) {
+    return nq_pad > kDecodeInGemmMaxQueries || nq_pad % 256 == 0;
+}
 
 size_t score_gemm_workspace(int d, int64_t n, int nq) {
     const int64_t nq_pad = (nq + 127) / 128 * 128;
     size_t bytes = align256((size_t)2 * nq_pad * 2 * d * 2);
-    if (nq_pad > kDecodeInGemmMaxQueries) {
+    if (score_gemm_materialises(nq_pad)) {
         const int64_t chunk = n < kScoreGemmChunk ? n : kScoreGemmChunk;
         bytes += align256((size_t)2 * chunk * 2 * d * 2);
     }
@@ -168,7 +176,7 @@ int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_code
         k_query_operand<<<(unsigned)((qn + 255) / 256), 256, 0, s>>>(
             qr + (int64_t)g * nq * d, u + (int64_t)g * nq * d, nq, nq_pad, d, Bq);
         TQ_CHECK_LAUNCH();
-        if (nq_pad > kDecodeInGemmMaxQueries) {  // decoded keys through HBM, chunk by chunk
+        if (score_gemm_materialises(nq_pad)) {  // decoded keys through HBM, chunk by chunk
             __nv_bfloat16* Ak =
                 (__nv_bfloat16*)((char*)op_ws + align256((size_t)2 * nq_pad * 2 * d * 2));
             const KCodebook kc = make_kcodebook(cb);

@@ -633,6 +633,30 @@ def test_topk_merge_of_shards(quant, oparams, tq_lib, cuda, nshards, k):
 
 
 # ---------------------------------------------------------------- scores and top-k in one call
+@pytest.mark.parametrize("n", [37888 + 64, 2 * 37888 + 200])
+def test_decoded_key_topk_ragged_chunks(quant, oparams, tq_lib, cuda, n):
+    """256 queries at d = 512: the decoded keys go through chunks of 37,888 keys
+    and the CTA-pair GEMM; the last chunk ends inside a 256-key pair tile (one
+    CTA of the pair has no live rows).  Every query's top-10 values equal the
+    top-10 of its scores; 4 queries against the oracle."""
+    d, b, nq, k = 512, 4, 256, 10
+    c, xn, rn = synth.random_records(n, b * d // 32, seed=91)
+    q = synth.gaussian_rows(nq, d, seed=92, norm_range=None)
+    tq = quant(d, b)
+    codes = _to_codes(tq_lib, c, xn, rn, cuda)
+    s = tq.score(codes, q.cuda()[None])
+    vals, ids = tq.topk(codes, q.cuda()[None], k)
+    torch.cuda.synchronize()
+    tv, _ = torch.topk(s[0], k, dim=1)
+    assert torch.equal(vals[0], tv)
+    pick = [0, 1, 127, 255]
+    qs = _f64(q[pick])
+    s_ora = O.score(oparams(d, b, 0), c, xn, rn, qs)
+    qn = np.linalg.norm(qs, axis=1)
+    PT.compare_scores(_np(s[0, pick]), s_ora, qn, xn.astype(np.float64))
+    PT.compare_topk(_np(vals[0, pick]), _np(ids[0, pick]), s_ora, k, qn, float(xn.max()))
+
+
 @pytest.mark.parametrize("d,b,G,n,nq", [(128, 4, 2, 5000, 4), (128, 4, 1, 3001, 16),
                                         (256, 4, 1, 2000, 70), (128, 2, 1, 2_200_000, 8),
                                         (128, 3, 3, 777, 1)])
