@@ -54,53 +54,52 @@ __device__ __forceinline__ void field_of(const uint32_t* w, int j, int& cell, in
 }
 
 // A pieces [2][rows][2d] of the records of one key chunk; one thread per
-// (key, 32-coordinate block).
+// (key, 8 coordinates), so a warp's 16-byte stores to each of the four
+// planes are contiguous (whole sectors: no read-for-ownership of partly
+// written sectors).
 template <int B>
 __global__ void k_key_operand(const uint32_t* __restrict__ codes, const float* __restrict__ rnorm,
                               int64_t rows, int d, KCodebook cb, __nv_bfloat16* __restrict__ out) {
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int nb = d / 32;
-    if (e >= rows * nb) return;
-    const int64_t v = e / nb;
-    const int blk = (int)(e % nb);
-    const uint32_t* w = codes + v * (int64_t)(nb * B) + blk * B;
+    const int nc = d / 8;  // 8-coordinate chunks per key
+    if (e >= rows * nc) return;
+    const int64_t v = e / nc;
+    const int ch = (int)(e % nc);
+    const int blk = ch >> 2, j0 = 8 * (ch & 3);
+    const uint32_t* w = codes + v * (int64_t)(d / 32 * B) + blk * B;
     uint32_t ww[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int i = 0; i < B; ++i) ww[i] = __ldg(w + i);
     const float kap = kSqrtHalfPi / (float)d * __ldg(rnorm + v);
     const int64_t K = 2 * (int64_t)d, plane = rows * K;
-    __nv_bfloat16* row = out + v * K + blk * 32;
+    __nv_bfloat16* row = out + v * K + 8 * ch;
+    uint32_t chi[4] = {0u, 0u, 0u, 0u}, clo[4] = {0u, 0u, 0u, 0u};
+    uint32_t shi[4] = {0u, 0u, 0u, 0u}, slo[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int j0 = 0; j0 < 32; j0 += 8) {  // 8 coordinates -> one 16-byte store per output
-        uint32_t chi[4] = {0u, 0u, 0u, 0u}, clo[4] = {0u, 0u, 0u, 0u};
-        uint32_t shi[4] = {0u, 0u, 0u, 0u}, slo[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            int cell, z;
-            field_of<B>(ww, j0 + h, cell, z);
-            float c, sgn;
-            if (cb.mse) {
-                c = cb.c[(B == 1) ? z : (cell | (z << (B - 1)))];
-                sgn = 0.f;
-            } else {
-                c = (B == 1) ? 0.f : cb.c[cell];
-                sgn = z ? kap : -kap;
-            }
-            __nv_bfloat16 ch, cl, sh, sl;
-            split2(c, ch, cl);
-            split2(sgn, sh, sl);
-            const int sft = 16 * (h & 1);
-            const uint32_t m = (h & 1) ? 0xFFFFu : 0u;
-            chi[h >> 1] = (chi[h >> 1] & m) | ((uint32_t)__bfloat16_as_ushort(ch) << sft);
-            clo[h >> 1] = (clo[h >> 1] & m) | ((uint32_t)__bfloat16_as_ushort(cl) << sft);
-            shi[h >> 1] = (shi[h >> 1] & m) | ((uint32_t)__bfloat16_as_ushort(sh) << sft);
-            slo[h >> 1] = (slo[h >> 1] & m) | ((uint32_t)__bfloat16_as_ushort(sl) << sft);
+    for (int h = 0; h < 8; ++h) {
+        int cell, z;
+        field_of<B>(ww, j0 + h, cell, z);
+        float c, sgn;
+        if (cb.mse) {
+            c = cb.c[(B == 1) ? z : (cell | (z << (B - 1)))];
+            sgn = 0.f;
+        } else {
+            c = (B == 1) ? 0.f : cb.c[cell];
+            sgn = z ? kap : -kap;
         }
-        *reinterpret_cast<uint4*>(row + j0) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
-        *reinterpret_cast<uint4*>(row + plane + j0) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
-        *reinterpret_cast<uint4*>(row + d + j0) = make_uint4(shi[0], shi[1], shi[2], shi[3]);
-        *reinterpret_cast<uint4*>(row + plane + d + j0) = make_uint4(slo[0], slo[1], slo[2], slo[3]);
+        __nv_bfloat16 c1, c2, s1, s2;
+        split2(c, c1, c2);
+        split2(sgn, s1, s2);
+        const int sft = 16 * (h & 1);
+        chi[h >> 1] |= (uint32_t)__bfloat16_as_ushort(c1) << sft;
+        clo[h >> 1] |= (uint32_t)__bfloat16_as_ushort(c2) << sft;
+        shi[h >> 1] |= (uint32_t)__bfloat16_as_ushort(s1) << sft;
+        slo[h >> 1] |= (uint32_t)__bfloat16_as_ushort(s2) << sft;
     }
+    *reinterpret_cast<uint4*>(row) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
+    *reinterpret_cast<uint4*>(row + plane) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
+    *reinterpret_cast<uint4*>(row + d) = make_uint4(shi[0], shi[1], shi[2], shi[3]);
+    *reinterpret_cast<uint4*>(row + plane + d) = make_uint4(slo[0], slo[1], slo[2], slo[3]);
 }
 
 // B pieces [2][nq_pad][2d] of one group's queries (rows >= nq are zero).
@@ -184,7 +183,7 @@ int score_gemm(const tq_codebook_t* cb, int G, int64_t n, const uint32_t* d_code
             for (int64_t r0 = 0; r0 < n; r0 += chunk) {
                 const int64_t rows = (n - r0) < chunk ? (n - r0) : chunk;
                 const int64_t off = (int64_t)g * n + r0;
-                const unsigned blocks = (unsigned)((rows * (d / 32) + 255) / 256);
+                const unsigned blocks = (unsigned)((rows * (d / 8) + 255) / 256);
                 switch (b) {
                     case 1: k_key_operand<1><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
                     case 2: k_key_operand<2><<<blocks, 256, 0, s>>>(d_codes + off * W, d_rnorm + off, rows, d, kc, Ak); break;
