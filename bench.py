@@ -84,16 +84,16 @@ NCU_TRAFFIC = {
         "bytes": 68254208 + 4477696,
     },
     # the encode call of the large-d workload: one 65,536-row chunk captured
-    # (k_rownorm_split16, k_gemm_pair<1>, k_gemm_pair<2>: 7,205,393,920 bytes)
+    # (k_rownorm_split16, k_gemm_pair<1>, k_gemm_pair<2>: 7,056,975,360 bytes)
     # scaled by rows to 10^6, plus the once-per-call fp16 pieces of Pi and S
-    # (k_split2h x 2: 77,169,664 bytes)
+    # (k_split2h x 2: 77,008,896 bytes)
     ("larged", "encode"): {
         "sources": ["kv_cache_embedding_b200/csrc/tq_encode.cu",
                     "kv_cache_embedding_b200/csrc/tq_gemm_tc.cu",
                     "kv_cache_embedding_b200/csrc/tq_sm100.cuh",
                     "kv_cache_embedding_b200/csrc/tq_internal.cuh"],
-        "sha1": "411c04b786ffce29b3a17959fa12d3d1aef4023a",
-        "bytes": 110022755602,
+        "sha1": "4ec944ae8d124d02d35f999f3166ecc941ba1499",
+        "bytes": 107757907334,
     },
 }
 
