@@ -396,6 +396,22 @@ extern "C" int tq_encode(const tq_codebook_t* cb, const float* d_Pi, const float
                     if (rc) return rc;
                     continue;
                 }
+                if (mse && d == 128) {
+                    // the rotation with the bucketize and packing of whole rows in
+                    // its epilogue (the MSE-only records have no QJL product)
+                    EncodeEpi e4 = {};
+                    e4.mode = 4;
+                    e4.b = b;
+                    e4.codes = d_codes + (size_t)off * W;
+                    e4.rnorm = rn;
+                    e4.cb = kc;
+                    rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP,
+                                        x_dtype == TQ_F32 ? 2 : 1, (const __nv_bfloat16*)PiP,
+                                        nullptr, d, RS, 1, err, s, 2, false, 0, nullptr, 0, true,
+                                        false, &e4);
+                    if (rc) return rc;
+                    continue;
+                }
                 rc = launch_gemm_tc((int)rows, d, d, (const __nv_bfloat16*)AP,
                                     x_dtype == TQ_F32 ? 2 : 1, (const __nv_bfloat16*)PiP, Y, d, RS,
                                     1, err, s, 2, false, 0, nullptr, 0, true);

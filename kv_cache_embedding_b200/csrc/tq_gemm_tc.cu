@@ -64,6 +64,7 @@ struct SmemG {
     uint32_t dtab[16];                   // decoded-A mode: packed bf16 pieces of c[cell]
     uint2 dpair[256][8];                 // b = 4: code byte -> (hi pair, lo pair) words, 8 copies
     uint32_t dsign[256];                 // b = 4: code byte -> sign flips of the pair (z = 0)
+    float g_c[16], g_b[16];              // MSE-only encode epilogue: the grid
     uint64_t full[kMaxStages], empty[kMaxStages], acc_full[2], acc_empty[2], mma_done, tmax_bar, tmax_bar2;
     uint32_t tmem_base;
     int abort;
@@ -238,12 +239,66 @@ __device__ bool decode_loop(const KeyDecode& kd, SmemG& sm, int64_t M, int tiles
     }
 }
 
+// MSE-only encode epilogue (mode 4) of a whole row (N = K = d = 128: the
+// tile holds every coordinate of its rows): y = sum * sc, the cell (the count
+// of boundaries <= y, binary search over the 2^b-level grid), |r| = |y -
+// c[cell]|, and the record of the MSE-only layout (the cell's low b - 1 bits
+// in the index fields, its top bit in the sign positions) -- the arithmetic
+// of k_quantize and k_pack, without the rotated rows crossing HBM.
+template <int L, int B>
+__device__ __forceinline__ void epi_mse_row(const float (&sum)[kTN], float sc, const float* bt,
+                                            const float* ct, const EncodeEpi& ep, int64_t row) {
+    constexpr int W = B * kTN / 32;
+    uint32_t out[W];
+#pragma unroll
+    for (int i = 0; i < W; ++i) out[i] = 0u;
+    float rr = 0.f;
+#pragma unroll
+    for (int j = 0; j < kTN; ++j) {
+        const float y = sum[j] * sc;
+        int cell = 0;
+#pragma unroll
+        for (int step = L >> 1; step > 0; step >>= 1)
+            if (bt[cell + step - 1] <= y) cell += step;
+        const float r = y - ct[cell];
+        rr = fmaf(r, r, rr);
+        const uint32_t iv = (uint32_t)cell & ((1u << (B - 1)) - 1u), z = (uint32_t)cell >> (B - 1);
+        const int w = j >> 5, jj = j & 31;
+        if (B == 1) {
+            out[w] |= z << jj;
+        } else if (B == 2) {
+            out[2 * w + (jj >> 4)] |= (iv | (z << 1)) << (2 * (jj & 15));
+        } else if (B == 3) {
+            out[3 * w + (jj >> 4)] |= iv << (2 * (jj & 15));
+            out[3 * w + 2] |= z << jj;
+        } else {
+            out[4 * w + (jj >> 3)] |= (iv | (z << 3)) << (4 * (jj & 7));
+        }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(ep.codes + row * W);
+#pragma unroll
+    for (int i = 0; i < W / 4; ++i)
+        dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+    ep.rnorm[row] = sqrtf(rr);
+}
+
+template <int B>
+__device__ __forceinline__ void epi_mse_row_b(const float (&sum)[kTN], float sc, const float* bt,
+                                              const float* ct, const EncodeEpi& ep, int64_t row) {
+    switch (ep.cb.levels) {  // 2^b levels
+        case 2: epi_mse_row<2, B>(sum, sc, bt, ct, ep, row); break;
+        case 4: epi_mse_row<4, B>(sum, sc, bt, ct, ep, row); break;
+        case 8: epi_mse_row<8, B>(sum, sc, bt, ct, ep, row); break;
+        default: epi_mse_row<16, B>(sum, sc, bt, ct, ep, row); break;
+    }
+}
+
 __global__ void __launch_bounds__(kThreadsDecode, 1)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
           int M, int N, int K, int pa, int pb, float* __restrict__ C, int64_t ldc,
           const float* __restrict__ row_scale, int scale_mode, int transposed, int n_store,
           float* __restrict__ tmax, int64_t ldt, int* __restrict__ err, KeyDecode kd,
-          int decode, uint32_t idesc) {
+          int decode, uint32_t idesc, const __grid_constant__ EncodeEpi ep) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = smem_u32(smem_raw);
     SmemG& sm = *reinterpret_cast<SmemG*>(smem_raw + (((sbase + 1023u) & ~1023u) - sbase));
@@ -271,6 +326,10 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
         sm.abort = 0;
         sm.zero = 0;
         fence_mbar_init();
+    }
+    if (ep.mode == 4 && threadIdx.x >= 32 && threadIdx.x < 48) {
+        sm.g_c[threadIdx.x - 32] = ep.cb.c[threadIdx.x - 32];
+        sm.g_b[threadIdx.x - 32] = ep.cb.beta[threadIdx.x - 32];
     }
     if (decode && threadIdx.x < 16) {
         uint32_t v = 0u;
@@ -427,7 +486,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CU
             } else if (live && scale_mode == 2) {
                 sc = row_scale[row];
             }
-            if (!transposed) {
+            if (ep.mode == 4) {
+                if (live) {
+                    switch (ep.b) {
+                        case 1: epi_mse_row_b<1>(sum, sc, sm.g_b, sm.g_c, ep, row); break;
+                        case 2: epi_mse_row_b<2>(sum, sc, sm.g_b, sm.g_c, ep, row); break;
+                        case 3: epi_mse_row_b<3>(sum, sc, sm.g_b, sm.g_c, ep, row); break;
+                        default: epi_mse_row_b<4>(sum, sc, sm.g_b, sm.g_c, ep, row); break;
+                    }
+                }
+            } else if (!transposed) {
                 if (live) {
                     float4* dst = reinterpret_cast<float4*>(C + row * ldc + n0);
 #pragma unroll
@@ -983,9 +1051,11 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     TQ_TRY_CUDA(cudaGetDevice(&dev));
     TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
     const int epi_mode = epi ? epi->mode : 0;
-    if (epi_mode != 0 && (transposed || tmax || N % kPN != 0 || nsm < 2 || !pair_form))
+    if ((epi_mode == 1 || epi_mode == 2) &&
+        (transposed || tmax || N % kPN != 0 || nsm < 2 || !pair_form))
         return TQ_ERR_ARG;
-    if ((transposed || !tmax) && N % kPN == 0 && nsm >= 2 && pair_form) {
+    if (epi_mode == 4 && (transposed || tmax || N != kTN || K != kTN)) return TQ_ERR_ARG;
+    if (epi_mode != 4 && (transposed || !tmax) && N % kPN == 0 && nsm >= 2 && pair_form) {
         const int64_t ptiles = (int64_t)((M + 2 * kTM - 1) / (2 * kTM)) * (N / kPN);
         const int npairs = (int)(ptiles < nsm / 2 ? ptiles : nsm / 2);
         auto kern = transposed ? k_gemm_pair<3>
@@ -1015,10 +1085,12 @@ int launch_gemm_tc(int M, int N, int K, const __nv_bfloat16* A, int pa, const __
     const int nctas = (int)(tiles < nsm ? tiles : nsm);
     TQ_TRY_CUDA(cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)kSmemBytes));
+    EncodeEpi e1 = {};
+    if (epi) e1 = *epi;
     k_gemm_tc<<<nctas, kThreads, kSmemBytes, s>>>(ma, mb, M, N, K, pa, pb, C, ldc, row_scale,
                                                   scale_mode, transposed ? 1 : 0, n_store, tmax,
                                                   ldt, d_err, KeyDecode{}, 0,
-                                                  idesc_f16(fp16 ? 0u : 1u, kTM, kTN));
+                                                  idesc_f16(fp16 ? 0u : 1u, kTM, kTN), e1);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
@@ -1041,7 +1113,7 @@ int launch_gemm_tc_decoded(int M, int N, const KeyDecode& kd, const __nv_bfloat1
     // the A map is unused in this mode: the B map stands in for the parameter
     k_gemm_tc<<<nctas, kThreadsDecode, kSmemBytes, s>>>(mb, mb, M, N, K, 2, 2, C, ldc, row_scale,
                                                         2, 1, n_store, tmax, ldt, d_err, kd, 1,
-                                                        idesc_f16(1u, kTM, kTN));
+                                                        idesc_f16(1u, kTM, kTN), EncodeEpi{});
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }

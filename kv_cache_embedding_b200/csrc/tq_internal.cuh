@@ -106,7 +106,9 @@ bool encode_tc_supported(const tq_codebook_t* cb, int x_dtype, int G, int64_t n)
 // d % 256 == 0, inner-product records).  Mode 1, on the rotation product:
 // bucketize y = C, write the cells, the fp16 pieces of rscale * r and |r|^2 of
 // every 128 coordinates.  Mode 2, on the QJL product: the signs of C with the
-// cells -> code records, and |r| from the partial sums.  Mode 0 stores C.
+// cells -> code records, and |r| from the partial sums.  Mode 4 (one-CTA GEMM,
+// d = 128, the MSE-only variant): bucketize, |r| and the MSE-only records of
+// whole rows.  Mode 0 stores C.
 struct EncodeEpi {
     int mode;
     int b;
