@@ -84,16 +84,16 @@ NCU_TRAFFIC = {
         "bytes": 68254208 + 4477696,
     },
     # the encode call of the large-d workload: one 65,536-row chunk captured
-    # (k_rownorm_split16, k_gemm_pair<1>, k_gemm_pair<2>: 7,056,975,360 bytes)
+    # (k_rownorm_split16, k_gemm_pair<1>, k_gemm_pair<2>: 7,318,083,584 bytes)
     # scaled by rows to 10^6, plus the once-per-call fp16 pieces of Pi and S
-    # (k_split2h x 2: 77,008,896 bytes)
+    # (k_split2h x 2: 77,417,984 bytes)
     ("larged", "encode"): {
         "sources": ["kv_cache_embedding_b200/csrc/tq_encode.cu",
                     "kv_cache_embedding_b200/csrc/tq_gemm_tc.cu",
                     "kv_cache_embedding_b200/csrc/tq_sm100.cuh",
                     "kv_cache_embedding_b200/csrc/tq_internal.cuh"],
-        "sha1": "4ec944ae8d124d02d35f999f3166ecc941ba1499",
-        "bytes": 107757907334,
+        "sha1": "7eaf6b4b254e4974a13efe3b92089d613ff45741",
+        "bytes": 111742511734,
     },
 }
 
