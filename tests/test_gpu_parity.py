@@ -513,6 +513,25 @@ def test_mse_encode_bf16_and_large_d(quant_mse, d, b, G):
         _mse_compare(d, b, gpu, ora, P.beta)
 
 
+@pytest.mark.parametrize("b,G,n,kind", [(4, 3, 1024, "kv"), (2, 8, 384, "kv"), (3, 2, 768, "rows"),
+                                        (1, 4, 128, "rows")])
+def test_mse_encode_groups(quant_mse, b, G, n, kind):
+    """d = 128 (the rotation with the bucketize and packing of whole rows in
+    its epilogue), several groups with whole 128-row tiles, bf16 keys and fp32
+    rows; every group against the oracle."""
+    d = 128
+    if kind == "kv":
+        x = synth.kv_keys(G, n, d, seed=4)
+    else:
+        x = synth.gaussian_rows(G * n, d, seed=4).reshape(G, n, d)
+    codes = quant_mse(d, b, 0, G).encode(x.cuda())
+    for g in range(G):
+        P = O.MseParams(d, b, g)
+        ora = O.mse_encode(P, x[g].to(torch.float64).numpy(), diagnostics=True)
+        gpu = (_np(codes.codes[g]).view(np.uint32), _np(codes.xnorm[g]), _np(codes.rnorm[g]))
+        _mse_compare(d, b, gpu, ora, P.beta)
+
+
 @pytest.mark.parametrize("b,nq", [(4, 64), (2, 3), (1, 5)])
 def test_mse_score_and_topk(quant_mse, tq_lib, cuda, b, nq):
     d, n, k = 128, 3000, 10
