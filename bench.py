@@ -451,6 +451,45 @@ def time_steps(run, flush, steps):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def graph_call_time(run, flush, reps=20, trials=5):
+    """Device time (ms) of one call of run() inside a CUDA graph, L2 flushed
+    before each call: a graph of `reps` x [flush, call] is timed with one
+    event pair, a graph of `reps` x [flush] likewise, and the difference is
+    divided by `reps` (median of `trials` replays each).  This leaves out the
+    per-launch submission gaps of an eager stream and the event timer's
+    granularity, which a single event pair around a ~50 us call does not."""
+    def capture(fn):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    fn()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        return g
+
+    def timed(g):
+        ts = []
+        for _ in range(trials):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    gf = capture(lambda: flush.zero_())
+    gc = capture(lambda: (flush.zero_(), run()))
+    ms = (timed(gc) - timed(gf)) / reps
+    del gc, gf
+    return ms
+
+
 def e2e_time(tq, cfg, x, q, steps, dist, dev, shard):
     """End-to-end step through the public API with host buffers: every step
     copies its inputs from pinned host memory, runs the same calls and copies
@@ -671,12 +710,15 @@ def score_alone_time(tq, cfg, step, flush, args, nq):
         tq.score(step.codes, q, out=out)
     ts = time_steps(lambda: tq.score(step.codes, q, out=out), flush, max(10, min(args.steps, 50)))
     ms = statistics.median(ts)
+    gms = graph_call_time(lambda: tq.score(step.codes, q, out=out), flush)
     rec = cfg["b"] * cfg["d"] // 8 + 8
     byts = cfg["G"] * step.codes.n * rec + out.numel() * 4
     pk = peaks()
     return {"ms": round(ms, 5), "queries_per_group": nq, "gbs": round(byts / ms / 1e6, 1),
             "hbm_frac": round(byts / ms / 1e6 / pk["hbm"], 4),
-            "scores_s": round(out.numel() / ms * 1e3, 1), "call": "tq_score"}
+            "scores_s": round(out.numel() / ms * 1e3, 1), "call": "tq_score",
+            "graph_ms": round(gms, 5), "graph_gbs": round(byts / gms / 1e6, 1),
+            "timing": "ms: event pair around each eager call; graph_ms: per call inside a CUDA graph"}
 
 
 def search_recall(tq, step, x, q, cfg, shard):
@@ -717,9 +759,10 @@ def attention_decode_time(cfg, x, q, flush, args):
     ts = time_steps(lambda: tk.attention_decode(kc, tv, vc, q, out=out), flush,
                     max(3, min(args.steps, 50)))
     ms = sum(ts) / len(ts)
+    gms = graph_call_time(lambda: tk.attention_decode(kc, tv, vc, q, out=out), flush)
     byts = (kc.codes.numel() * 4 + kc.xnorm.numel() * 8 + vc.codes.numel() * 4 +
             vc.xnorm.numel() * 4 + q.numel() * q.element_size() + out.numel() * 4)
-    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1),
+    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1), "graph_ms": round(gms, 5),
             "values": "4-bit MSE-only records (seeded keys-like rows)", "scale": "1/sqrt(d)"}
 
 
@@ -732,8 +775,9 @@ def fp32_baseline(cfg, x, q, flush, args):
         K.logits_fp32(keys, q, out)
     ts = time_steps(lambda: K.logits_fp32(keys, q, out), flush, max(3, min(args.steps, 50)))
     ms = sum(ts) / len(ts)
+    gms = graph_call_time(lambda: K.logits_fp32(keys, q, out), flush)
     byts = keys.numel() * 4 + out.numel() * 4
-    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1)}
+    return {"ms": round(ms, 5), "gbs": round(byts / ms / 1e6, 1), "graph_ms": round(gms, 5)}
 
 
 # ---------------------------------------------------------------- oracle arm
