@@ -43,28 +43,48 @@ __device__ __forceinline__ uint32_t value_cell(const uint32_t* blk, int j) {
     return (blk[0] >> j) & 1u;
 }
 
+// Asynchronous 16-byte global -> shared copies (completion per thread,
+// cp.async.wait_all; a barrier then makes every thread's copies visible).
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(smem))),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // One split of `split` keys of group g for queries q0 .. q0 + NQ - 1:
 //   M_q = max_j l_qj over the split (one pass over its logits, so the
 //         weights need no rescaling as the tiles go by),
 //   w_qj = e^(l_qj - M_q) |v_j|,  L_q = sum_j e^(l_qj - M_q),
 //   acc_q = sum_j w_qj c_v[cell_j]   (the rotated value domain).
-// Per tile of 256 keys, thread t forms key t's weights (shared memory); then
-// thread (8-coordinate word wi = t % 16, key lane kl = t / 16) walks keys
-// kl, kl + 16, ... of the tile: one code word of the record (coalesced: 16
-// threads read one record), 8 centroids from a 16-entry table (one entry per
-// bank: no conflicts), 16 packed fp32x2 FMAs for the 4 queries.  The 16 key
-// lanes' sums are merged once per split.
+// Tiles of 256 keys, software-pipelined: the value records of tile i + 1 are
+// copied into shared memory (cp.async) and its logits loaded into registers
+// while tile i is summed, so the sums never wait on HBM.  Per tile, thread t
+// forms key t's weights (shared memory); then thread (8-coordinate word
+// wi = t % 16, key lane kl = t / 16) walks keys kl, kl + 16, ... of the tile:
+// one code word of the record (16 threads read one record: no bank
+// conflicts), 8 centroids from a byte-pair table (b_v = 4) or the 16-entry
+// table, 16 packed fp32x2 FMAs for the 4 queries.  The 16 key lanes' sums are
+// merged once per split.
 template <int BV, int NQ>
 __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     const float* __restrict__ logits, const uint32_t* __restrict__ vcodes,
     const float* __restrict__ vxn, int64_t n, int nq, KCodebook vcb, float scale, int split,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_acc) {
     constexpr int WV = BV * kAD / 32;  // record words
+    static_assert(16 * 4 * NQ * 16 * sizeof(float2) <= 2 * kAT * WV * sizeof(uint32_t) || BV < 4,
+                  "the key-lane merge reuses the record buffers");
     __shared__ float s_vc[16];
     __shared__ float2 s_vpair[256];  // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble])
-    __shared__ __align__(16) float s_w[kAT][4];
+    __shared__ __align__(16) float s_w[2][kAT][4];
     __shared__ float s_red[kAT / 32][4];
-    __shared__ float2 s_acc[16][4][NQ][16];  // [key lane][coordinate pair of the word][query][word]
+    // two tiles' value records; after the tile loop, the key lanes' sums
+    // [key lane][coordinate pair of the word][query][word] (float2)
+    constexpr int kBufWords = (2 * kAT * WV > 16 * 4 * NQ * 16 * 2) ? 2 * kAT * WV : 16 * 4 * NQ * 16 * 2;
+    __shared__ __align__(16) uint32_t s_buf[kBufWords];
+    float2 (*s_acc)[4][NQ][16] = reinterpret_cast<float2 (*)[4][NQ][16]>(s_buf);
     const int g = blockIdx.y, sp = blockIdx.x, nsplit = gridDim.x;
     const int q0 = blockIdx.z * NQ;
     const int qn = min(NQ, nq - q0);
@@ -86,8 +106,24 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     const float* lg[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) lg[q] = logits + ((int64_t)g * nq + q0 + (q < qn ? q : 0)) * n;
+    const uint32_t* vg = vcodes + (int64_t)g * n * WV;
+    const float* vxg = vxn + (int64_t)g * n;
+    const bool vec = ((reinterpret_cast<uintptr_t>(vg) & 15u) == 0);
+    // the records of keys [r, r + cnt) into buffer b: 16-byte copies when the
+    // records are 16-byte aligned (every record is 16 b_v bytes), else words
+    auto stage = [&](int64_t r, int cnt, int b) {
+        uint32_t* dst = s_buf + b * (kAT * WV);
+        const uint32_t* src = vg + r * WV;
+        if (vec) {
+            for (int c = t; c < cnt * BV; c += kAT) cp_async16(dst + 4 * c, src + 4 * c);
+            cp_async_commit();
+        } else {
+            for (int c = t; c < cnt * WV; c += kAT) dst[c] = __ldg(src + c);
+        }
+    };
 
-    // ---- the split's maximum per query
+    // ---- the split's maximum per query; the first tile's records in flight
+    stage(r_beg, (int)min((int64_t)kAT, r_end - r_beg), 0);
     float M[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) M[q] = -INFINITY;
@@ -119,62 +155,62 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     float Lp[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) Lp[q] = 0.f;
-    const uint32_t* vg = vcodes + (int64_t)g * n * WV;
-    const float* vxg = vxn + (int64_t)g * n;
-    for (int64_t r = r_beg; r < r_end; r += kAT) {
+    // logits and value norm of key r + t of the next tile to weigh
+    float lnext[NQ], vnext = 0.f;
+    auto load_key = [&](int64_t r, int cnt) {
+        const bool ok = t < cnt;
+        vnext = ok ? vxg[r + t] : 0.f;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) lnext[q] = (ok && q < qn) ? lg[q][r + t] : -INFINITY;
+    };
+    load_key(r_beg, (int)min((int64_t)kAT, r_end - r_beg));
+    int buf = 0;
+    for (int64_t r = r_beg; r < r_end; r += kAT, buf ^= 1) {
         const int cnt = (int)min((int64_t)kAT, r_end - r);
-        // the weights of key r + t
-        {
-            const bool ok = t < cnt;
-            const float vx = ok ? vxg[r + t] : 0.f;
+        {  // the weights of key r + t
             float w4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
-                const float pq = (ok && q < qn) ? __expf(scale * lg[q][r + t] - M[q]) : 0.f;
+                const float pq = lnext[q] == -INFINITY ? 0.f : __expf(scale * lnext[q] - M[q]);
                 Lp[q] += pq;
-                w4[q] = pq * vx;
+                w4[q] = pq * vnext;
             }
-            *reinterpret_cast<float4*>(&s_w[t][0]) = make_float4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<float4*>(&s_w[buf][t][0]) = make_float4(w4[0], w4[1], w4[2], w4[3]);
         }
-        __syncthreads();  // s_w complete
-        // this thread's code word(s) of the tile's keys kl, kl + 16, ..., in two
-        // batches of 8 loads
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-            uint32_t cw[8][BV == 4 ? 1 : BV];
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int key = kl + 16 * (8 * hb + kk);
-                const int64_t v = r + (key < cnt ? key : 0);
+        const int64_t rn = r + kAT;
+        const int cntn = rn < r_end ? (int)min((int64_t)kAT, r_end - rn) : 0;
+        if (cntn > 0) load_key(rn, cntn);
+        if (vec) cp_async_wait_all();
+        __syncthreads();  // this tile's records and weights complete; the other buffers free
+        if (cntn > 0) stage(rn, cntn, buf ^ 1);
+        const uint32_t* rec = s_buf + buf * (kAT * WV);
+#pragma unroll 4
+        for (int kk = 0; kk < 16; ++kk) {
+            const int key = kl + 16 * kk;
+            if (key < cnt) {
+                uint32_t cw[BV == 4 ? 1 : BV];
 #pragma unroll
                 for (int i = 0; i < (BV == 4 ? 1 : BV); ++i)
-                    cw[kk][i] = __ldg(vg + v * WV + (BV == 4 ? wi : (wi >> 2) * BV + i));
-            }
+                    cw[i] = rec[key * WV + (BV == 4 ? wi : (wi >> 2) * BV + i)];
+                const float4 w = *reinterpret_cast<const float4*>(&s_w[buf][key][0]);
+                const float wq[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int key = kl + 16 * (8 * hb + kk);
-                if (key < cnt) {
-                    const float4 w = *reinterpret_cast<const float4*>(&s_w[key][0]);
-                    const float wq[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float2 c2;
-                        if (BV == 4) {  // one code byte = one coordinate pair
-                            c2 = s_vpair[__byte_perm(cw[kk][0], 0u, 0x4440u | e)];
-                        } else {
-                            const int j = 8 * (wi & 3) + 2 * e;
-                            c2 = make_float2(s_vc[value_cell<BV>(cw[kk], j)],
-                                             s_vc[value_cell<BV>(cw[kk], j + 1)]);
-                        }
-#pragma unroll
-                        for (int q = 0; q < NQ; ++q)
-                            acc[e][q] = ffma2(make_float2(wq[q], wq[q]), c2, acc[e][q]);
+                for (int e = 0; e < 4; ++e) {
+                    float2 c2;
+                    if (BV == 4) {  // one code byte = one coordinate pair
+                        c2 = s_vpair[__byte_perm(cw[0], 0u, 0x4440u | e)];
+                    } else {
+                        const int j = 8 * (wi & 3) + 2 * e;
+                        c2 = make_float2(s_vc[value_cell<BV>(cw, j)], s_vc[value_cell<BV>(cw, j + 1)]);
                     }
+#pragma unroll
+                    for (int q = 0; q < NQ; ++q)
+                        acc[e][q] = ffma2(make_float2(wq[q], wq[q]), c2, acc[e][q]);
                 }
             }
         }
-        __syncthreads();  // s_w is rewritten by the next tile
     }
+    __syncthreads();  // every thread is done with the record buffers
     // ---- merge the 16 key lanes; the split's sums per query
 #pragma unroll
     for (int e = 0; e < 4; ++e)
