@@ -32,6 +32,7 @@ using sc::ffma2;
 constexpr int kAD = 128;         // head dimension
 constexpr int kAT = 256;         // keys per tile = threads per block
 constexpr int kAttnSplitMax = 4096;
+constexpr int kPairCopies = 8;   // copies of the byte-pair centroid table (b_v = 4)
 
 // Value cell of coordinate j (0..31) of a block of the MSE-only layout (the
 // index's top bit sits in the z position): the b-bit Lloyd-Max cell.
@@ -77,7 +78,10 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     static_assert(16 * 4 * NQ * 16 * sizeof(float2) <= 2 * kAT * WV * sizeof(uint32_t) || BV < 4,
                   "the key-lane merge reuses the record buffers");
     __shared__ float s_vc[16];
-    __shared__ float2 s_vpair[256];  // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble])
+    // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble]), kPairCopies
+    // copies side by side (dynamic shared memory); lane l reads copy l % 8,
+    // so lanes of different copies never share a bank
+    extern __shared__ float2 s_vpair[];
     __shared__ __align__(16) float s_w[2][kAT][4];
     __shared__ float s_red[kAT / 32][4];
     // two tiles' value records; after the tile loop, the key lanes' sums
@@ -100,7 +104,12 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
         s_vc[t] = c;
     }
     __syncthreads();
-    if (BV == 4) s_vpair[t] = make_float2(s_vc[t & 15], s_vc[t >> 4]);
+    if (BV == 4) {
+        const float2 pv = make_float2(s_vc[t & 15], s_vc[t >> 4]);
+#pragma unroll
+        for (int r = 0; r < kPairCopies; ++r) s_vpair[t * kPairCopies + r] = pv;
+    }
+    const int pcopy = lane % kPairCopies;
     const int64_t r_beg = (int64_t)sp * split;
     const int64_t r_end = min(n, r_beg + split);
     const float* lg[NQ];
@@ -198,7 +207,7 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
                 for (int e = 0; e < 4; ++e) {
                     float2 c2;
                     if (BV == 4) {  // one code byte = one coordinate pair
-                        c2 = s_vpair[__byte_perm(cw[0], 0u, 0x4440u | e)];
+                        c2 = s_vpair[__byte_perm(cw[0], 0u, 0x4440u | e) * kPairCopies + pcopy];
                     } else {
                         const int j = 8 * (wi & 3) + 2 * e;
                         c2 = make_float2(s_vc[value_cell<BV>(cw, j)], s_vc[value_cell<BV>(cw, j + 1)]);
@@ -280,8 +289,12 @@ template <int BV, int NQ>
 int launch_partial(dim3 grid, const float* logits, const uint32_t* vc, const float* vx, int64_t n,
                    int nq, const KCodebook& vcb, float scale, int split, float* pm, float* pl,
                    float* pa, cudaStream_t s) {
-    k_attn_partial<BV, NQ><<<grid, kAT, 0, s>>>(logits, vc, vx, n, nq, vcb, scale, split, pm, pl,
-                                               pa);
+    const int dyn = BV == 4 ? 256 * kPairCopies * (int)sizeof(float2) : 0;
+    if (dyn > 0)
+        TQ_TRY_CUDA(cudaFuncSetAttribute(k_attn_partial<BV, NQ>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, dyn));
+    k_attn_partial<BV, NQ><<<grid, kAT, dyn, s>>>(logits, vc, vx, n, nq, vcb, scale, split, pm, pl,
+                                                 pa);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
