@@ -669,6 +669,13 @@ __global__ __launch_bounds__(512) void k_query_prep(const float* __restrict__ Pi
     extern __shared__ __align__(16) float sq[];  // [0, d): q   [d, 2d): qr
     constexpr int R = 8;  // rows per warp in flight
     const int g = blockIdx.y;
+    // S of the group toward L2 while Pi q is formed (the second product then
+    // reads it from L2), by one block of the group, for d <= 256
+    if (S && blockIdx.x == 0 && d <= 256) {
+        const char* sg = reinterpret_cast<const char*>(S + (size_t)g * d * d);
+        for (int e = threadIdx.x; e * 128 < d * d * 4; e += blockDim.x)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(sg + (size_t)e * 128));
+    }
     const int64_t row = (int64_t)g * nq + blockIdx.x;
     for (int j = threadIdx.x; j < d; j += blockDim.x) sq[j] = load_f32(q, row * d + j);
     __syncthreads();
