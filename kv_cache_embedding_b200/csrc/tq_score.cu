@@ -300,6 +300,19 @@ __global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict
     const int lane = threadIdx.x % 32;
     const float* sr = scores + row * n;
     const float* cm = cmax + row * nchunks;
+    const int64_t per = (n + P - 1) / P;
+    const int64_t e0 = (int64_t)blockIdx.x * per;
+    const int64_t e1 = min(n, e0 + per);
+    constexpr int U = 16;
+    float v[U];
+    auto load = [&](int64_t base) {
+#pragma unroll
+        for (int j = 0; j < U; ++j) {
+            const int64_t e = base + (int64_t)j * blockDim.x + threadIdx.x;
+            v[j] = e < e1 ? sr[e] : -INFINITY;
+        }
+    };
+    load(e0);  // the first pass's scores are in flight while the threshold is formed
     float f[2] = {-INFINITY, -INFINITY};
     for (int c = lane; c < nchunks; c += 64) {
         f[0] = fmaxf(f[0], cm[c]);
@@ -308,19 +321,10 @@ __global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict
     warp_sort64_desc(f, lane);
     // the K-th largest slot (-inf when fewer than K chunks)
     const float thr = __shfl_sync(0xffffffffu, ((K - 1) & 1) ? f[1] : f[0], (K - 1) >> 1);
-    const int64_t per = (n + P - 1) / P;
-    const int64_t e0 = (int64_t)blockIdx.x * per;
-    const int64_t e1 = min(n, e0 + per);
     float* cv = cand_v + row * kCandCapG;
     int* ci = cand_i + row * kCandCapG;
-    constexpr int U = 16;
     for (int64_t base = e0; base < e1; base += (int64_t)U * blockDim.x) {
-        float v[U];
-#pragma unroll
-        for (int j = 0; j < U; ++j) {
-            const int64_t e = base + (int64_t)j * blockDim.x + threadIdx.x;
-            v[j] = e < e1 ? sr[e] : -INFINITY;
-        }
+        if (base != e0) load(base);
 #pragma unroll
         for (int j = 0; j < U; ++j) {
             const int64_t e = base + (int64_t)j * blockDim.x + threadIdx.x;
