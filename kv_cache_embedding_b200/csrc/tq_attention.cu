@@ -258,31 +258,86 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
 
 // Merge the splits of one (group, query) row and rotate back:
 //   a = sum_s e^{m_s - M} acc_s / sum_s e^{m_s - M} l_s,   out = Pi_v^T a.
-__global__ __launch_bounds__(kAD) void k_attn_combine(const float* __restrict__ part_m,
-                                                      const float* __restrict__ part_l,
-                                                      const float* __restrict__ part_acc,
-                                                      int nsplit, int nq,
-                                                      const float* __restrict__ Pi_v,
-                                                      float* __restrict__ out) {
+// 256 threads: the split weights e^{m_s - M} go through shared memory in
+// chunks of kCombChunk splits; warp w sums splits s = w mod 8 of a chunk for
+// the 4 coordinates 4 lane .. 4 lane + 3 (float4 loads), the 8 warps' sums
+// are added in shared memory, and the two halves of the block each apply
+// half of the rows of Pi_v.
+constexpr int kCombThreads = 256;
+constexpr int kCombChunk = 1024;
+__global__ __launch_bounds__(kCombThreads) void k_attn_combine(const float* __restrict__ part_m,
+                                                               const float* __restrict__ part_l,
+                                                               const float* __restrict__ part_acc,
+                                                               int nsplit, int nq,
+                                                               const float* __restrict__ Pi_v,
+                                                               float* __restrict__ out) {
+    __shared__ float s_e[kCombChunk];
+    __shared__ float s_red[kCombThreads / 32];
+    __shared__ __align__(16) float s_part[kCombThreads / 32][kAD];
     __shared__ float s_a[kAD];
-    const int q = blockIdx.x, g = blockIdx.y, k = threadIdx.x;
+    __shared__ float s_o[2][kAD];
+    const int q = blockIdx.x, g = blockIdx.y, t = threadIdx.x, lane = t % 32, w = t / 32;
+    constexpr int NW = kCombThreads / 32;
     const int64_t row = (int64_t)g * nq + q;
     const float* pm = part_m + row * nsplit;
     const float* pl = part_l + row * nsplit;
+    const float* pa = part_acc + row * nsplit * kAD;
+    // M = max_s m_s
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pm[s]);
-    float L = 0.f, a = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-        const float e = __expf(pm[s] - M);
-        L = fmaf(e, pl[s], L);
-        a = fmaf(e, part_acc[(row * nsplit + s) * kAD + k], a);
-    }
-    s_a[k] = a / L;
+    for (int s = t; s < nsplit; s += kCombThreads) M = fmaxf(M, pm[s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_red[w] = M;
     __syncthreads();
+    M = s_red[0];
+#pragma unroll
+    for (int i = 1; i < NW; ++i) M = fmaxf(M, s_red[i]);
+    __syncthreads();  // s_red is reused for L
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < nsplit; c0 += kCombChunk) {
+        const int cn = min(kCombChunk, nsplit - c0);
+        for (int s = t; s < cn; s += kCombThreads) {
+            const float e = __expf(pm[c0 + s] - M);
+            s_e[s] = e;
+            L = fmaf(e, pl[c0 + s], L);
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int s = w; s < cn; s += NW) {
+            const float e = s_e[s];
+            const float4 v = reinterpret_cast<const float4*>(pa + (int64_t)(c0 + s) * kAD)[lane];
+            acc.x = fmaf(e, v.x, acc.x);
+            acc.y = fmaf(e, v.y, acc.y);
+            acc.z = fmaf(e, v.z, acc.z);
+            acc.w = fmaf(e, v.w, acc.w);
+        }
+        __syncthreads();  // s_e is rewritten by the next chunk
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) s_red[w] = L;
+    reinterpret_cast<float4*>(s_part[w])[lane] = acc;
+    __syncthreads();
+    if (t < kAD) {
+        float a = 0.f, Ls = 0.f;
+#pragma unroll
+        for (int i = 0; i < NW; ++i) {
+            a += s_part[i][t];
+            Ls += s_red[i];
+        }
+        s_a[t] = a / Ls;
+    }
+    __syncthreads();
+    // out = Pi_v^T a: thread (half h, coordinate k) sums rows j of its half
+    const int k = t % kAD, h = t / kAD;
     const float* P = Pi_v + (size_t)g * kAD * kAD;
     float o = 0.f;
-    for (int j = 0; j < kAD; ++j) o = fmaf(P[(size_t)j * kAD + k], s_a[j], o);
-    out[row * kAD + k] = o;
+#pragma unroll 8
+    for (int j = h * (kAD / 2); j < (h + 1) * (kAD / 2); ++j) o = fmaf(P[(size_t)j * kAD + k], s_a[j], o);
+    s_o[h][k] = o;
+    __syncthreads();
+    if (t < kAD) out[row * kAD + t] = s_o[0][t] + s_o[1][t];
 }
 
 template <int BV, int NQ>
@@ -380,8 +435,8 @@ extern "C" int tq_attention_decode(const tq_codebook_t* cb_k, const float* d_Pi_
         default: rc = launch_partial_nq<4>(grid, NQ, logits, d_vcodes, d_vxnorm, n, nq, vcb, scale, (int)split, pm, pl, pa, s); break;
     }
     if (rc) return rc;
-    k_attn_combine<<<dim3((unsigned)nq, (unsigned)G), kAD, 0, s>>>(pm, pl, pa, (int)nsplit, nq,
-                                                                    d_Pi_v, d_out);
+    k_attn_combine<<<dim3((unsigned)nq, (unsigned)G), kCombThreads, 0, s>>>(pm, pl, pa, (int)nsplit,
+                                                                            nq, d_Pi_v, d_out);
     TQ_CHECK_LAUNCH();
     return TQ_OK;
 }
