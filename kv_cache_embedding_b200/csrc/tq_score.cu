@@ -313,14 +313,31 @@ __global__ __launch_bounds__(256, 4) void k_topk_collect(const float* __restrict
         }
     };
     load(e0);  // the first pass's scores are in flight while the threshold is formed
-    float f[2] = {-INFINITY, -INFINITY};
-    for (int c = lane; c < nchunks; c += 64) {
-        f[0] = fmaxf(f[0], cm[c]);
-        if (c + 32 < nchunks) f[1] = fmaxf(f[1], cm[c + 32]);
+    // slot s (0..63) = the maximum of the chunk maxima c = s (mod 64): the
+    // block's 256 threads read the chunk maxima once (4 threads per slot),
+    // warp 0 sorts the 64 slots and the K-th largest is the threshold
+    __shared__ float s_slot[4][64];
+    __shared__ float s_thr;
+    {
+        const int sl = threadIdx.x & 63, part = threadIdx.x >> 6;
+        float m = -INFINITY;
+#pragma unroll 4
+        for (int c = sl + 64 * part; c < nchunks; c += 256) m = fmaxf(m, cm[c]);
+        s_slot[part][sl] = m;
     }
-    warp_sort64_desc(f, lane);
-    // the K-th largest slot (-inf when fewer than K chunks)
-    const float thr = __shfl_sync(0xffffffffu, ((K - 1) & 1) ? f[1] : f[0], (K - 1) >> 1);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float f[2];
+        f[0] = fmaxf(fmaxf(s_slot[0][lane], s_slot[1][lane]), fmaxf(s_slot[2][lane], s_slot[3][lane]));
+        f[1] = fmaxf(fmaxf(s_slot[0][lane + 32], s_slot[1][lane + 32]),
+                     fmaxf(s_slot[2][lane + 32], s_slot[3][lane + 32]));
+        warp_sort64_desc(f, lane);
+        // the K-th largest slot (-inf when fewer than K chunks)
+        const float t = __shfl_sync(0xffffffffu, ((K - 1) & 1) ? f[1] : f[0], (K - 1) >> 1);
+        if (lane == 0) s_thr = t;
+    }
+    __syncthreads();
+    const float thr = s_thr;
     float* cv = cand_v + row * kCandCapG;
     int* ci = cand_i + row * kCandCapG;
     for (int64_t base = e0; base < e1; base += (int64_t)U * blockDim.x) {
