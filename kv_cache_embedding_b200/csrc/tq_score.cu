@@ -840,6 +840,22 @@ extern "C" int tq_score(const tq_codebook_t* cb, const float* d_Pi, const float*
 }
 
 namespace tq {
+// Blocks per score row of k_topk_collect: 16 scores per thread (one pass of
+// loads), at least enough blocks for every SM; when that would take more than
+// one wave of resident blocks (4 per SM), as many as one wave holds, each
+// thread then taking several passes (the per-block threshold and the
+// last-block selection are latency chains, paid once per wave).
+int64_t collect_blocks_per_row(int64_t n, int64_t rows, int nsm) {
+    int64_t P = (n + 256 * 16 - 1) / (256 * 16);
+    const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
+    const int64_t pmax = (n + 255) / 256;
+    const int64_t wave = 4 * (int64_t)nsm / rows;
+    if (rows * P > 4 * (int64_t)nsm) P = wave;
+    P = P < pmin ? pmin : P;
+    P = P > pmax ? pmax : P;
+    return P < 1 ? 1 : P;
+}
+
 int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G, int64_t n,
              const uint32_t* d_codes, const float* d_xnorm, const float* d_rnorm, int nq,
              const void* d_q, int q_dtype, int k, float* d_vals, int64_t* d_ids, void* d_ws,
@@ -908,12 +924,7 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
         TQ_TRY_CUDA(cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev));
         // blocks per row: 16 scores per thread (one pass of loads), more when
         // the rows alone would leave most SMs idle
-        int64_t P = (n + 256 * 16 - 1) / (256 * 16);
-        const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
-        const int64_t pmax = (n + 255) / 256;
-        P = P < pmin ? pmin : P;
-        P = P > pmax ? pmax : P;
-        dim3 grid((unsigned)P, (unsigned)rows);
+        dim3 grid((unsigned)collect_blocks_per_row(n, rows, nsm), (unsigned)rows);
         k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, n, nchunks, k, cnt, cnt + rows, cv, ci, d_vals,
                                             d_ids, 0);
         TQ_CHECK_LAUNCH();
@@ -961,12 +972,7 @@ int topk_run(const tq_codebook_t* cb, const float* d_Pi, const float* d_S, int G
                 rc = launch_score_i8(cb, G, len, d_codes, d_xnorm, d_rnorm, nq, qr, u, sc, cm, cnt,
                                      err, s, n, k0);
                 if (rc) return rc;
-                int64_t P = (len + 256 * 16 - 1) / (256 * 16);
-                const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
-                const int64_t pmax = (len + 255) / 256;
-                P = P < pmin ? pmin : P;
-                P = P > pmax ? pmax : P;
-                dim3 grid((unsigned)P, (unsigned)rows);
+                dim3 grid((unsigned)collect_blocks_per_row(len, rows, nsm), (unsigned)rows);
                 k_topk_collect<<<grid, 256, 0, s>>>(sc, cm, len, (int)((len + 127) / 128), k, cnt,
                                                     cnt + rows, cv, ci, pv + h * rows * k,
                                                     pi + h * rows * k, k0);
