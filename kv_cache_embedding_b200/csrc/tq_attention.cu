@@ -75,8 +75,6 @@ __global__ __launch_bounds__(kAT, 3) void k_attn_partial(
     const float* __restrict__ vxn, int64_t n, int nq, KCodebook vcb, float scale, int split,
     float* __restrict__ part_m, float* __restrict__ part_l, float* __restrict__ part_acc) {
     constexpr int WV = BV * kAD / 32;  // record words
-    static_assert(16 * 4 * NQ * 16 * sizeof(float2) <= 2 * kAT * WV * sizeof(uint32_t) || BV < 4,
-                  "the key-lane merge reuses the record buffers");
     __shared__ float s_vc[16];
     // b_v = 4: code byte -> (c_v[low nibble], c_v[high nibble]), kPairCopies
     // copies side by side (dynamic shared memory); lane l reads copy l % 8,
