@@ -845,7 +845,7 @@ namespace tq {
 // one wave of resident blocks (4 per SM), as many as one wave holds, each
 // thread then taking several passes (the per-block threshold and the
 // last-block selection are latency chains, paid once per wave).
-int64_t collect_blocks_per_row(int64_t n, int64_t rows, int nsm) {
+static int64_t collect_blocks_per_row(int64_t n, int64_t rows, int nsm) {
     int64_t P = (n + 256 * 16 - 1) / (256 * 16);
     const int64_t pmin = ((int64_t)nsm + rows - 1) / rows;
     const int64_t pmax = (n + 255) / 256;
